@@ -1,0 +1,128 @@
+"""Plant plausible mistakes in the oracle (CPU only) and check that the pins catch them.
+
+Each mutant replaces one oracle function with a subtly wrong copy (a dropped term,
+a wrong sign, a transposed operand, a non-strict comparison, a wrong tie-break);
+the test passes only if at least one pin then fails.
+"""
+import numpy as np
+import pytest
+
+import oracle.attention as OA
+import oracle.flashblock as OF
+import oracle.sparse as OS
+
+from tests import test_oracle_attention as TA
+from tests import test_oracle_flashblock as TF
+from tests import test_oracle_sparse as TS
+
+_orig_attend = OA.attend
+_orig_merge = OA.merge
+
+
+def _merge_den_drop(a1, l1, a2, l2):
+    m = np.maximum(l1, l2)
+    w1, w2 = np.exp(l1 - m), np.exp(l2 - m)
+    return (w1[..., None] * a1 + w2[..., None] * a2) / np.maximum(w1, 1e-300)[..., None], m + np.log(w1 + w2)
+
+
+def _merge_L_drop(a1, l1, a2, l2):
+    A, L = _orig_merge(a1, l1, a2, l2)
+    m = np.maximum(l1, l2)
+    return A, np.where(np.isneginf(m), m, m)
+
+
+def _merge_sign(a1, l1, a2, l2):
+    m = np.maximum(l1, l2)
+    w1, w2 = np.exp(m - l1), np.exp(m - l2)
+    return (w1[..., None] * a1 + w2[..., None] * a2) / (w1 + w2)[..., None], m + np.log(w1 + w2)
+
+
+def _attend_no_scale(q, k, v, scale):
+    return _orig_attend(q, k, v, 1.0)
+
+
+def _attend_kv_swapped(q, k, v, scale):
+    if k.shape == v.shape:
+        return _orig_attend(q, k, k, scale)
+    return _orig_attend(q, k, v, scale)
+
+
+def _attend_L_no_max(q, k, v, scale):
+    A, L = _orig_attend(q, k, v, scale)
+    if k.shape[0] == 0:
+        return A, L
+    s = scale * (np.asarray(q) @ np.asarray(k).T)
+    return A, np.log(np.exp(s - s.max(1, keepdims=True)).sum(1))
+
+
+def _tau_le(M, tau, first_step):
+    return np.zeros(M.shape, bool) if first_step else M <= tau
+
+
+def _gamma_ge(sim, gamma, first_step, shape):
+    if first_step:
+        return np.zeros(shape, bool)
+    if sim is None:
+        return np.ones(shape, bool)
+    return np.asarray(sim, np.float32) >= np.float32(gamma)
+
+
+def _est_min(q_rows, kmin, kmax):
+    q_rows = np.asarray(q_rows, np.float64)
+    est = np.zeros((q_rows.shape[0], kmin.shape[0]))
+    for d in range(q_rows.shape[1]):
+        qd = q_rows[:, d:d + 1]
+        est = est + np.minimum(qd * kmin[None, :, d], qd * kmax[None, :, d])
+    return est
+
+
+def _select_high_tie(est, k_sel):
+    out = np.zeros((est.shape[0], k_sel), dtype=np.int64)
+    for r in range(est.shape[0]):
+        order = sorted(range(est.shape[1]), key=lambda p: (-est[r, p], -p))
+        out[r] = np.sort(order[:k_sel])
+    return out
+
+
+PINS_ATTN = [
+    lambda: TA.test_attend_matches_torch_sdpa_and_logsumexp(3, 7, 16, 0.25),
+    lambda: TA.test_golden_attention_cases(),
+    lambda: TA.test_golden_merge_cases(),
+    lambda: TA.test_merge_of_partition_equals_dense_over_union(0),
+]
+PINS_GATE = [lambda: TF.test_golden_gate_cases()]
+PINS_SPARSE = [lambda: TS.test_page_estimate_bounds_every_score_in_page(),
+               lambda: TS.test_select_pages_matches_full_lexsort(0),
+               lambda: TS.test_select_ties_prefer_lower_page()]
+
+MUTANTS = [
+    ("merge: denominator drops w_in", [(OA, "merge"), (OF, "merge"), (OS, "merge")], _merge_den_drop, PINS_ATTN),
+    ("merge: L drops ln(w1+w2)", [(OA, "merge"), (OF, "merge"), (OS, "merge")], _merge_L_drop, PINS_ATTN),
+    ("merge: exponent sign flipped", [(OA, "merge"), (OF, "merge"), (OS, "merge")], _merge_sign, PINS_ATTN),
+    ("attend: softmax scale dropped", [(OA, "attend"), (OF, "attend"), (OS, "attend")], _attend_no_scale, PINS_ATTN),
+    ("attend: K used in place of V", [(OA, "attend"), (OF, "attend"), (OS, "attend")], _attend_kv_swapped, PINS_ATTN),
+    ("attend: L drops the max term", [(OA, "attend"), (OF, "attend"), (OS, "attend")], _attend_L_no_max, PINS_ATTN),
+    ("tau gate: <= instead of <", [(OF, "tau_reuse")], _tau_le, PINS_GATE),
+    ("gamma gate: >= instead of >", [(OF, "gamma_reuse")], _gamma_ge, PINS_GATE),
+    ("page bound: min instead of max", [(OS, "page_estimates")], _est_min, PINS_SPARSE),
+    ("top-k: ties to the higher page", [(OS, "select_pages")], _select_high_tie, PINS_SPARSE),
+]
+
+
+@pytest.mark.parametrize("name,targets,mutant,pins", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(monkeypatch, name, targets, mutant, pins):
+    for mod, attr in targets:
+        if hasattr(mod, attr):
+            monkeypatch.setattr(mod, attr, mutant)
+    caught = 0
+    for pin in pins:
+        try:
+            pin()
+        except AssertionError:
+            caught += 1
+    assert caught >= 1, f"no pin caught the planted mistake: {name}"
+
+
+def test_pins_pass_on_unmutated_oracle():
+    for pin in PINS_ATTN + PINS_GATE + PINS_SPARSE:
+        pin()
