@@ -1,0 +1,446 @@
+"""Benchmark of cached block-diffusion attention (FlashBlock) on B200.
+
+One step = one denoising step of one attention layer: the reuse gate, the
+prefix (out-of-block) pass when the gate says recompute, the in-block pass and
+the log-space merge -- the two C-ABI calls fb_prefix_attn(gate) and
+fb_block_merge that make up fb_step.  Steps follow the seeded schedule of the
+workload (16 steps per block for the dLM-like layer; step 0 of each block
+recomputes), so the reported rate mixes recompute and reuse steps as the
+method does.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints one JSON line (rank 0).  Under torchrun every rank runs its own replica
+of the workload (weak scaling, no collective on the data path); the timed
+region is bracketed by a barrier and a device synchronise and the slowest
+rank's time is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from block_diffusion_attention_prefix_b200 import workloads as W  # noqa: E402
+
+METRIC = "block-attention steps/sec and achieved HBM GB/s (% of B200 peak) vs context length"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return float(p["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_diffusion_attention_prefix_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per launch of the prefix kernel from the committed ncu summary,
+    or None when the summary is absent or was taken on other kernel sources."""
+    path = os.path.join(ROOT, "profiles", f"prefix_pass_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: record that no clocks were sampled
+            self._nv = None
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((mhz, reasons))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "source": "nvml unavailable" if self._nv is None else "nvml"}
+        mhz = [m for m, _ in self.samples]
+        seen = set()
+        for _, r in self.samples:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    seen.add(name)
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz, "reasons": sorted(seen),
+                "samples": len(mhz), "source": "nvml"}
+
+
+# ----------------------------------------------------------------------------- device arm
+
+
+class DeviceWorkload:
+    """The workload's inputs resident in HBM and the layer state, stepped through libfb."""
+
+    def __init__(self, fb, w: W.Workload, seed: int):
+        self.fb, self.w = fb, w
+        dev = torch.device("cuda")
+        k, v = W.prefix_kv(w, seed)
+        self.k, self.v = k.to(dev), v.to(dev)
+        del k, v
+        self.sched = []
+        for s in W.block_schedule(w, seed):
+            self.sched.append(dict(
+                q=s.q.to(dev), k_blk=s.k_blk.to(dev), v_blk=s.v_blk.to(dev), mask=s.mask.to(dev),
+                sim=None if s.sim is None else s.sim.to(dev), first=s.first,
+                host=s))
+        self.shape = fb.make_shape(w.batch, w.h_q, w.h_kv, w.head_dim, w.block, w.n_prefix, w.dtype)
+        f32 = dict(device=dev, dtype=torch.float32)
+        self.a_out = torch.zeros((w.batch, w.h_q, w.block, w.head_dim), **f32)
+        self.l_out = torch.full((w.batch, w.h_q, w.block), float("-inf"), **f32)
+        self.a_full = torch.zeros((w.batch, w.h_q, w.block, w.head_dim), device=dev, dtype=w.torch_dtype)
+        self.l_full = torch.zeros((w.batch, w.h_q, w.block), **f32)
+        n = fb.fb_workspace_bytes(self.shape)
+        self.ws = torch.zeros(((n + 15) // 16 * 16,), device=dev, dtype=torch.uint8)
+        self.gates = [fb.make_gate(s["mask"], s["first"], w.tau, s["sim"], w.gamma or 0.0) for s in self.sched]
+
+    def launches_per_step(self) -> int:
+        big = self.w.block > 64
+        return 2 + (1 if big else 0)
+
+    def run_step(self, i: int, dec_M, dec_reuse, ev=None, tau_override=None):
+        fb, s = self.fb, self.sched[i % len(self.sched)]
+        g = self.gates[i % len(self.sched)]
+        if tau_override is not None:
+            g = fb.make_gate(s["mask"], s["first"], tau_override, s["sim"], self.w.gamma or 0.0)
+        if ev is not None:
+            ev[0].record()
+        fb.fb_prefix_attn(self.shape, s["q"], self.k, self.v, g, self.a_out, self.l_out, self.ws)
+        if ev is not None:
+            ev[1].record()
+        fb.fb_block_merge(self.shape, s["q"], s["k_blk"], s["v_blk"], g, self.a_out, self.l_out, self.a_full,
+                          self.l_full, dec_M, dec_reuse, self.ws)
+        if ev is not None:
+            ev[2].record()
+
+    def prefix_algorithmic_bytes(self) -> int:
+        """Bytes a recompute launch of the prefix pass must move: prefix K and V,
+        the block queries, and the cache rows it writes (A_out fp32, L_out fp32)."""
+        w = self.w
+        q = w.batch * w.h_q * w.block * w.head_dim * w.elem_bytes
+        cache = w.batch * w.h_q * w.block * (w.head_dim + 1) * 4
+        return w.prefix_bytes() + q + cache
+
+
+def device_arm(args, rank, world):
+    from block_diffusion_attention_prefix_b200 import fb
+    fb.load()
+    w = W.get(args.workload)
+    dw = DeviceWorkload(fb, w, seed=args.seed + rank)
+    K, Wm = args.steps, args.warmup
+    dev = torch.device("cuda")
+    flush = torch.empty((L2_FLUSH_BYTES,), device=dev, dtype=torch.uint8)
+    dec_M = torch.zeros((K, w.batch), device=dev, dtype=torch.int32)
+    dec_R = torch.zeros((K, w.batch, w.h_q), device=dev, dtype=torch.uint8)
+    wdM = torch.zeros((w.batch,), device=dev, dtype=torch.int32)
+    wdR = torch.zeros((w.batch, w.h_q), device=dev, dtype=torch.uint8)
+    fb.fb_workspace_init(dw.ws)
+    # warm-up: whole blocks from step 0 so the cache is valid
+    for i in range(Wm):
+        flush.zero_()
+        dw.run_step(i, wdM, wdR)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start = Wm  # continue the schedule where warm-up stopped
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        t0 = time.perf_counter()
+        for i in range(K):
+            flush.zero_()                      # L2 flush between timed steps (outside the events)
+            dw.run_step(start + i, dec_M[i], dec_R[i], evs[i])
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - t0
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
+    prefix_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    reuse = dec_R.cpu().numpy().astype(bool)            # [K, b, H_q]
+    recompute_steps = [i for i in range(K) if not reuse[i].all()]
+    reuse_steps = [i for i in range(K) if reuse[i].all()]
+    total_ms = sum(step_ms)
+    t_max = total_ms
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_max = float(t.item())
+    value = world * K / (t_max / 1e3)
+    hbm, peak_kind = peaks()
+    alg = dw.prefix_algorithmic_bytes()
+    rec_ms = [prefix_ms[i] for i in recompute_steps]
+    achieved = (alg * len(rec_ms)) / (sum(rec_ms) / 1e3) / 1e9 if rec_ms else None
+    traffic = ncu_traffic(args.workload)
+
+    # dense-recompute reference (standard block diffusion): gate forced to recompute
+    dense_ms = []
+    if args.dense_steps > 0:
+        evd = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.dense_steps)]
+        for i in range(args.dense_steps):
+            flush.zero_()
+            dw.run_step(i, wdM, wdR, evd[i], tau_override=0)
+        torch.cuda.synchronize()
+        dense_ms = [e[0].elapsed_time(e[2]) for e in evd]
+
+    e2e = e2e_arm(fb, dw, K, Wm) if args.e2e else None
+    res = dict(
+        metric=METRIC, value=value, unit="steps/s", n_gpus=world, steps=K, warmup=Wm,
+        ms_per_step=t_max / K, higher_is_better=True, scaling="weak", vs_baseline=None,
+        dtype=w.dtype, data="synthetic",
+        config=dict(workload=w.name, description=w.description, batch=w.batch, h_q=w.h_q, h_kv=w.h_kv,
+                    head_dim=w.head_dim, block=w.block, n_prefix=w.n_prefix, steps_per_block=w.steps,
+                    tau=w.tau, gamma=w.gamma, seed=args.seed,
+                    l2="flushed between timed steps (256 MiB write, outside the step events)",
+                    parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        roofline=dict(bound="hbm", kernel="pass_bf16_kernel (prefix split-KV pass)" if w.dtype == "bf16"
+                      else "pass_f32_kernel (prefix split-KV pass)",
+                      achieved=achieved, peak=hbm, unit="GB/s",
+                      frac=(achieved / hbm) if achieved else None,
+                      peak_source=f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                      frac_of_8tbs=(achieved / 8000.0) if achieved else None,
+                      alg_bytes_per_launch=alg, launches=len(rec_ms),
+                      avg_launch_us=(sum(rec_ms) / len(rec_ms) * 1e3) if rec_ms else None,
+                      traffic=traffic),
+        breakdown=dict(recompute_steps=len(recompute_steps), reuse_steps=len(reuse_steps),
+                       recompute_step_us=_mean_us(step_ms, recompute_steps),
+                       reuse_step_us=_mean_us(step_ms, reuse_steps),
+                       dense_recompute_step_us=(statistics.mean(dense_ms) * 1e3) if dense_ms else None,
+                       dense_steps_per_s=(1e3 / statistics.mean(dense_ms)) if dense_ms else None,
+                       wall_s=wall),
+        gpu_launches=dw.launches_per_step() * K,
+        clocks=clocks.summary(),
+        kernel_source_sha=kernel_source_hash(),
+    )
+    if e2e:
+        res["e2e"] = e2e
+    return res
+
+
+def _mean_us(ms, idx):
+    return statistics.mean(ms[i] for i in idx) * 1e3 if idx else None
+
+
+def e2e_arm(fb, dw, K, Wm):
+    """Same metric through fb_step with the step's inputs in pinned host memory:
+    every step copies its inputs host->device, runs fb_step and reads A_full and
+    the decisions back to the host."""
+    w = dw.w
+    hosts = []
+    for s in dw.sched:
+        h = s["host"]
+        hosts.append(dict(q=h.q.pin_memory(), k_blk=h.k_blk.pin_memory(), v_blk=h.v_blk.pin_memory(),
+                          mask=h.mask.pin_memory(), sim=None if h.sim is None else h.sim.pin_memory(),
+                          first=h.first))
+    dev = torch.device("cuda")
+    d_in = dict(q=torch.empty_like(dw.sched[0]["q"]), k_blk=torch.empty_like(dw.sched[0]["k_blk"]),
+                v_blk=torch.empty_like(dw.sched[0]["v_blk"]), mask=torch.empty_like(dw.sched[0]["mask"]),
+                sim=None if dw.sched[0]["sim"] is None else torch.empty_like(dw.sched[0]["sim"]))
+    dM = torch.zeros((w.batch,), device=dev, dtype=torch.int32)
+    dR = torch.zeros((w.batch, w.h_q), device=dev, dtype=torch.uint8)
+    out_a = torch.empty(dw.a_full.shape, dtype=dw.a_full.dtype).pin_memory()
+    out_M = torch.empty((w.batch,), dtype=torch.int32).pin_memory()
+    out_R = torch.empty((w.batch, w.h_q), dtype=torch.uint8).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for k, t in hosts[0].items() if isinstance(t, torch.Tensor))
+    d2h = out_a.numel() * out_a.element_size() + out_M.numel() * 4 + out_R.numel()
+
+    def one(i):
+        h = hosts[i % len(hosts)]
+        for key in ("q", "k_blk", "v_blk", "mask", "sim"):
+            if h[key] is not None:
+                d_in[key].copy_(h[key], non_blocking=True)
+        g = fb.make_gate(d_in["mask"], h["first"], w.tau, d_in["sim"], w.gamma or 0.0)
+        fb.fb_step(dw.shape, d_in["q"], dw.k, dw.v, d_in["k_blk"], d_in["v_blk"], g, dw.a_out, dw.l_out,
+                   dw.a_full, dw.l_full, dM, dR, dw.ws)
+        out_a.copy_(dw.a_full, non_blocking=True)
+        out_M.copy_(dM, non_blocking=True)
+        out_R.copy_(dR, non_blocking=True)
+        torch.cuda.current_stream().synchronize()   # the result is on the host
+
+    for i in range(Wm):
+        one(i)
+    t0 = time.perf_counter()
+    for i in range(K):
+        one(Wm + i)
+    el = time.perf_counter() - t0
+    return dict(value=K / el, unit="steps/s", h2d_bytes_per_step=h2d, d2h_bytes_per_step=d2h,
+                note="wall clock per step incl. pinned H2D of the step inputs, fb_step, D2H of A_full + "
+                     "decisions and a host sync; prefix KV cache resident in HBM")
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_steps(w: W.Workload, seed: int, budget_s: float, max_steps: int, kv_groups: int):
+    """Time the CPU oracle's cached step on the workload, restricted to the first
+    `kv_groups` KV-head groups (a bounded sample).  Returns (steps, seconds,
+    scale) where scale converts the sample's time to a whole-layer step."""
+    import numpy as np
+    from oracle import flashblock as OF
+    k, v = W.prefix_kv(w, seed)
+    hk = min(kv_groups, w.h_kv)
+    hq = hk * w.group
+    kk = k[:, :hk].double().numpy()
+    vv = v[:, :hk].double().numpy()
+    del k, v
+    st = OF.CachedBlockAttention(kk, vv, hq, 1 / math.sqrt(w.head_dim))
+    sched = list(W.block_schedule(w, seed))
+    conv = [(s.q[:, :hq].double().numpy(), s.k_blk[:, :hk].double().numpy(), s.v_blk[:, :hk].double().numpy(),
+             s.mask.numpy(), s.first, None if s.sim is None else s.sim[:, :hq].numpy()) for s in sched]
+    n, el = 0, 0.0
+    while n < max_steps and (el < budget_s or n < 1):
+        q, kb, vb, mask, first, sim = conv[n % len(conv)]
+        t0 = time.perf_counter()
+        st.step(q, kb, vb, mask, first, w.tau, sim, w.gamma or 0.0)
+        el += time.perf_counter() - t0
+        n += 1
+    return n, el, w.h_kv / hk
+
+
+def cpu_baseline(w, seed, budget_s=12.0):
+    n, el, scale = oracle_steps(w, seed, budget_s, 10 ** 6, kv_groups=1)
+    return dict(value=n / (el * scale), unit="steps/s", cores=blas_threads(), kind="oracle",
+                sample=f"{n} steps of the seeded schedule through the float64 oracle, 1 of {w.h_kv} KV-head "
+                       f"groups ({w.group} query heads) at full prefix length; time x{scale:g} = whole layer")
+
+
+def reference_arm(args):
+    w = W.get(args.workload)
+    _, _, _ = oracle_steps(w, args.seed, 0.0, max(1, min(args.warmup, 16)), kv_groups=1)
+    n, el, scale = oracle_steps(w, args.seed, 1e9, args.steps, kv_groups=1)
+    value = n / (el * scale)
+    return dict(metric=METRIC, value=value, unit="steps/s", n_gpus=args.gpus, steps=n, warmup=args.warmup,
+                ms_per_step=el * scale / n * 1e3, higher_is_better=True, scaling="weak", vs_baseline=None,
+                dtype="f64", data="synthetic", impl="reference",
+                config=dict(workload=w.name, description=w.description, batch=w.batch, h_q=w.h_q, h_kv=w.h_kv,
+                            head_dim=w.head_dim, block=w.block, n_prefix=w.n_prefix, tau=w.tau,
+                            l2="n/a (host)", parallelism="host cores"),
+                cpu_baseline=dict(value=value, unit="steps/s", cores=blas_threads(), kind="oracle",
+                                  sample=f"each step: the float64 oracle on 1 of {w.h_kv} KV-head groups at full "
+                                         f"prefix length, time x{scale:g} = whole layer"),
+                e2e=dict(value=value, unit="steps/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+
+
+# ----------------------------------------------------------------------------- main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=32)
+    ap.add_argument("--workload", default="dlm8b_b4", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="fb", choices=["fb", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--dense-steps", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(reference_arm(args)), flush=True)
+        return
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    res = device_arm(args, rank, world)
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(W.get(args.workload), args.seed)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

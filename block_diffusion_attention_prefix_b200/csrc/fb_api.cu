@@ -1,0 +1,411 @@
+// fb_api.cu -- the C-ABI of libfb (declared in include/fb.h): argument
+// validation, split-KV planning, TMA descriptor encoding and kernel dispatch.
+//
+// Every entry point validates on the host and returns a negative fb_status
+// before launching anything.  No entry point allocates device memory or
+// synchronises the stream (fb_device_error excepted).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fb.h"
+#include "fb_internal.h"
+
+namespace fb {
+
+__device__ uint32_t g_device_error;  // bounded-wait timeouts (see fb_ptx.cuh)
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices];
+uint32_t* g_err_ptr[kMaxDevices];
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return (dev >= 0 && dev < kMaxDevices) ? dev : -1;
+}
+
+int device_sms(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 0;
+    g_sms[dev] = n;
+  }
+  return g_sms[dev];
+}
+
+uint32_t* device_err(int dev) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<uint32_t*>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+bool get_encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode) return true;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !fn)
+    return false;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D map over a bf16 KV tensor: (D, keys, b*H_kv), box (64, 64, 1), 128-B swizzle.
+int encode_kv_map(CUtensorMap* m, const void* base, int D, long long keys, long long row_stride,
+                  long long head_stride, int bh) {
+  std::memset(m, 0, sizeof(*m));
+  if (keys == 0) return FB_OK;  // never loaded
+  if (!get_encoder()) return FB_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)keys, (cuuint64_t)bh};
+  cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, (cuuint64_t)head_stride * 2};
+  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FB_OK : FB_ERR_CUDA;
+}
+
+int resolve(const fb_shape* s, Dims* d) {
+  if (!s) return FB_ERR_NULL;
+  if (s->dtype != FB_F32 && s->dtype != FB_BF16) return FB_ERR_DTYPE;
+  if (s->batch < 1 || s->h_q < 1 || s->h_kv < 1 || s->block < 1 || s->n_prefix < 0) return FB_ERR_SHAPE;
+  if (s->h_q % s->h_kv) return FB_ERR_SHAPE;
+  if (s->dtype == FB_BF16) {
+    if (s->head_dim != 64 && s->head_dim != 128) return FB_ERR_UNSUPPORTED;
+  } else {
+    if (s->head_dim < 32 || s->head_dim > 128 || s->head_dim % 32) return FB_ERR_UNSUPPORTED;
+  }
+  if ((long long)s->batch * s->h_kv > 65535) return FB_ERR_SHAPE;
+  if ((long long)s->block * (s->h_q / s->h_kv) > (1LL << 24)) return FB_ERR_SHAPE;
+  if (s->n_prefix > (1LL << 31) - 64) return FB_ERR_SHAPE;
+  const long long rs = s->kv_row_stride ? s->kv_row_stride : s->head_dim;
+  if (rs < s->head_dim) return FB_ERR_SHAPE;
+  const long long hs = s->kv_head_stride ? s->kv_head_stride : s->n_prefix * rs;
+  if (s->n_prefix > 0 && hs < (s->n_prefix - 1) * rs + s->head_dim) return FB_ERR_SHAPE;
+  const int eb = s->dtype == FB_BF16 ? 2 : 4;
+  if ((rs * eb) % 16 || (hs * eb) % 16) return FB_ERR_ALIGN;
+  if (!(s->scale >= 0.f) || std::isinf(s->scale)) return FB_ERR_ARG;
+  d->b = s->batch;
+  d->hq = s->h_q;
+  d->hkv = s->h_kv;
+  d->G = s->h_q / s->h_kv;
+  d->D = s->head_dim;
+  d->B = s->block;
+  d->N = s->n_prefix;
+  d->row_stride = rs;
+  d->head_stride = hs;
+  d->scale = s->scale > 0.f ? s->scale : 1.f / std::sqrt((float)s->head_dim);
+  d->dtype = s->dtype;
+  d->R = d->G * d->B;
+  return FB_OK;
+}
+
+int check_ptr(const void* p) {
+  if (!p) return FB_ERR_NULL;
+  return aligned16(p) ? FB_OK : FB_ERR_ALIGN;
+}
+
+int gate_params(const fb_gate* g, const Dims& d, GateParams* gp) {
+  std::memset(gp, 0, sizeof(*gp));
+  if (!g) return FB_OK;
+  if (!g->updated_mask) return FB_ERR_NULL;
+  if (g->head_sim && !aligned16(g->head_sim)) return FB_ERR_ALIGN;
+  if (!std::isfinite(g->gamma) && g->head_sim) return FB_ERR_ARG;
+  gp->mask = g->updated_mask;
+  gp->sim = g->head_sim;
+  gp->enabled = 1;
+  gp->first = g->first_step ? 1 : 0;
+  gp->tau = g->tau;
+  gp->gamma = g->gamma;
+  (void)d;
+  return FB_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? FB_OK : FB_ERR_CUDA; }
+
+#define FB_TRY(x)            \
+  do {                       \
+    const int _st = (x);     \
+    if (_st != FB_OK) return _st; \
+  } while (0)
+
+// One split-KV attention pass over `keys` keys (prefix or large in-block).
+int run_pass(const Dims& d0, long long keys, const void* q, const void* k, const void* v, long long row_stride,
+             long long head_stride, const GateParams& gp, const Epilogue& ep, void* ws, size_t ws_bytes,
+             cudaStream_t stream) {
+  if (!ws) return FB_ERR_WORKSPACE;
+  if (!aligned16(ws)) return FB_ERR_ALIGN;
+  const int dev = current_device();
+  if (dev < 0) return FB_ERR_CUDA;
+  const int sms = device_sms(dev);
+  uint32_t* err = device_err(dev);
+  if (!sms || !err) return FB_ERR_CUDA;
+  Dims d = d0;
+  d.N = keys;
+  d.row_stride = row_stride;
+  d.head_stride = head_stride;
+  PassArgs a;
+  a.d = d;
+  a.plan = plan_split(d.R, d.D, keys, d.b, d.hkv, d.dtype, sms);
+  if (a.plan.n_row_tiles > 65535) return FB_ERR_SHAPE;
+  if (ws_bytes < a.plan.total()) return FB_ERR_WORKSPACE;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.gate = gp;
+  a.ep = ep;
+  a.counters = static_cast<unsigned int*>(ws);
+  a.partials = reinterpret_cast<float*>(static_cast<char*>(ws) + a.plan.counter_bytes);
+  a.err = err;
+  if (d.dtype == FB_BF16) {
+    if (!bf16_pass_supported(d.D, a.plan.row_tile)) return FB_ERR_UNSUPPORTED;
+    CUtensorMap tk, tv;
+    FB_TRY(encode_kv_map(&tk, k, d.D, keys, row_stride, head_stride, d.b * d.hkv));
+    FB_TRY(encode_kv_map(&tv, v, d.D, keys, row_stride, head_stride, d.b * d.hkv));
+    return cuda_status(launch_pass_bf16(a, tk, tv, stream));
+  }
+  return cuda_status(launch_pass_f32(a, stream));
+}
+
+size_t pass_bytes(const Dims& d, long long keys) {
+  const int dev = current_device();
+  const int sms = dev >= 0 ? device_sms(dev) : 0;
+  return plan_split(d.R, d.D, keys, d.b, d.hkv, d.dtype, sms > 0 ? sms : 148).total();
+}
+
+}  // namespace
+
+SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int num_sms) {
+  SplitPlan p;
+  std::memset(&p, 0, sizeof(p));
+  if (dtype == FB_BF16) {
+    p.row_tile = R <= 16 ? 16 : (R <= 32 ? 32 : 64);
+    p.key_tile = 64;
+  } else {
+    p.row_tile = 16;
+    p.key_tile = 32;
+  }
+  const int ctas_per_sm = dtype == FB_BF16 ? 1 : 4;
+  p.n_row_tiles = (R + p.row_tile - 1) / p.row_tile;
+  const long long units = (long long)b * hkv * p.n_row_tiles;
+  const long long total_tiles = (N + p.key_tile - 1) / p.key_tile;
+  long long target = (long long)num_sms * ctas_per_sm;
+  long long splits = units > 0 ? target / units : 1;
+  if (splits < 1) splits = 1;
+  if (total_tiles > 0 && splits > total_tiles) splits = total_tiles;
+  if (total_tiles > 0) {
+    p.tiles_per_split = (int)((total_tiles + splits - 1) / splits);
+    p.splits = (int)((total_tiles + p.tiles_per_split - 1) / p.tiles_per_split);
+  } else {
+    p.tiles_per_split = 0;
+    p.splits = 1;
+  }
+  p.counter_bytes = ((size_t)units * 4 + 255) / 256 * 256;
+  p.partial_bytes = (size_t)units * p.splits * p.row_tile * (D + 4) * sizeof(float);
+  return p;
+}
+
+}  // namespace fb
+
+using namespace fb;
+
+extern "C" {
+
+int fb_version(void) { return 100; }
+
+const char* fb_status_string(int status) {
+  switch (status) {
+    case FB_OK: return "ok";
+    case FB_ERR_NULL: return "required pointer is NULL";
+    case FB_ERR_SHAPE: return "sizes out of range or inconsistent";
+    case FB_ERR_ALIGN: return "pointer or stride not 16-byte aligned";
+    case FB_ERR_DTYPE: return "dtype not supported";
+    case FB_ERR_WORKSPACE: return "workspace missing or too small";
+    case FB_ERR_CUDA: return "CUDA call failed";
+    case FB_ERR_UNSUPPORTED: return "configuration not implemented";
+    case FB_ERR_ARG: return "invalid argument";
+    default: return "unknown status";
+  }
+}
+
+int fb_device_error(int32_t* code) {
+  if (!code) return FB_ERR_NULL;
+  const int dev = current_device();
+  if (dev < 0) return FB_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return FB_ERR_CUDA;
+  uint32_t v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return FB_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return FB_ERR_CUDA;
+  *code = (int32_t)v;
+  return FB_OK;
+}
+
+size_t fb_workspace_bytes(const fb_shape* shape) {
+  Dims d;
+  if (resolve(shape, &d) != FB_OK) return 0;
+  size_t n = pass_bytes(d, d.N);
+  if (d.B > kSmallBlockMax) {
+    const size_t nb = pass_bytes(d, d.B);
+    if (nb > n) n = nb;
+  }
+  return n;
+}
+
+int fb_workspace_init(void* ws, size_t ws_bytes, fb_stream_t stream) {
+  if (!ws) return FB_ERR_NULL;
+  return cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream) == cudaSuccess ? FB_OK : FB_ERR_CUDA;
+}
+
+int fb_gate_eval(const fb_shape* shape, const fb_gate* gate, int32_t* dec_M, uint8_t* dec_reuse,
+                 fb_stream_t stream) {
+  Dims d;
+  FB_TRY(resolve(shape, &d));
+  if (!gate || (!dec_M && !dec_reuse)) return FB_ERR_NULL;
+  GateParams gp;
+  FB_TRY(gate_params(gate, d, &gp));
+  return cuda_status(launch_gate_eval(d, gp, dec_M, dec_reuse, (cudaStream_t)stream));
+}
+
+int fb_prefix_attn(const fb_shape* shape, const void* q, const void* k_cache, const void* v_cache,
+                   const fb_gate* gate, float* a_out, float* l_out, void* ws, size_t ws_bytes,
+                   fb_stream_t stream) {
+  Dims d;
+  FB_TRY(resolve(shape, &d));
+  FB_TRY(check_ptr(q));
+  FB_TRY(check_ptr(a_out));
+  FB_TRY(check_ptr(l_out));
+  if (d.N > 0) {
+    FB_TRY(check_ptr(k_cache));
+    FB_TRY(check_ptr(v_cache));
+  }
+  GateParams gp;
+  FB_TRY(gate_params(gate, d, &gp));
+  Epilogue ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.mode = 0;
+  ep.a_dst = a_out;
+  ep.l_dst = l_out;
+  return run_pass(d, d.N, q, k_cache, v_cache, d.row_stride, d.head_stride, gp, ep, ws, ws_bytes,
+                  (cudaStream_t)stream);
+}
+
+int fb_block_attn(const fb_shape* shape, const void* q, const void* k_blk, const void* v_blk, float* a_in,
+                  float* l_in, void* ws, size_t ws_bytes, fb_stream_t stream) {
+  Dims d;
+  FB_TRY(resolve(shape, &d));
+  FB_TRY(check_ptr(q));
+  FB_TRY(check_ptr(k_blk));
+  FB_TRY(check_ptr(v_blk));
+  FB_TRY(check_ptr(a_in));
+  FB_TRY(check_ptr(l_in));
+  Epilogue ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.mode = 0;
+  ep.a_dst = a_in;
+  ep.l_dst = l_in;
+  GateParams none;
+  std::memset(&none, 0, sizeof(none));
+  if (d.B <= kSmallBlockMax) {
+    SmallBlockArgs a;
+    a.d = d;
+    a.q = q;
+    a.k_blk = k_blk;
+    a.v_blk = v_blk;
+    a.gate = none;
+    a.ep = ep;
+    a.dec_M = nullptr;
+    a.dec_reuse = nullptr;
+    return cuda_status(launch_small_block(a, (cudaStream_t)stream));
+  }
+  return run_pass(d, d.B, q, k_blk, v_blk, d.D, (long long)d.B * d.D, none, ep, ws, ws_bytes,
+                  (cudaStream_t)stream);
+}
+
+int fb_merge(const fb_shape* shape, const float* a1, const float* l1, const float* a2, const float* l2,
+             void* a_full, float* l_full, fb_stream_t stream) {
+  Dims d;
+  FB_TRY(resolve(shape, &d));
+  FB_TRY(check_ptr(a1));
+  FB_TRY(check_ptr(a2));
+  FB_TRY(check_ptr(a_full));
+  if (!l1 || !l2) return FB_ERR_NULL;
+  return cuda_status(launch_merge(d, a1, l1, a2, l2, a_full, l_full, (cudaStream_t)stream));
+}
+
+int fb_block_merge(const fb_shape* shape, const void* q, const void* k_blk, const void* v_blk,
+                   const fb_gate* gate, const float* a_out, const float* l_out, void* a_full, float* l_full,
+                   int32_t* dec_M, uint8_t* dec_reuse, void* ws, size_t ws_bytes, fb_stream_t stream) {
+  Dims d;
+  FB_TRY(resolve(shape, &d));
+  FB_TRY(check_ptr(q));
+  FB_TRY(check_ptr(k_blk));
+  FB_TRY(check_ptr(v_blk));
+  FB_TRY(check_ptr(a_out));
+  FB_TRY(check_ptr(a_full));
+  if (!l_out) return FB_ERR_NULL;
+  GateParams gp;
+  FB_TRY(gate_params(gate, d, &gp));
+  if (!gp.enabled && (dec_M || dec_reuse)) return FB_ERR_NULL;
+  Epilogue ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.mode = 1;
+  ep.a_prev = a_out;
+  ep.l_prev = l_out;
+  ep.a_full = a_full;
+  ep.l_full = l_full;
+  ep.out_bf16 = d.dtype == FB_BF16;
+  if (d.B <= kSmallBlockMax) {
+    SmallBlockArgs a;
+    a.d = d;
+    a.q = q;
+    a.k_blk = k_blk;
+    a.v_blk = v_blk;
+    a.gate = gp;
+    a.ep = ep;
+    a.dec_M = dec_M;
+    a.dec_reuse = dec_reuse;
+    return cuda_status(launch_small_block(a, (cudaStream_t)stream));
+  }
+  if (gp.enabled && (dec_M || dec_reuse))
+    FB_TRY(cuda_status(launch_gate_eval(d, gp, dec_M, dec_reuse, (cudaStream_t)stream)));
+  GateParams none;
+  std::memset(&none, 0, sizeof(none));
+  return run_pass(d, d.B, q, k_blk, v_blk, d.D, (long long)d.B * d.D, none, ep, ws, ws_bytes,
+                  (cudaStream_t)stream);
+}
+
+int fb_step(const fb_shape* shape, const void* q, const void* k_cache, const void* v_cache, const void* k_blk,
+            const void* v_blk, const fb_gate* gate, float* a_out, float* l_out, void* a_full, float* l_full,
+            int32_t* dec_M, uint8_t* dec_reuse, void* ws, size_t ws_bytes, fb_stream_t stream) {
+  if (!gate) return FB_ERR_NULL;
+  Dims d;
+  FB_TRY(resolve(shape, &d));
+  FB_TRY(check_ptr(k_blk));
+  FB_TRY(check_ptr(v_blk));
+  FB_TRY(check_ptr(a_full));
+  if (ws_bytes < fb_workspace_bytes(shape)) return FB_ERR_WORKSPACE;
+  FB_TRY(fb_prefix_attn(shape, q, k_cache, v_cache, gate, a_out, l_out, ws, ws_bytes, stream));
+  return fb_block_merge(shape, q, k_blk, v_blk, gate, a_out, l_out, a_full, l_full, dec_M, dec_reuse, ws,
+                        ws_bytes, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,100 @@
+// fb_internal.h -- declarations shared by the translation units of libfb.
+//
+// Plain structs passed by value to kernels, the split-KV workspace plan, and the
+// launch functions each kernel file provides to the C-ABI layer (fb_api.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace fb {
+
+// Gate of one denoising step, as device-readable arguments.  enabled == 0 means
+// "recompute every row" (no gate).  See fb_gate in include/fb.h.
+struct GateParams {
+  const uint8_t* mask;  // [b, B]
+  const float* sim;     // [b, H_q] or nullptr
+  int enabled;
+  int first;
+  int tau;
+  float gamma;
+};
+
+// Resolved problem sizes (strides in elements).
+struct Dims {
+  int b, hq, hkv, G, D, B;
+  long long N;            // keys of the pass (prefix N, or B for an in-block pass)
+  long long row_stride;   // elements between keys
+  long long head_stride;  // elements between KV heads
+  float scale;            // softmax temperature (natural units)
+  int dtype;              // 0 = fp32, 1 = bf16
+  int R;                  // query rows per KV head = G * B
+};
+
+// Split-KV plan of one attention pass over N keys for R rows per KV head.
+struct SplitPlan {
+  int row_tile;         // rows per CTA
+  int n_row_tiles;      // ceil(R / row_tile)
+  int key_tile;         // keys per pipeline tile
+  int splits;           // CTAs along the key axis per (b, kv head, row tile)
+  int tiles_per_split;  // key tiles per split
+  size_t counter_bytes; // arrival counters, one per (b, kv head, row tile), 256-B padded
+  size_t partial_bytes; // [b*hkv][n_row_tiles][splits][row_tile][D + 4] fp32
+  size_t total() const { return counter_bytes + partial_bytes; }
+};
+
+// What the last-arriving CTA of a (b, kv head, row tile) does with the combined rows.
+struct Epilogue {
+  int mode;               // 0: write (A, L) fp32 to a_dst / l_dst; 1: merge with (a_prev, l_prev)
+  float* a_dst;           // mode 0, [b, H_q, B, D]
+  float* l_dst;           // mode 0, [b, H_q, B]
+  const float* a_prev;    // mode 1: cached (A_out, L_out)
+  const float* l_prev;
+  void* a_full;           // mode 1: output in the shape dtype
+  float* l_full;          // mode 1: nullable
+  int out_bf16;
+};
+
+// Arguments of a split-KV attention pass (prefix, or in-block for large B).
+struct PassArgs {
+  Dims d;
+  SplitPlan plan;
+  const void* q;          // [b, H_q, B, D] in d.dtype
+  const void* k;          // keys base (fp32 path reads through pointers; bf16 path uses TMA maps)
+  const void* v;
+  GateParams gate;
+  Epilogue ep;
+  unsigned int* counters; // workspace
+  float* partials;        // workspace
+  uint32_t* err;          // device error word
+};
+
+SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int num_sms);
+
+// Launchers (return cudaError_t of the launch).
+cudaError_t launch_pass_f32(const PassArgs& a, cudaStream_t s);
+cudaError_t launch_pass_bf16(const PassArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                             cudaStream_t s);
+int bf16_pass_supported(int D, int row_tile);
+
+// Small in-block pass fused with gate and merge (B <= kSmallBlockMax).
+constexpr int kSmallBlockMax = 64;
+struct SmallBlockArgs {
+  Dims d;
+  const void* q;
+  const void* k_blk;
+  const void* v_blk;
+  GateParams gate;
+  Epilogue ep;            // mode 0: write (A_in, L_in); mode 1: merge with the cache
+  int32_t* dec_M;         // nullable
+  uint8_t* dec_reuse;     // nullable
+};
+cudaError_t launch_small_block(const SmallBlockArgs& a, cudaStream_t s);
+cudaError_t launch_gate_eval(const Dims& d, const GateParams& g, int32_t* dec_M, uint8_t* dec_reuse,
+                             cudaStream_t s);
+cudaError_t launch_merge(const Dims& d, const float* a1, const float* l1, const float* a2,
+                         const float* l2, void* a_full, float* l_full, cudaStream_t s);
+
+}  // namespace fb

