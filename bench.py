@@ -106,7 +106,9 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
-                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+                reasons = fn(self._h)
                 self.samples.append((mhz, reasons))
             except Exception:
                 pass
