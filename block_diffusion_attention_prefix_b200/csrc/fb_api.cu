@@ -409,3 +409,63 @@ int fb_step(const fb_shape* shape, const void* q, const void* k_cache, const voi
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// fb_prefix_attn_noalloc: the prefix pass with its split-KV workspace in a
+// library-owned static device array, for callers that cannot allocate.
+namespace fb {
+namespace {
+
+static __device__ __align__(256) unsigned char g_static_scratch[FB_STATIC_SCRATCH_BYTES];
+void* g_static_scratch_ptr[kMaxDevices];
+
+// Device address of g_static_scratch on `dev` (which must be current).  In host
+// code the array's name is only a stand-in, so the address is looked up once per
+// device and cached.
+int static_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_static_scratch_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || !p) return FB_ERR_CUDA;
+    g_static_scratch_ptr[dev] = p;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return FB_OK;
+}
+
+}  // namespace
+}  // namespace fb
+
+extern "C" int fb_prefix_attn_noalloc(const fb_shape* shape, const void* q, const void* k_cache,
+                                      const void* v_cache, const fb_gate* gate, float* a_out, float* l_out,
+                                      fb_stream_t stream) {
+  Dims d;
+  FB_TRY(resolve(shape, &d));
+  FB_TRY(check_ptr(q));
+  FB_TRY(check_ptr(a_out));
+  FB_TRY(check_ptr(l_out));
+  if (d.N > 0) {
+    FB_TRY(check_ptr(k_cache));
+    FB_TRY(check_ptr(v_cache));
+  }
+  GateParams gp;
+  FB_TRY(gate_params(gate, d, &gp));
+  const int dev = current_device();
+  if (dev < 0) return FB_ERR_CUDA;
+  const int sms = device_sms(dev);
+  if (!sms) return FB_ERR_CUDA;
+  const SplitPlan plan = plan_split(d.R, d.D, d.N, d.b, d.hkv, d.dtype, sms);
+  if (plan.total() > (size_t)FB_STATIC_SCRATCH_BYTES) return FB_ERR_WORKSPACE;
+  void* ws = nullptr;
+  FB_TRY(static_scratch(dev, &ws));
+  // The array keeps the previous call's contents: the arrival counters must start at zero.
+  if (cudaMemsetAsync(ws, 0, plan.counter_bytes, (cudaStream_t)stream) != cudaSuccess) return FB_ERR_CUDA;
+  Epilogue ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.mode = 0;
+  ep.a_dst = a_out;
+  ep.l_dst = l_out;
+  return run_pass(d, d.N, q, k_cache, v_cache, d.row_stride, d.head_stride, gp, ep, ws,
+                  (size_t)FB_STATIC_SCRATCH_BYTES, (cudaStream_t)stream);
+}

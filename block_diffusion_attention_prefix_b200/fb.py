@@ -16,7 +16,7 @@ import torch
 __all__ = [
     "FBError", "Shape", "Gate", "load", "lib_path", "make_shape", "make_gate", "FB_F32", "FB_BF16",
     "fb_version", "fb_status_string", "fb_device_error", "fb_workspace_bytes", "fb_workspace_init",
-    "fb_gate_eval", "fb_prefix_attn", "fb_block_attn", "fb_merge", "fb_block_merge", "fb_step",
+    "fb_gate_eval", "fb_prefix_attn", "fb_prefix_attn_noalloc", "fb_block_attn", "fb_merge", "fb_block_merge", "fb_step",
     "CachedAttentionLayer", "EXPORTED",
 ]
 
@@ -69,6 +69,7 @@ EXPORTED = {
     "fb_merge": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fb_block_merge": (_i, [_PS, _vp, _vp, _vp, _PG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fb_step": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _PG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "fb_prefix_attn_noalloc": (_i, [_PS, _vp, _vp, _vp, _PG, _vp, _vp, _vp]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -190,6 +191,13 @@ def fb_step(shape, q, k_cache, v_cache, k_blk, v_blk, gate, a_out, l_out, a_full
     _check("fb_step", load().fb_step(
         ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_blk), _ptr(v_blk), _gref(gate),
         _ptr(a_out), _ptr(l_out), _ptr(a_full), _ptr(l_full), _ptr(dec_M), _ptr(dec_reuse), *_wsargs(ws),
+        _stream()))
+
+
+def fb_prefix_attn_noalloc(shape, q, k_cache, v_cache, gate, a_out, l_out):
+    """fb_prefix_attn with the workspace in library-owned static device memory (no allocation)."""
+    _check("fb_prefix_attn_noalloc", load().fb_prefix_attn_noalloc(
+        ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache), _gref(gate), _ptr(a_out), _ptr(l_out),
         _stream()))
 
 

@@ -158,6 +158,32 @@ int fb_step(const fb_shape* shape, const void* q, const void* k_cache, const voi
             float* l_out, void* a_full, float* l_full, int32_t* dec_M, uint8_t* dec_reuse,
             void* ws, size_t ws_bytes, fb_stream_t stream);
 
+/* Out-of-block attention for callers that cannot allocate device memory.
+ *
+ * The pages have no counterpart: this is a deployment variant of fb_prefix_attn.
+ * Some callers cannot call cudaMalloc (or any allocator) at the point where they
+ * run attention -- for example code running under a fixed memory budget whose
+ * pools are already carved up, or hosts that forbid allocation on their hot path.
+ * They cannot provide the split-KV workspace that fb_prefix_attn takes, so this
+ * entry point keeps it in library-owned device memory instead: a file-scope
+ * static device array of FB_STATIC_SCRATCH_BYTES, which every GPU that loads the
+ * library holds until the process exits.  Nothing is allocated or freed by the
+ * call.  The caller still passes q, the KV cache and the outputs, with the same
+ * meaning, layout and gate as fb_prefix_attn.
+ *
+ *  - Shapes whose workspace (fb_workspace_bytes for the prefix pass) exceeds
+ *    FB_STATIC_SCRATCH_BYTES are rejected with FB_ERR_WORKSPACE before any launch.
+ *  - The first call on a device looks up the array's device address (with that
+ *    device current); make that first call before any stream capture.
+ *  - All calls on a device share the one array, and it keeps the last call's
+ *    contents: each call first clears the arrival counters it needs on `stream`.
+ *    Calls that overlap on the GPU (other streams, other threads) race on the
+ *    array and give wrong results: serialise them. */
+#define FB_STATIC_SCRATCH_BYTES (8u << 20)
+int fb_prefix_attn_noalloc(const fb_shape* shape, const void* q, const void* k_cache,
+                           const void* v_cache, const fb_gate* gate, float* a_out, float* l_out,
+                           fb_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
