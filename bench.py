@@ -142,6 +142,23 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- device arm
 
 
+class L2Flush:
+    """Evicts the step's data from L2 between timed steps: writes a buffer larger
+    than L2, then reads another one.  The read evicts the dirty lines of the write
+    (their write-back happens here, outside the timed step), so the next step
+    starts with an L2 full of clean, unrelated lines -- as after the other layers'
+    attention in a model -- instead of paying ~126 MB of write-back itself."""
+
+    def __init__(self, dev):
+        self.w = torch.empty((L2_FLUSH_BYTES,), device=dev, dtype=torch.uint8)
+        self.r = torch.ones((L2_FLUSH_BYTES // 4,), device=dev, dtype=torch.float32)
+        self.sink = torch.empty((), device=dev, dtype=torch.float32)
+
+    def __call__(self):
+        self.w.zero_()
+        torch.sum(self.r, dim=0, out=self.sink)
+
+
 class DeviceWorkload:
     """The workload's inputs resident in HBM and the layer state, stepped through libfb."""
 
@@ -168,31 +185,35 @@ class DeviceWorkload:
         self.gates = [fb.make_gate(s["mask"], s["first"], w.tau, s["sim"], w.gamma or 0.0) for s in self.sched]
 
     def launches_per_step(self) -> int:
-        big = self.w.block > 64
-        return 2 + (1 if big else 0)
+        # fb_step is one fused launch for blocks of up to 64 tokens; larger blocks
+        # take the prefix pass, the gate record and the in-block pass.
+        return 1 if self.w.block <= 64 else 3
 
-    def run_step(self, i: int, dec_M, dec_reuse, ev=None, tau_override=None):
+    def step_args(self, i: int, dec_M, dec_reuse, tau_override=None):
+        """Marshalled ctypes arguments of fb_step for schedule position i."""
+        import ctypes
         fb, s = self.fb, self.sched[i % len(self.sched)]
-        g = self.gates[i % len(self.sched)]
-        if tau_override is not None:
-            g = fb.make_gate(s["mask"], s["first"], tau_override, s["sim"], self.w.gamma or 0.0)
-        if ev is not None:
-            ev[0].record()
-        fb.fb_prefix_attn(self.shape, s["q"], self.k, self.v, g, self.a_out, self.l_out, self.ws)
-        if ev is not None:
-            ev[1].record()
-        fb.fb_block_merge(self.shape, s["q"], s["k_blk"], s["v_blk"], g, self.a_out, self.l_out, self.a_full,
-                          self.l_full, dec_M, dec_reuse, self.ws)
-        if ev is not None:
-            ev[2].record()
+        tau = self.w.tau if tau_override is None else tau_override
+        g = fb.make_gate(s["mask"], s["first"], tau, s["sim"], self.w.gamma or 0.0)
+        vp = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        args = (ctypes.byref(self.shape), vp(s["q"]), vp(self.k), vp(self.v), vp(s["k_blk"]), vp(s["v_blk"]),
+                ctypes.byref(g), vp(self.a_out), vp(self.l_out), vp(self.a_full), vp(self.l_full), vp(dec_M),
+                vp(dec_reuse), vp(self.ws), self.ws.numel(), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        return args, g
 
-    def prefix_algorithmic_bytes(self) -> int:
-        """Bytes a recompute launch of the prefix pass must move: prefix K and V,
-        the block queries, and the cache rows it writes (A_out fp32, L_out fp32)."""
+    def algorithmic_bytes(self):
+        """(recompute, reuse) bytes of one step: what the fused step kernel must move.
+
+        Recompute: prefix K and V, Q, the block's K and V, the cache rows written
+        (A_out and L_out, fp32) and the output (A_full in the dtype, L_full fp32).
+        Reuse: the same without the prefix K/V, with the cache read instead of written.
+        """
         w = self.w
         q = w.batch * w.h_q * w.block * w.head_dim * w.elem_bytes
+        kvb = 2 * w.batch * w.h_kv * w.block * w.head_dim * w.elem_bytes
         cache = w.batch * w.h_q * w.block * (w.head_dim + 1) * 4
-        return w.prefix_bytes() + q + cache
+        out = w.batch * w.h_q * w.block * (w.head_dim * w.elem_bytes + 4)
+        return w.prefix_bytes() + q + kvb + cache + out, q + kvb + cache + out
 
 
 def device_arm(args, rank, world):
@@ -202,33 +223,43 @@ def device_arm(args, rank, world):
     dw = DeviceWorkload(fb, w, seed=args.seed + rank)
     K, Wm = args.steps, args.warmup
     dev = torch.device("cuda")
-    flush = torch.empty((L2_FLUSH_BYTES,), device=dev, dtype=torch.uint8)
+    flush = L2Flush(dev)
     dec_M = torch.zeros((K, w.batch), device=dev, dtype=torch.int32)
     dec_R = torch.zeros((K, w.batch, w.h_q), device=dev, dtype=torch.uint8)
     wdM = torch.zeros((w.batch,), device=dev, dtype=torch.int32)
     wdR = torch.zeros((w.batch, w.h_q), device=dev, dtype=torch.uint8)
     fb.fb_workspace_init(dw.ws)
-    # warm-up: whole blocks from step 0 so the cache is valid
+    lib = fb.load()
+    npos = len(dw.sched)
+    # pre-marshalled fb_step arguments per schedule position (the timed steps write
+    # their decisions to per-step rows of dec_M / dec_R)
+    warm = [dw.step_args(i, wdM, wdR) for i in range(npos)]
     for i in range(Wm):
-        flush.zero_()
-        dw.run_step(i, wdM, wdR)
+        flush()
+        st = lib.fb_step(*warm[i % npos][0])
+        assert st == 0, fb.fb_status_string(st)
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     start = Wm  # continue the schedule where warm-up stopped
+    timed = [dw.step_args(start + i, dec_M[i], dec_R[i]) for i in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    bad = 0
     with ClockSampler(torch.cuda.current_device()) as clocks:
         t0 = time.perf_counter()
         for i in range(K):
-            flush.zero_()                      # L2 flush between timed steps (outside the events)
-            dw.run_step(start + i, dec_M[i], dec_R[i], evs[i])
+            flush()                      # L2 flush between timed steps (outside the events)
+            evs[i][0].record()
+            bad |= lib.fb_step(*timed[i][0])
+            evs[i][1].record()
         torch.cuda.synchronize()
         wall = time.perf_counter() - t0
+    if bad:
+        raise RuntimeError("fb_step failed inside the timed region")
     if world > 1:
         torch.distributed.barrier()
-    step_ms = [e[0].elapsed_time(e[2]) for e in evs]
-    prefix_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
     reuse = dec_R.cpu().numpy().astype(bool)            # [K, b, H_q]
     recompute_steps = [i for i in range(K) if not reuse[i].all()]
     reuse_steps = [i for i in range(K) if reuse[i].all()]
@@ -240,20 +271,23 @@ def device_arm(args, rank, world):
         t_max = float(t.item())
     value = world * K / (t_max / 1e3)
     hbm, peak_kind = peaks()
-    alg = dw.prefix_algorithmic_bytes()
-    rec_ms = [prefix_ms[i] for i in recompute_steps]
+    alg, alg_reuse = dw.algorithmic_bytes()
+    rec_ms = [step_ms[i] for i in recompute_steps]
     achieved = (alg * len(rec_ms)) / (sum(rec_ms) / 1e3) / 1e9 if rec_ms else None
     traffic = ncu_traffic(args.workload)
 
     # dense-recompute reference (standard block diffusion): gate forced to recompute
     dense_ms = []
     if args.dense_steps > 0:
-        evd = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.dense_steps)]
+        dense = [dw.step_args(i, wdM, wdR, tau_override=0) for i in range(args.dense_steps)]
+        evd = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.dense_steps)]
         for i in range(args.dense_steps):
-            flush.zero_()
-            dw.run_step(i, wdM, wdR, evd[i], tau_override=0)
+            flush()
+            evd[i][0].record()
+            lib.fb_step(*dense[i][0])
+            evd[i][1].record()
         torch.cuda.synchronize()
-        dense_ms = [e[0].elapsed_time(e[2]) for e in evd]
+        dense_ms = [e[0].elapsed_time(e[1]) for e in evd]
 
     e2e = e2e_arm(fb, dw, K, Wm) if args.e2e else None
     res = dict(
@@ -263,10 +297,12 @@ def device_arm(args, rank, world):
         config=dict(workload=w.name, description=w.description, batch=w.batch, h_q=w.h_q, h_kv=w.h_kv,
                     head_dim=w.head_dim, block=w.block, n_prefix=w.n_prefix, steps_per_block=w.steps,
                     tau=w.tau, gamma=w.gamma, seed=args.seed,
-                    l2="flushed between timed steps (256 MiB write, outside the step events)",
+                    l2="flushed between timed steps, outside the step events: 256 MiB write then 256 MiB read "
+                       "(the read evicts the write's dirty lines)",
                     parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
-        roofline=dict(bound="hbm", kernel="pass_bf16_kernel (prefix split-KV pass)" if w.dtype == "bf16"
-                      else "pass_f32_kernel (prefix split-KV pass)",
+        roofline=dict(bound="hbm", kernel=("pass_bf16_kernel" if w.dtype == "bf16" else "pass_f32_kernel")
+                      + (" (fused step: gate + prefix split-KV pass + in-block + merge), recompute launches"
+                         if w.block <= 64 else " (prefix split-KV pass)"),
                       achieved=achieved, peak=hbm, unit="GB/s",
                       frac=(achieved / hbm) if achieved else None,
                       peak_source=f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
@@ -277,6 +313,7 @@ def device_arm(args, rank, world):
         breakdown=dict(recompute_steps=len(recompute_steps), reuse_steps=len(reuse_steps),
                        recompute_step_us=_mean_us(step_ms, recompute_steps),
                        reuse_step_us=_mean_us(step_ms, reuse_steps),
+                       reuse_step_alg_bytes=alg_reuse,
                        dense_recompute_step_us=(statistics.mean(dense_ms) * 1e3) if dense_ms else None,
                        dense_steps_per_s=(1e3 / statistics.mean(dense_ms)) if dense_ms else None,
                        wall_s=wall),

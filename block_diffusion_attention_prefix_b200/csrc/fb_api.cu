@@ -13,7 +13,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/fb.h"
+#include "fb.h"
 #include "fb_internal.h"
 
 namespace fb {
@@ -68,11 +68,50 @@ bool get_encoder() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Small cache of encoded tensor maps: a step re-encodes the same K/V maps every
+// call otherwise.  Keyed by every input of the encoding.
+struct MapKey {
+  const void* base;
+  long long keys, row_stride, head_stride;
+  int D, bh;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && keys == o.keys && row_stride == o.row_stride && head_stride == o.head_stride &&
+           D == o.D && bh == o.bh;
+  }
+};
+constexpr int kMapCache = 16;
+MapKey g_map_keys[kMapCache];
+CUtensorMap g_map_vals[kMapCache];
+int g_map_used = 0, g_map_next = 0;
+
+int encode_kv_map_uncached(CUtensorMap* m, const void* base, int D, long long keys, long long row_stride,
+                           long long head_stride, int bh);
+
 // 3-D map over a bf16 KV tensor: (D, keys, b*H_kv), box (64, 64, 1), 128-B swizzle.
 int encode_kv_map(CUtensorMap* m, const void* base, int D, long long keys, long long row_stride,
                   long long head_stride, int bh) {
   std::memset(m, 0, sizeof(*m));
   if (keys == 0) return FB_OK;  // never loaded
+  const MapKey key{base, keys, row_stride, head_stride, D, bh};
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (int i = 0; i < g_map_used; ++i)
+      if (g_map_keys[i] == key) {
+        *m = g_map_vals[i];
+        return FB_OK;
+      }
+  }
+  const int st = encode_kv_map_uncached(m, base, D, keys, row_stride, head_stride, bh);
+  if (st != FB_OK) return st;
+  std::lock_guard<std::mutex> lk(g_mu);
+  const int slot = g_map_used < kMapCache ? g_map_used++ : (g_map_next++ % kMapCache);
+  g_map_keys[slot] = key;
+  g_map_vals[slot] = *m;
+  return FB_OK;
+}
+
+int encode_kv_map_uncached(CUtensorMap* m, const void* base, int D, long long keys, long long row_stride,
+                           long long head_stride, int bh) {
   if (!get_encoder()) return FB_ERR_CUDA;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)keys, (cuuint64_t)bh};
   cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, (cuuint64_t)head_stride * 2};
@@ -151,7 +190,7 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? FB_OK : FB_ERR_CUDA; 
 // One split-KV attention pass over `keys` keys (prefix or large in-block).
 int run_pass(const Dims& d0, long long keys, const void* q, const void* k, const void* v, long long row_stride,
              long long head_stride, const GateParams& gp, const Epilogue& ep, void* ws, size_t ws_bytes,
-             cudaStream_t stream) {
+             cudaStream_t stream, const StepArgs* step = nullptr) {
   if (!ws) return FB_ERR_WORKSPACE;
   if (!aligned16(ws)) return FB_ERR_ALIGN;
   const int dev = current_device();
@@ -165,7 +204,7 @@ int run_pass(const Dims& d0, long long keys, const void* q, const void* k, const
   d.head_stride = head_stride;
   PassArgs a;
   a.d = d;
-  a.plan = plan_split(d.R, d.D, keys, d.b, d.hkv, d.dtype, sms);
+  a.plan = plan_split(d.R, d.D, keys, d.b, d.hkv, d.dtype, sms, step != nullptr && step->enabled);
   if (a.plan.n_row_tiles > 65535) return FB_ERR_SHAPE;
   if (ws_bytes < a.plan.total()) return FB_ERR_WORKSPACE;
   a.q = q;
@@ -173,8 +212,15 @@ int run_pass(const Dims& d0, long long keys, const void* q, const void* k, const
   a.v = v;
   a.gate = gp;
   a.ep = ep;
+  if (step)
+    a.step = *step;
+  else
+    std::memset(&a.step, 0, sizeof(a.step));
   a.counters = static_cast<unsigned int*>(ws);
   a.partials = reinterpret_cast<float*>(static_cast<char*>(ws) + a.plan.counter_bytes);
+  a.inblock = a.plan.inblock_bytes
+                  ? reinterpret_cast<float*>(static_cast<char*>(ws) + a.plan.counter_bytes + a.plan.partial_bytes)
+                  : nullptr;
   a.err = err;
   if (d.dtype == FB_BF16) {
     if (!bf16_pass_supported(d.D, a.plan.row_tile)) return FB_ERR_UNSUPPORTED;
@@ -186,15 +232,15 @@ int run_pass(const Dims& d0, long long keys, const void* q, const void* k, const
   return cuda_status(launch_pass_f32(a, stream));
 }
 
-size_t pass_bytes(const Dims& d, long long keys) {
+size_t pass_bytes(const Dims& d, long long keys, bool with_inblock = false) {
   const int dev = current_device();
   const int sms = dev >= 0 ? device_sms(dev) : 0;
-  return plan_split(d.R, d.D, keys, d.b, d.hkv, d.dtype, sms > 0 ? sms : 148).total();
+  return plan_split(d.R, d.D, keys, d.b, d.hkv, d.dtype, sms > 0 ? sms : 148, with_inblock).total();
 }
 
 }  // namespace
 
-SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int num_sms) {
+SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int num_sms, bool with_inblock) {
   SplitPlan p;
   std::memset(&p, 0, sizeof(p));
   if (dtype == FB_BF16) {
@@ -221,6 +267,7 @@ SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int n
   }
   p.counter_bytes = ((size_t)units * 4 + 255) / 256 * 256;
   p.partial_bytes = (size_t)units * p.splits * p.row_tile * (D + 4) * sizeof(float);
+  p.inblock_bytes = with_inblock ? (size_t)units * p.row_tile * (D + 4) * sizeof(float) : 0;
   return p;
 }
 
@@ -262,7 +309,7 @@ int fb_device_error(int32_t* code) {
 size_t fb_workspace_bytes(const fb_shape* shape) {
   Dims d;
   if (resolve(shape, &d) != FB_OK) return 0;
-  size_t n = pass_bytes(d, d.N);
+  size_t n = pass_bytes(d, d.N, d.B <= kSmallBlockMax);
   if (d.B > kSmallBlockMax) {
     const size_t nb = pass_bytes(d, d.B);
     if (nb > n) n = nb;
@@ -403,6 +450,34 @@ int fb_step(const fb_shape* shape, const void* q, const void* k_cache, const voi
   FB_TRY(check_ptr(v_blk));
   FB_TRY(check_ptr(a_full));
   if (ws_bytes < fb_workspace_bytes(shape)) return FB_ERR_WORKSPACE;
+  if (d.B <= kSmallBlockMax) {
+    // One launch: the prefix pass (gated) whose finishing CTAs also run the
+    // in-block pass, the merge and the decision record.
+    FB_TRY(check_ptr(q));
+    FB_TRY(check_ptr(a_out));
+    FB_TRY(check_ptr(l_out));
+    if (d.N > 0) {
+      FB_TRY(check_ptr(k_cache));
+      FB_TRY(check_ptr(v_cache));
+    }
+    GateParams gp;
+    FB_TRY(gate_params(gate, d, &gp));
+    Epilogue ep;
+    std::memset(&ep, 0, sizeof(ep));
+    ep.mode = 0;
+    ep.a_dst = a_out;
+    ep.l_dst = l_out;
+    StepArgs st;
+    st.enabled = 1;
+    st.k_blk = k_blk;
+    st.v_blk = v_blk;
+    st.a_full = a_full;
+    st.l_full = l_full;
+    st.dec_M = dec_M;
+    st.dec_reuse = dec_reuse;
+    return run_pass(d, d.N, q, k_cache, v_cache, d.row_stride, d.head_stride, gp, ep, ws, ws_bytes,
+                    (cudaStream_t)stream, &st);
+  }
   FB_TRY(fb_prefix_attn(shape, q, k_cache, v_cache, gate, a_out, l_out, ws, ws_bytes, stream));
   return fb_block_merge(shape, q, k_blk, v_blk, gate, a_out, l_out, a_full, l_full, dec_M, dec_reuse, ws,
                         ws_bytes, stream);

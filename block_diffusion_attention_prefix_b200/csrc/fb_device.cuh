@@ -14,6 +14,7 @@
 #include <math_constants.h>
 
 #include "fb_internal.h"
+#include "fb_ptx.cuh"
 
 namespace fb {
 
@@ -66,11 +67,12 @@ __device__ __forceinline__ bool head_reuse(const GateParams& g, bool tau_ok, int
 // every thread of the block.
 __device__ __forceinline__ int gate_row_flags(const GateParams& g, const Dims& d, int b, int kvh,
                                               int row0, int rows_valid, int row_tile, int* s_flags,
-                                              int* s_red) {
+                                              int* s_red, int* s_M = nullptr) {
   bool tau_ok = false;
   if (g.enabled) {
     const int M = block_updated_count(g.mask + (size_t)b * d.B, d.B, s_red);
     tau_ok = tau_reuse(g, M);
+    if (s_M && threadIdx.x == 0) *s_M = M;
   }
   int mine = 0;
   for (int r = threadIdx.x; r < row_tile; r += blockDim.x) {
@@ -173,6 +175,331 @@ __device__ __forceinline__ void combine_splits(const float* part, int splits, in
       L = M + logf(den);
     }
     epilogue4(ep, D, grow0 + r, d4, A, L);
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ float ldf(const T* p, size_t i);
+template <>
+__device__ __forceinline__ float ldf<float>(const float* p, size_t i) { return p[i]; }
+template <>
+__device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16* p, size_t i) {
+  return __bfloat162float(p[i]);
+}
+
+// Load DC consecutive elements as floats.
+template <int DC>
+__device__ __forceinline__ void load_vec(const float* p, float (&x)[DC]) {
+  if constexpr (DC == 4) {
+    const float4 v = *reinterpret_cast<const float4*>(p);
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+  } else if constexpr (DC == 2) {
+    const float2 v = *reinterpret_cast<const float2*>(p);
+    x[0] = v.x; x[1] = v.y;
+  } else {
+#pragma unroll
+    for (int t = 0; t < DC; ++t) x[t] = p[t];
+  }
+}
+template <int DC>
+__device__ __forceinline__ void load_vec(const __nv_bfloat16* p, float (&x)[DC]) {
+  if constexpr (DC == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+    x[0] = lo.x; x[1] = lo.y; x[2] = hi.x; x[3] = hi.y;
+  } else if constexpr (DC == 2) {
+    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+    x[0] = v.x; x[1] = v.y;
+  } else {
+#pragma unroll
+    for (int t = 0; t < DC; ++t) x[t] = __bfloat162float(p[t]);
+  }
+}
+
+// In-block attention of one query row by one warp (FlashBlock "Core mechanism":
+// A_in over J_in, the B tokens of the current block, bidirectional; fp32 math).
+// Lane l owns dims [l*DC, l*DC + DC).  Keys go in chunks of 8 whose dot products
+// are reduced across the warp together (independent butterflies), with an online
+// softmax across chunks.  Returns L_in (natural log); `a` gets the lane's dims of
+// the normalised A_in.  `kb` / `vb` point at the KV group's [B][D] block keys.
+template <typename T, int D>
+__device__ __forceinline__ float inblock_row(const T* qrow, const T* kb, const T* vb, int B, float scale,
+                                             float (&a)[D / 32], int lane) {
+  constexpr int DC = D / 32;
+  float q[DC];
+  load_vec<DC>(qrow + lane * DC, q);
+  float m = -CUDART_INF_F, l = 0.f, acc[DC];
+#pragma unroll
+  for (int t = 0; t < DC; ++t) acc[t] = 0.f;
+  for (int j0 = 0; j0 < B; j0 += 8) {
+    const int nj = min(8, B - j0);
+    float s[8], v[8][DC];
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      s[jj] = 0.f;
+#pragma unroll
+      for (int t = 0; t < DC; ++t) v[jj][t] = 0.f;
+      if (jj < nj) {
+        float k[DC];
+        load_vec<DC>(kb + (size_t)(j0 + jj) * D + lane * DC, k);
+        load_vec<DC>(vb + (size_t)(j0 + jj) * D + lane * DC, v[jj]);
+#pragma unroll
+        for (int t = 0; t < DC; ++t) s[jj] = fmaf(q[t], k[t], s[jj]);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+      for (int jj = 0; jj < 8; ++jj) s[jj] += __shfl_xor_sync(0xffffffffu, s[jj], o);
+    }
+    float cm = -CUDART_INF_F;
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      s[jj] = jj < nj ? s[jj] * scale : -CUDART_INF_F;
+      cm = fmaxf(cm, s[jj]);
+    }
+    const float mn = fmaxf(m, cm);
+    const float alpha = m == -CUDART_INF_F ? 0.f : expf(m - mn);
+    l *= alpha;
+#pragma unroll
+    for (int t = 0; t < DC; ++t) acc[t] *= alpha;
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const float p = jj < nj ? expf(s[jj] - mn) : 0.f;
+      l += p;
+#pragma unroll
+      for (int t = 0; t < DC; ++t) acc[t] = fmaf(p, v[jj][t], acc[t]);
+    }
+    m = mn;
+  }
+  const float inv = 1.f / l;
+#pragma unroll
+  for (int t = 0; t < DC; ++t) a[t] = acc[t] * inv;
+  return m + logf(l);
+}
+
+// In-block rows [r_begin, r_end) of tile rows (group rows row0 + r) of KV group
+// (b, kvh), one warp per row, executed by warps [0, nwarps) of the CTA.  In mode 1
+// the cache row is loaded before the in-block math so the two latencies overlap.
+template <typename T, int D>
+__device__ void inblock_rows(const Dims& d, const T* q, const T* k_blk, const T* v_blk, int b, int kvh,
+                             int row0, int r_begin, int r_end, const Epilogue& ep, int warp, int nwarps,
+                             int lane) {
+  constexpr int DC = D / 32;
+  const T* kb = k_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
+  const T* vb = v_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
+  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B + row0;
+  for (int r = r_begin + warp; r < r_end; r += nwarps) {
+    const size_t grow = grow0 + r;
+    float ap[DC], lp = 0.f;
+    if (ep.mode == 1) {
+      lp = __ldcg(ep.l_prev + grow);
+#pragma unroll
+      for (int t = 0; t < DC; ++t) ap[t] = __ldcg(ep.a_prev + grow * D + lane * DC + t);
+    }
+    float a[DC];
+    const float L = inblock_row<T, D>(q + grow * D, kb, vb, d.B, d.scale, a, lane);
+    const size_t off = grow * D + (size_t)lane * DC;
+    if (ep.mode == 0) {
+#pragma unroll
+      for (int t = 0; t < DC; ++t) ep.a_dst[off + t] = a[t];
+      if (lane == 0) ep.l_dst[grow] = L;
+      continue;
+    }
+    const float m = fmaxf(lp, L);
+    const float wp = m == -CUDART_INF_F ? 0.f : expf(lp - m);
+    const float wi = m == -CUDART_INF_F ? 0.f : expf(L - m);
+    const float den = wp + wi;
+    const float rden = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+    for (int t = 0; t < DC; ++t) {
+      const float v = (wp * ap[t] + wi * a[t]) * rden;
+      if (ep.out_bf16)
+        static_cast<__nv_bfloat16*>(ep.a_full)[off + t] = __float2bfloat16_rn(v);
+      else
+        static_cast<float*>(ep.a_full)[off + t] = v;
+    }
+    if (lane == 0 && ep.l_full) ep.l_full[grow] = den > 0.f ? m + logf(den) : -CUDART_INF_F;
+  }
+}
+
+// In-block rows [r_begin, r_end) of one tile written as (A_in, L_in) into the
+// tile's [RT][D + 4] fp32 slot of the workspace (the fused step merges them later).
+template <typename T, int D>
+__device__ void inblock_rows_to_ws(const Dims& d, const T* q, const T* k_blk, const T* v_blk, int b, int kvh,
+                                   int row0, int r_begin, int r_end, float* slot, int warp, int nwarps,
+                                   int lane) {
+  constexpr int DC = D / 32;
+  const T* kb = k_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
+  const T* vb = v_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
+  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B + row0;
+  for (int r = r_begin + warp; r < r_end; r += nwarps) {
+    float a[DC];
+    const float L = inblock_row<T, D>(q + (grow0 + r) * D, kb, vb, d.B, d.scale, a, lane);
+    float* dst = slot + (size_t)r * (D + 4);
+#pragma unroll
+    for (int t = 0; t < DC; ++t) dst[lane * DC + t] = a[t];
+    if (lane == 0) dst[D] = L;
+  }
+}
+
+// Fused-step merge of a finished tile: A_full = merge(cache row, in-block row) for
+// rows [0, rows_valid), reading the cache (possibly just written by this CTA) and
+// the in-block slot with L2-coherent loads.  Threads [0, nthr).
+template <int D>
+__device__ void merge_tile_from_ws(const Epilogue& ep, size_t grow0, int rows_valid, const float* slot, int tid,
+                                   int nthr) {
+  constexpr int D4 = D / 4;
+  for (int idx = tid; idx < rows_valid * D4; idx += nthr) {
+    const int r = idx / D4, d4 = idx - r * D4;
+    const size_t grow = grow0 + r;
+    const size_t off = grow * D + (size_t)d4 * 4;
+    const float4 ap = __ldcg(reinterpret_cast<const float4*>(ep.a_prev + off));
+    const float lp = __ldcg(ep.l_prev + grow);
+    const float4 ai = __ldcg(reinterpret_cast<const float4*>(slot + (size_t)r * (D + 4)) + d4);
+    const float li = __ldcg(slot + (size_t)r * (D + 4) + D);
+    float4 af;
+    float lf;
+    merge4(ap, lp, ai, li, af, lf);
+    store4(ep.a_full, off, af, ep.out_bf16);
+    if (d4 == 0 && ep.l_full) ep.l_full[grow] = lf;
+  }
+}
+
+// Record the gate's decisions for the rows of one tile: dec_reuse[b, h] for every
+// head with a row in the tile, and dec_M[b] when `write_M`.
+__device__ __forceinline__ void record_decisions(const GateParams& g, const Dims& d, int b, int kvh, int row0,
+                                                 int nrows, const int* s_flags, int M, int32_t* dec_M,
+                                                 uint8_t* dec_reuse, bool write_M, int tid, int nthr) {
+  if (!g.enabled) return;
+  if (dec_reuse) {
+    for (int r = tid; r < nrows; r += nthr) {
+      const int gr = row0 + r;
+      if (r == 0 || gr % d.B == 0) {
+        const int h = kvh * d.G + gr / d.B;
+        dec_reuse[(size_t)b * d.hq + h] = s_flags[r] ? 0 : 1;
+      }
+    }
+  }
+  if (write_M && dec_M && tid == 0) dec_M[b] = M;
+}
+
+// Finish one (b, kv head, row tile) in the CTA that arrived last: merge the
+// `splits` partials in fixed split order (deterministic) and write the results.
+// Partials are [splits][RT][D + 4] fp32 (A normalised in cols 0..D-1, natural-log
+// L in col D), contiguous in global memory; they reach shared memory through 1-D
+// bulk TMA copies (chunks of as many splits as `buf` holds), together with the
+// tile's in-block slot (A_in, L_in) in a fused step.  Each thread keeps an online
+// log-space merge (the FlashBlock merge equation applied split by split) for its
+// (row, 4-column) items, then:
+//   - rows flagged for recompute: the combined (A, L) goes through `ep`
+//     (mode 0: write the cache rows; mode 1: merge with the cache into A_full);
+//   - fused step (`step_ep` != nullptr): A_full = merge(cache row, in-block row),
+//     where the cache row is the one just combined (flagged rows) or the cached
+//     one (rows of reusing heads in a mixed tile).
+// Executed by threads [0, NT) with barrier `bar_id`; `buf` is `buf_bytes` of
+// 1024-byte aligned shared memory; `mbar` is an initialised mbarrier (count 1)
+// whose next phase has parity `*phase`.
+template <int D, int RT, int NT>
+__device__ void finish_tile(const float* part, int splits, const float* inblock_slot, int rows_valid,
+                            const int* s_flags, size_t grow0, const Epilogue& ep, const Epilogue* step_ep,
+                            uint8_t* buf, int buf_bytes, uint64_t* mbar, uint32_t* phase, uint32_t* err, int tid,
+                            int bar_id) {
+  constexpr int RS = D + 4;
+  constexpr int SPLIT_FLOATS = RT * RS;
+  constexpr int D4 = D / 4;
+  constexpr int IT = (RT * D4 + NT - 1) / NT;
+  const bool step = step_ep != nullptr;
+  const int in_bytes = step ? (SPLIT_FLOATS * 4 + 127) / 128 * 128 : 0;
+  float* s_in = reinterpret_cast<float*>(buf);
+  float* chunk = reinterpret_cast<float*>(buf + in_bytes);
+  const int cs = (buf_bytes - in_bytes) / (SPLIT_FLOATS * 4);
+
+  float m[IT], den[IT];
+  float4 acc[IT];
+#pragma unroll
+  for (int k = 0; k < IT; ++k) {
+    m[k] = -CUDART_INF_F;
+    den[k] = 0.f;
+    acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  bool ok = true;
+  for (int c0 = 0; c0 < splits && ok; c0 += cs) {
+    const int nsp = min(cs, splits - c0);
+    const uint32_t bytes = (uint32_t)nsp * SPLIT_FLOATS * 4;
+    const bool with_in = step && c0 == 0;
+    if (tid == 0) {
+      fence_proxy_async_global();
+      mbar_arrive_expect_tx(mbar, bytes + (with_in ? (uint32_t)SPLIT_FLOATS * 4 : 0u));
+      bulk_load(chunk, part + (size_t)c0 * SPLIT_FLOATS, bytes, mbar);
+      if (with_in) bulk_load(s_in, inblock_slot, (uint32_t)SPLIT_FLOATS * 4, mbar);
+    }
+    ok = mbar_wait_bounded(mbar, *phase, err, DEV_ERR_WAIT_COMBINE);
+    *phase ^= 1u;
+    if (ok) {
+#pragma unroll
+      for (int k = 0; k < IT; ++k) {
+        const int idx = tid + k * NT;
+        if (idx < RT * D4) {
+          const int r = idx / D4, d4 = idx - r * D4;
+          for (int s = 0; s < nsp; ++s) {
+            const float* pr = chunk + (size_t)s * SPLIT_FLOATS + (size_t)r * RS;
+            const float L = pr[D];
+            if (L == -CUDART_INF_F) continue;
+            if (L > m[k]) {
+              const float sc = m[k] == -CUDART_INF_F ? 0.f : expf(m[k] - L);
+              acc[k].x *= sc;
+              acc[k].y *= sc;
+              acc[k].z *= sc;
+              acc[k].w *= sc;
+              den[k] *= sc;
+              m[k] = L;
+            }
+            const float w = expf(L - m[k]);
+            const float4 a = *reinterpret_cast<const float4*>(pr + d4 * 4);
+            acc[k].x += w * a.x;
+            acc[k].y += w * a.y;
+            acc[k].z += w * a.z;
+            acc[k].w += w * a.w;
+            den[k] += w;
+          }
+        }
+      }
+    }
+    ok = named_barrier_and(bar_id, NT, ok);  // also: chunk buffer free again
+  }
+#pragma unroll
+  for (int k = 0; k < IT; ++k) {
+    const int idx = tid + k * NT;
+    if (idx >= RT * D4) continue;
+    const int r = idx / D4, d4 = idx - r * D4;
+    if (r >= rows_valid) continue;
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+    float L = -CUDART_INF_F;
+    if (den[k] > 0.f) {
+      const float inv = 1.f / den[k];
+      A = make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
+      L = m[k] + logf(den[k]);
+    }
+    const size_t grow = grow0 + r;
+    if (s_flags[r]) epilogue4(ep, D, grow, d4, A, L);
+    if (step) {
+      const size_t off = grow * D + (size_t)d4 * 4;
+      float4 ap = A;
+      float lp = L;
+      if (!s_flags[r]) {
+        ap = __ldcg(reinterpret_cast<const float4*>(step_ep->a_prev + off));
+        lp = __ldcg(step_ep->l_prev + grow);
+      }
+      const float4 ai = *reinterpret_cast<const float4*>(s_in + (size_t)r * RS + d4 * 4);
+      const float li = s_in[(size_t)r * RS + D];
+      float4 af;
+      float lf;
+      merge4(ap, lp, ai, li, af, lf);
+      store4(step_ep->a_full, off, af, step_ep->out_bf16);
+      if (d4 == 0 && step_ep->l_full) step_ep->l_full[grow] = lf;
+    }
   }
 }
 

@@ -11,6 +11,9 @@
 
 namespace fb {
 
+// Largest block handled by the fused small-block code (scores on CUDA cores).
+constexpr int kSmallBlockMax = 64;
+
 // Gate of one denoising step, as device-readable arguments.  enabled == 0 means
 // "recompute every row" (no gate).  See fb_gate in include/fb.h.
 struct GateParams {
@@ -42,7 +45,8 @@ struct SplitPlan {
   int tiles_per_split;  // key tiles per split
   size_t counter_bytes; // arrival counters, one per (b, kv head, row tile), 256-B padded
   size_t partial_bytes; // [b*hkv][n_row_tiles][splits][row_tile][D + 4] fp32
-  size_t total() const { return counter_bytes + partial_bytes; }
+  size_t inblock_bytes; // fused step only: [b*hkv][n_row_tiles][row_tile][D + 4] fp32 (A_in, L_in)
+  size_t total() const { return counter_bytes + partial_bytes + inblock_bytes; }
 };
 
 // What the last-arriving CTA of a (b, kv head, row tile) does with the combined rows.
@@ -57,6 +61,21 @@ struct Epilogue {
   int out_bf16;
 };
 
+// Fused-step extension of a prefix pass (blocks of at most kSmallBlockMax tokens):
+// the CTA that finishes a (b, kv head, row tile) -- the last to arrive, or split
+// 0 when every row of the tile reuses -- also computes the in-block attention of
+// its rows, merges it with the cache into A_full / L_full and records the gate's
+// decisions.  One launch is then one whole denoising step.
+struct StepArgs {
+  int enabled;
+  const void* k_blk;      // [b, H_kv, B, D]
+  const void* v_blk;
+  void* a_full;           // [b, H_q, B, D] in the shape dtype
+  float* l_full;          // nullable
+  int32_t* dec_M;         // nullable
+  uint8_t* dec_reuse;     // nullable
+};
+
 // Arguments of a split-KV attention pass (prefix, or in-block for large B).
 struct PassArgs {
   Dims d;
@@ -66,12 +85,15 @@ struct PassArgs {
   const void* v;
   GateParams gate;
   Epilogue ep;
+  StepArgs step;
   unsigned int* counters; // workspace
   float* partials;        // workspace
+  float* inblock;         // workspace, fused step only
   uint32_t* err;          // device error word
 };
 
-SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int num_sms);
+SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int num_sms,
+                     bool with_inblock = false);
 
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_pass_f32(const PassArgs& a, cudaStream_t s);
@@ -80,7 +102,6 @@ cudaError_t launch_pass_bf16(const PassArgs& a, const CUtensorMap& tk, const CUt
 int bf16_pass_supported(int D, int row_tile);
 
 // Small in-block pass fused with gate and merge (B <= kSmallBlockMax).
-constexpr int kSmallBlockMax = 64;
 struct SmallBlockArgs {
   Dims d;
   const void* q;

@@ -11,7 +11,8 @@
 //    (GQA packing: row_tile = 16..64 rows = B * G).
 //  * One producer warp issues TMA tensor loads (128-byte swizzle, no multicast)
 //    of 64-key K and V tiles into a STAGES-deep ring guarded by full/empty
-//    mbarriers.  Waits are time-bounded (fb_ptx.cuh).
+//    mbarriers.  Waits are time-bounded (fb_ptx.cuh).  One aux warp computes the
+//    CTA's share of the in-block rows meanwhile (fused step).
 //  * Consumer warps (WARPS_M x WARPS_N) run bf16 mma.sync m16n8k16 on the tiles:
 //    warp (wm, wn) owns query rows [16 wm, 16 wm + 16) and keys
 //    [wn * KW, (wn + 1) * KW) of every tile; Q stays in registers; the online
@@ -20,7 +21,13 @@
 //    its partial (A normalised, L natural) to the workspace, and the last CTA to
 //    arrive on the (b, kv head, row tile) counter merges all splits in fixed
 //    order (deterministic) and runs the epilogue (write the cache, or merge with
-//    the cache into A_full).  The counter is reset by that CTA.
+//    the cache into A_full).  The counter is reset by that CTA.  The combine
+//    brings the partials into the (now idle) ring with 1-D bulk TMA copies.
+//  * Fused step (small blocks): the in-block rows of a tile are spread over its
+//    split CTAs (aux warps) and parked in the workspace; the finishing CTA merges
+//    them with the combined cache rows into A_full and records the decisions, so
+//    a denoising step is one launch.  When every row of a tile reuses the cache,
+//    its CTAs read no K/V at all: they merge their in-block rows with the cache.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -46,7 +53,10 @@ __device__ __forceinline__ uint32_t swz(int key, int d) {
 template <int D, int WARPS_M, int WARPS_N, int STAGES>
 struct Cfg {
   static constexpr int kConsumerWarps = WARPS_M * WARPS_N;
-  static constexpr int kThreads = 32 * (kConsumerWarps + 1);
+  static constexpr int kProducerWarp = kConsumerWarps;
+  static constexpr int kAuxWarp = kConsumerWarps + 1;
+  static constexpr int kThreads = 32 * (kConsumerWarps + 2);
+  static constexpr int kFinishThreads = 32 * (kConsumerWarps + 1);  // consumers + aux
   static constexpr int kRowTile = 16 * WARPS_M;
   static constexpr int KW = kKeyTile / WARPS_N;  // keys per warp per tile
   static constexpr int kTileBytes = kKeyTile * D * 2;
@@ -56,7 +66,32 @@ struct Cfg {
   static constexpr int kSmemBytes = (kRingBytes > kScratchBytes ? kRingBytes : kScratchBytes) + 1024;
   static_assert(KW % 16 == 0, "each warp needs whole k16 steps of keys");
   static_assert(D % 64 == 0, "D must be a multiple of 64");
+  static_assert(kRingBytes >= 2 * kRowTile * (D + 4) * 4, "finisher needs the in-block slot and one split");
 };
+
+// Barrier ids: 0 = whole CTA, 1 = consumer warps, 2 = consumer + aux warps.
+constexpr int kBarConsumers = 1;
+constexpr int kBarFinish = 2;
+
+// Rows [r0, r1) of a tile assigned to split `split` for the in-block pass.
+__device__ __forceinline__ void split_rows(int rows_valid, int splits, int split, int& r0, int& r1) {
+  const int per = (rows_valid + splits - 1) / splits;
+  r0 = min(rows_valid, split * per);
+  r1 = min(rows_valid, r0 + per);
+}
+
+__device__ __forceinline__ Epilogue step_epilogue(const PassArgs& args) {
+  Epilogue ep;
+  ep.mode = 1;
+  ep.a_dst = nullptr;
+  ep.l_dst = nullptr;
+  ep.a_prev = args.ep.a_dst;
+  ep.l_prev = args.ep.l_dst;
+  ep.a_full = args.step.a_full;
+  ep.l_full = args.step.l_full;
+  ep.out_bf16 = 1;
+  return ep;
+}
 
 template <int D, int WARPS_M, int WARPS_N, int STAGES>
 __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
@@ -66,14 +101,17 @@ __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
   constexpr int NCW = C::kConsumerWarps;
   constexpr int KW = C::KW;
   constexpr int RT = C::kRowTile;
+  using bf16 = __nv_bfloat16;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t full_bar[STAGES];
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t comb_bar;
   __shared__ int s_flags[RT];
   __shared__ int s_red[32];
   __shared__ int s_last;
+  __shared__ int s_M;
 
   const Dims& d = args.d;
   const SplitPlan& plan = args.plan;
@@ -82,8 +120,30 @@ __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
   const int b = bg / d.hkv, kvh = bg - b * d.hkv;
   const int row0 = rt * RT;
   const int rows_valid = min(RT, d.R - row0);
+  const size_t unit = (size_t)bg * plan.n_row_tiles + rt;
+  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B + row0;
+  const bf16* q = static_cast<const bf16*>(args.q);
+  const bf16* k_blk = static_cast<const bf16*>(args.step.k_blk);
+  const bf16* v_blk = static_cast<const bf16*>(args.step.v_blk);
+  if (warp == C::kProducerWarp && lane == 0) {
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
 
-  if (!gate_row_flags(args.gate, d, b, kvh, row0, rows_valid, RT, s_flags, s_red)) return;
+  if (!gate_row_flags(args.gate, d, b, kvh, row0, rows_valid, RT, s_flags, s_red, &s_M)) {
+    // Every row of this tile reuses its cache: no K/V is read.  In a fused step the
+    // tile's CTAs still produce the step's output from the cache.
+    if (args.step.enabled) {
+      int r0, r1;
+      split_rows(rows_valid, plan.splits, split, r0, r1);
+      inblock_rows<bf16, D>(d, q, k_blk, v_blk, b, kvh, row0, r0, r1, step_epilogue(args), warp, C::kThreads / 32,
+                            lane);
+      if (split == 0)
+        record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, s_M, args.step.dec_M,
+                         args.step.dec_reuse, kvh == 0 && rt == 0, tid, C::kThreads);
+    }
+    return;
+  }
 
   const long long key_begin = (long long)split * plan.tiles_per_split * kKeyTile;
   const long long key_end = min(d.N, key_begin + (long long)plan.tiles_per_split * kKeyTile);
@@ -94,15 +154,14 @@ __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], NCW);
     }
+    mbar_init(&comb_bar, 1);
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == NCW) {
+  if (warp == C::kProducerWarp) {
     // ---------------- producer warp: TMA loads into the ring ----------------
     if (lane == 0 && ntiles > 0) {
-      prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % STAGES;
@@ -125,205 +184,221 @@ __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
     return;
   }
 
-  // ---------------------------- consumer warps ----------------------------
-  const int wm = warp / WARPS_N, wn = warp - (warp / WARPS_N) * WARPS_N;
-  const int c = lane & 3;
-  const int r0 = wm * 16 + (lane >> 2), r1 = r0 + 8;
+  if (warp == C::kAuxWarp) {
+    // ---------------- aux warp: this split's share of the in-block rows ------
+    if (args.step.enabled) {
+      int r0, r1;
+      split_rows(rows_valid, plan.splits, split, r0, r1);
+      inblock_rows_to_ws<bf16, D>(d, q, k_blk, v_blk, b, kvh, row0, r0, r1, args.inblock + unit * RT * (D + 4),
+                                  0, 1, lane);
+    }
+  } else {
+    // ---------------------------- consumer warps ----------------------------
+    const int wm = warp / WARPS_N, wn = warp - (warp / WARPS_N) * WARPS_N;
+    const int c = lane & 3;
+    const int r0 = wm * 16 + (lane >> 2), r1 = r0 + 8;
 
-  // Q fragments (A operand, row-major), rows beyond the group are zero.
-  uint32_t qf[D / 16][4];
-  {
-    const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(args.q) +
-                              ((size_t)(b * d.hq + kvh * d.G) * d.B + row0) * D;
-    const bool v0 = r0 < rows_valid, v1 = r1 < rows_valid;
+    // Q fragments (A operand, row-major), rows beyond the group are zero.
+    uint32_t qf[D / 16][4];
+    {
+      const bf16* qb = q + grow0 * D;
+      const bool v0 = r0 < rows_valid, v1 = r1 < rows_valid;
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const int col = kk * 16 + 2 * c;
-      qf[kk][0] = v0 ? *reinterpret_cast<const uint32_t*>(qb + (size_t)r0 * D + col) : 0u;
-      qf[kk][1] = v1 ? *reinterpret_cast<const uint32_t*>(qb + (size_t)r1 * D + col) : 0u;
-      qf[kk][2] = v0 ? *reinterpret_cast<const uint32_t*>(qb + (size_t)r0 * D + col + 8) : 0u;
-      qf[kk][3] = v1 ? *reinterpret_cast<const uint32_t*>(qb + (size_t)r1 * D + col + 8) : 0u;
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int col = kk * 16 + 2 * c;
+        qf[kk][0] = v0 ? *reinterpret_cast<const uint32_t*>(qb + (size_t)r0 * D + col) : 0u;
+        qf[kk][1] = v1 ? *reinterpret_cast<const uint32_t*>(qb + (size_t)r1 * D + col) : 0u;
+        qf[kk][2] = v0 ? *reinterpret_cast<const uint32_t*>(qb + (size_t)r0 * D + col + 8) : 0u;
+        qf[kk][3] = v1 ? *reinterpret_cast<const uint32_t*>(qb + (size_t)r1 * D + col + 8) : 0u;
+      }
+    }
+
+    float o[D / 8][4];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
+    const float sl2 = d.scale * 1.4426950408889634f;  // scale * log2(e)
+    bool ok = true;
+
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const int s = i % STAGES;
+      if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(i / STAGES) & 1u, args.err, DEV_ERR_WAIT_FULL)) {
+        ok = false;
+        break;
+      }
+      const uint32_t sK = smem_u32(smem + s * C::kStageBytes);
+      const uint32_t sV = sK + C::kTileBytes;
+      const long long tkey0 = key_begin + (long long)i * kKeyTile + wn * KW;
+
+      // S = Q K^T for this warp's KW keys.
+      float sc[KW / 8][4];
+#pragma unroll
+      for (int n = 0; n < KW / 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+        for (int n = 0; n < KW / 8; n += 2) {
+          const int key = wn * KW + n * 8 + (lane & 7) + ((lane >> 4) << 3);
+          const int dd = kk * 16 + ((lane >> 3) & 1) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(sK + swz(key, dd), b0, b1, b2, b3);
+          mma_bf16_16816(sc[n], qf[kk], b0, b1);
+          mma_bf16_16816(sc[n + 1], qf[kk], b2, b3);
+        }
+      }
+
+      // Online softmax in base 2; keys past the range end are masked.
+      const long long kvalid = key_end - tkey0;  // keys of this warp slice still in range
+      float mx0 = m0, mx1 = m1;
+#pragma unroll
+      for (int n = 0; n < KW / 8; ++n) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int col = n * 8 + 2 * c + (j & 1);
+          const float v = (col < kvalid) ? sc[n][j] * sl2 : -CUDART_INF_F;
+          sc[n][j] = v;
+          if (j < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
+        }
+      }
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+      const float base0 = (mx0 == -CUDART_INF_F) ? 0.f : mx0;
+      const float base1 = (mx1 == -CUDART_INF_F) ? 0.f : mx1;
+      const float al0 = ex2_approx(m0 - base0), al1 = ex2_approx(m1 - base1);
+      float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+      for (int n = 0; n < KW / 8; ++n) {
+        sc[n][0] = ex2_approx(sc[n][0] - base0);
+        sc[n][1] = ex2_approx(sc[n][1] - base0);
+        sc[n][2] = ex2_approx(sc[n][2] - base1);
+        sc[n][3] = ex2_approx(sc[n][3] - base1);
+        ps0 += sc[n][0] + sc[n][1];
+        ps1 += sc[n][2] + sc[n][3];
+      }
+      l0 = l0 * al0 + ps0;
+      l1 = l1 * al1 + ps1;
+      m0 = mx0;
+      m1 = mx1;
+#pragma unroll
+      for (int dn = 0; dn < D / 8; ++dn) {
+        o[dn][0] *= al0;
+        o[dn][1] *= al0;
+        o[dn][2] *= al1;
+        o[dn][3] *= al1;
+      }
+
+      // O += P V.
+#pragma unroll
+      for (int k2 = 0; k2 < KW / 16; ++k2) {
+        uint32_t pa[4];
+        pa[0] = pack_bf16x2(sc[2 * k2][0], sc[2 * k2][1]);
+        pa[1] = pack_bf16x2(sc[2 * k2][2], sc[2 * k2][3]);
+        pa[2] = pack_bf16x2(sc[2 * k2 + 1][0], sc[2 * k2 + 1][1]);
+        pa[3] = pack_bf16x2(sc[2 * k2 + 1][2], sc[2 * k2 + 1][3]);
+#pragma unroll
+        for (int dn = 0; dn < D / 8; dn += 2) {
+          const int key = wn * KW + k2 * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const int dd = dn * 8 + (lane >> 4) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(sV + swz(key, dd), b0, b1, b2, b3);
+          mma_bf16_16816(o[dn], pa, b0, b1);
+          mma_bf16_16816(o[dn + 1], pa, b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[s]);
+    }
+
+    // Row sums: reduce the per-thread partial sums over the quad.
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+
+    // Every issued tile has been consumed, so the ring is free: reuse it as scratch.
+    named_barrier_sync(kBarConsumers, NCW * 32);
+    float* scr = reinterpret_cast<float*>(smem);  // [NCW][16][D + 2]: O, then m, l
+    {
+      float* w = scr + (size_t)warp * 16 * (D + 2);
+      const int q0 = lane >> 2, q1 = q0 + 8;
+#pragma unroll
+      for (int dn = 0; dn < D / 8; ++dn) {
+        w[q0 * (D + 2) + dn * 8 + 2 * c] = o[dn][0];
+        w[q0 * (D + 2) + dn * 8 + 2 * c + 1] = o[dn][1];
+        w[q1 * (D + 2) + dn * 8 + 2 * c] = o[dn][2];
+        w[q1 * (D + 2) + dn * 8 + 2 * c + 1] = o[dn][3];
+      }
+      if (c == 0) {
+        w[q0 * (D + 2) + D] = m0;
+        w[q0 * (D + 2) + D + 1] = l0;
+        w[q1 * (D + 2) + D] = m1;
+        w[q1 * (D + 2) + D + 1] = l1;
+      }
+    }
+    named_barrier_sync(kBarConsumers, NCW * 32);
+
+    // CTA partial for this split: merge the WARPS_N key slices of each row.
+    const size_t rstride = (size_t)D + 4;
+    float* mypart = args.partials + (unit * plan.splits + split) * RT * rstride;
+    for (int idx = tid; idx < RT * (D / 4); idx += NCW * 32) {
+      const int r = idx / (D / 4), d4 = idx - r * (D / 4);
+      const int wmr = r >> 4, rr = r & 15;
+      float M = -CUDART_INF_F;
+#pragma unroll
+      for (int x = 0; x < WARPS_N; ++x) M = fmaxf(M, scr[((size_t)(wmr * WARPS_N + x) * 16 + rr) * (D + 2) + D]);
+      float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+      float L = -CUDART_INF_F;
+      if (M != -CUDART_INF_F) {
+        float den = 0.f;
+#pragma unroll
+        for (int x = 0; x < WARPS_N; ++x) {
+          const float* w = scr + ((size_t)(wmr * WARPS_N + x) * 16 + rr) * (D + 2);
+          const float scl = ex2_approx(w[D] - M);
+          den += scl * w[D + 1];
+          A.x += scl * w[d4 * 4 + 0];
+          A.y += scl * w[d4 * 4 + 1];
+          A.z += scl * w[d4 * 4 + 2];
+          A.w += scl * w[d4 * 4 + 3];
+        }
+        if (den > 0.f) {
+          const float inv = 1.f / den;
+          A.x *= inv;
+          A.y *= inv;
+          A.z *= inv;
+          A.w *= inv;
+          L = (M + __log2f(den)) * 0.6931471805599453f;
+        } else {
+          A = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+      }
+      *reinterpret_cast<float4*>(mypart + (size_t)r * rstride + d4 * 4) = A;
+      if (d4 == 0) mypart[(size_t)r * rstride + D] = L;
     }
   }
 
-  float o[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
-  const float sl2 = d.scale * 1.4426950408889634f;  // scale * log2(e)
-  bool ok = true;
-
-  for (int i = 0; i < ntiles && ok; ++i) {
-    const int s = i % STAGES;
-    if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(i / STAGES) & 1u, args.err, DEV_ERR_WAIT_FULL)) {
-      ok = false;
-      break;
-    }
-    const uint32_t sK = smem_u32(smem + s * C::kStageBytes);
-    const uint32_t sV = sK + C::kTileBytes;
-    const long long tkey0 = key_begin + (long long)i * kKeyTile + wn * KW;
-
-    // S = Q K^T for this warp's KW keys.
-    float sc[KW / 8][4];
-#pragma unroll
-    for (int n = 0; n < KW / 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-#pragma unroll
-      for (int n = 0; n < KW / 8; n += 2) {
-        const int key = wn * KW + n * 8 + (lane & 7) + ((lane >> 4) << 3);
-        const int dd = kk * 16 + ((lane >> 3) & 1) * 8;
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(sK + swz(key, dd), b0, b1, b2, b3);
-        mma_bf16_16816(sc[n], qf[kk], b0, b1);
-        mma_bf16_16816(sc[n + 1], qf[kk], b2, b3);
-      }
-    }
-
-    // Online softmax in base 2; keys past the range end are masked.
-    const long long kvalid = key_end - tkey0;  // keys of this warp slice still in range
-    float mx0 = m0, mx1 = m1;
-#pragma unroll
-    for (int n = 0; n < KW / 8; ++n) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int col = n * 8 + 2 * c + (j & 1);
-        const float v = (col < kvalid) ? sc[n][j] * sl2 : -CUDART_INF_F;
-        sc[n][j] = v;
-        if (j < 2) mx0 = fmaxf(mx0, v); else mx1 = fmaxf(mx1, v);
-      }
-    }
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-    const float base0 = (mx0 == -CUDART_INF_F) ? 0.f : mx0;
-    const float base1 = (mx1 == -CUDART_INF_F) ? 0.f : mx1;
-    const float al0 = ex2_approx(m0 - base0), al1 = ex2_approx(m1 - base1);
-    float ps0 = 0.f, ps1 = 0.f;
-#pragma unroll
-    for (int n = 0; n < KW / 8; ++n) {
-      sc[n][0] = ex2_approx(sc[n][0] - base0);
-      sc[n][1] = ex2_approx(sc[n][1] - base0);
-      sc[n][2] = ex2_approx(sc[n][2] - base1);
-      sc[n][3] = ex2_approx(sc[n][3] - base1);
-      ps0 += sc[n][0] + sc[n][1];
-      ps1 += sc[n][2] + sc[n][3];
-    }
-    l0 = l0 * al0 + ps0;
-    l1 = l1 * al1 + ps1;
-    m0 = mx0;
-    m1 = mx1;
-#pragma unroll
-    for (int dn = 0; dn < D / 8; ++dn) {
-      o[dn][0] *= al0;
-      o[dn][1] *= al0;
-      o[dn][2] *= al1;
-      o[dn][3] *= al1;
-    }
-
-    // O += P V.
-#pragma unroll
-    for (int k2 = 0; k2 < KW / 16; ++k2) {
-      uint32_t pa[4];
-      pa[0] = pack_bf16x2(sc[2 * k2][0], sc[2 * k2][1]);
-      pa[1] = pack_bf16x2(sc[2 * k2][2], sc[2 * k2][3]);
-      pa[2] = pack_bf16x2(sc[2 * k2 + 1][0], sc[2 * k2 + 1][1]);
-      pa[3] = pack_bf16x2(sc[2 * k2 + 1][2], sc[2 * k2 + 1][3]);
-#pragma unroll
-      for (int dn = 0; dn < D / 8; dn += 2) {
-        const int key = wn * KW + k2 * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int dd = dn * 8 + (lane >> 4) * 8;
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(sV + swz(key, dd), b0, b1, b2, b3);
-        mma_bf16_16816(o[dn], pa, b0, b1);
-        mma_bf16_16816(o[dn + 1], pa, b2, b3);
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[s]);
-  }
-
-  // Row sums: reduce the per-thread partial sums over the quad.
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-
-  // Every issued tile has been consumed, so the ring is free: reuse it as scratch.
-  named_barrier_sync(1, NCW * 32);
-  float* scr = reinterpret_cast<float*>(smem);  // [NCW][16][D + 2]: O, then m, l
-  {
-    float* w = scr + (size_t)warp * 16 * (D + 2);
-    const int q0 = lane >> 2, q1 = q0 + 8;
-#pragma unroll
-    for (int dn = 0; dn < D / 8; ++dn) {
-      w[q0 * (D + 2) + dn * 8 + 2 * c] = o[dn][0];
-      w[q0 * (D + 2) + dn * 8 + 2 * c + 1] = o[dn][1];
-      w[q1 * (D + 2) + dn * 8 + 2 * c] = o[dn][2];
-      w[q1 * (D + 2) + dn * 8 + 2 * c + 1] = o[dn][3];
-    }
-    if (c == 0) {
-      w[q0 * (D + 2) + D] = m0;
-      w[q0 * (D + 2) + D + 1] = l0;
-      w[q1 * (D + 2) + D] = m1;
-      w[q1 * (D + 2) + D + 1] = l1;
-    }
-  }
-  named_barrier_sync(1, NCW * 32);
-
-  // CTA partial for this split: merge the WARPS_N key slices of each row.
-  const size_t rstride = (size_t)D + 4;
-  const size_t unit = ((size_t)bg * plan.n_row_tiles + rt);
-  float* part_base = args.partials + unit * (size_t)plan.splits * RT * rstride;
-  float* mypart = part_base + (size_t)split * RT * rstride;
-  for (int idx = tid; idx < RT * (D / 4); idx += NCW * 32) {
-    const int r = idx / (D / 4), d4 = idx - r * (D / 4);
-    const int wmr = r >> 4, rr = r & 15;
-    float M = -CUDART_INF_F;
-#pragma unroll
-    for (int x = 0; x < WARPS_N; ++x) M = fmaxf(M, scr[((size_t)(wmr * WARPS_N + x) * 16 + rr) * (D + 2) + D]);
-    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-    float L = -CUDART_INF_F;
-    if (M != -CUDART_INF_F) {
-      float den = 0.f;
-#pragma unroll
-      for (int x = 0; x < WARPS_N; ++x) {
-        const float* w = scr + ((size_t)(wmr * WARPS_N + x) * 16 + rr) * (D + 2);
-        const float sc = ex2_approx(w[D] - M);
-        den += sc * w[D + 1];
-        A.x += sc * w[d4 * 4 + 0];
-        A.y += sc * w[d4 * 4 + 1];
-        A.z += sc * w[d4 * 4 + 2];
-        A.w += sc * w[d4 * 4 + 3];
-      }
-      if (den > 0.f) {
-        const float inv = 1.f / den;
-        A.x *= inv;
-        A.y *= inv;
-        A.z *= inv;
-        A.w *= inv;
-        L = (M + __log2f(den)) * 0.6931471805599453f;
-      } else {
-        A = make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-    }
-    *reinterpret_cast<float4*>(mypart + (size_t)r * rstride + d4 * 4) = A;
-    if (d4 == 0) mypart[(size_t)r * rstride + D] = L;
-  }
-
-  // Last CTA of the unit combines all splits.
-  __threadfence();
-  named_barrier_sync(1, NCW * 32);
+  // ------------- consumers + aux: arrive; the last CTA finishes the tile -------------
+  named_barrier_sync(kBarFinish, C::kFinishThreads);
   if (tid == 0) {
+    __threadfence();  // release this CTA's partial and in-block rows (cumulative over the barrier)
     const unsigned prev = atomicAdd(args.counters + unit, 1u);
+    __threadfence();  // acquire the other CTAs' writes when last
     s_last = (prev == (unsigned)plan.splits - 1u);
   }
-  named_barrier_sync(1, NCW * 32);
+  named_barrier_sync(kBarFinish, C::kFinishThreads);
   if (!s_last) return;
-  __threadfence();
-  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B + row0;
-  combine_splits(part_base, plan.splits, RT, D, rows_valid, s_flags, grow0, args.ep, tid, NCW * 32);
+  // Finisher threads are the consumer warps and the aux warp: number them 0..kFinishThreads-1.
+  const int ftid = warp < NCW ? tid : NCW * 32 + lane;
+  uint32_t comb_phase = 0;
+  const Epilogue sep = step_epilogue(args);
+  finish_tile<D, RT, C::kFinishThreads>(args.partials + unit * plan.splits * RT * (D + 4), plan.splits,
+                                        args.step.enabled ? args.inblock + unit * RT * (D + 4) : nullptr,
+                                        rows_valid, s_flags, grow0, args.ep, args.step.enabled ? &sep : nullptr,
+                                        smem, C::kRingBytes, &comb_bar, &comb_phase, args.err, ftid, kBarFinish);
+  if (args.step.enabled)
+    record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, s_M, args.step.dec_M, args.step.dec_reuse,
+                     kvh == 0 && rt == 0, ftid, C::kFinishThreads);
   if (tid == 0) args.counters[unit] = 0u;
 }
 
@@ -331,8 +406,14 @@ template <int D, int WM, int WN, int STAGES>
 cudaError_t launch_cfg(const PassArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s) {
   using C = Cfg<D, WM, WN, STAGES>;
   auto kern = pass_bf16_kernel<D, WM, WN, STAGES>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-  if (e != cudaSuccess) return e;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
   dim3 grid(a.plan.splits, a.plan.n_row_tiles, a.d.b * a.d.hkv);
   kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(tk, tv, a);
   return cudaGetLastError();

@@ -18,17 +18,24 @@ constexpr int kThreads = 128;
 constexpr int kRowTileF32 = 16;
 constexpr int kKeyTileF32 = 32;
 
+// Dynamic shared memory (floats): Q tile, K and V key tiles.
+__host__ __device__ constexpr size_t f32_smem_floats(int D) {
+  return (size_t)kRowTileF32 * D + (size_t)kKeyTileF32 * (D + 1) + (size_t)kKeyTileF32 * D;
+}
+
 template <int DC>  // D = 32 * DC
 __global__ void __launch_bounds__(kThreads) pass_f32_kernel(const PassArgs args) {
   constexpr int D = 32 * DC;
   constexpr int RT = kRowTileF32;
   constexpr int KT = kKeyTileF32;
-  __shared__ float sQ[RT][D];
-  __shared__ float sK[KT][D + 1];
-  __shared__ float sV[KT][D];
+  extern __shared__ float fsm[];
+  float (*sQ)[D] = reinterpret_cast<float (*)[D]>(fsm);
+  float (*sK)[D + 1] = reinterpret_cast<float (*)[D + 1]>(fsm + RT * D);
+  float (*sV)[D] = reinterpret_cast<float (*)[D]>(fsm + RT * D + KT * (D + 1));
   __shared__ int s_flags[RT];
   __shared__ int s_red[32];
   __shared__ int s_last;
+  __shared__ int s_M;
 
   const Dims& d = args.d;
   const SplitPlan& plan = args.plan;
@@ -38,7 +45,35 @@ __global__ void __launch_bounds__(kThreads) pass_f32_kernel(const PassArgs args)
   const int row0 = rt * RT;
   const int rows_valid = min(RT, d.R - row0);
 
-  if (!gate_row_flags(args.gate, d, b, kvh, row0, rows_valid, RT, &s_flags[0], s_red)) return;
+  Epilogue step_ep;
+  step_ep.mode = 1;
+  step_ep.a_dst = nullptr;
+  step_ep.l_dst = nullptr;
+  step_ep.a_prev = args.ep.a_dst;
+  step_ep.l_prev = args.ep.l_dst;
+  step_ep.a_full = args.step.a_full;
+  step_ep.l_full = args.step.l_full;
+  step_ep.out_bf16 = 0;
+  const int per = (rows_valid + plan.splits - 1) / plan.splits;
+  const int ib0 = min(rows_valid, split * per), ib1 = min(rows_valid, ib0 + per);
+  const size_t unit = (size_t)bg * plan.n_row_tiles + rt;
+
+  if (!gate_row_flags(args.gate, d, b, kvh, row0, rows_valid, RT, &s_flags[0], s_red, &s_M)) {
+    // Every row reuses its cache: in a fused step, merge this split's rows with it.
+    if (args.step.enabled) {
+      inblock_rows<float, D>(d, static_cast<const float*>(args.q), static_cast<const float*>(args.step.k_blk),
+                             static_cast<const float*>(args.step.v_blk), b, kvh, row0, ib0, ib1, step_ep, warp,
+                             kThreads / 32, lane);
+      if (split == 0)
+        record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, s_M, args.step.dec_M,
+                         args.step.dec_reuse, kvh == 0 && rt == 0, tid, kThreads);
+    }
+    return;
+  }
+  if (args.step.enabled)
+    inblock_rows_to_ws<float, D>(d, static_cast<const float*>(args.q), static_cast<const float*>(args.step.k_blk),
+                                 static_cast<const float*>(args.step.v_blk), b, kvh, row0, ib0, ib1,
+                                 args.inblock + unit * RT * (D + 4), warp, kThreads / 32, lane);
 
   const float* q = static_cast<const float*>(args.q) + ((size_t)(b * d.hq + kvh * d.G) * d.B + row0) * D;
   for (int i = tid; i < RT * D; i += kThreads) {
@@ -96,7 +131,6 @@ __global__ void __launch_bounds__(kThreads) pass_f32_kernel(const PassArgs args)
   }
 
   const size_t rstride = (size_t)D + 4;
-  const size_t unit = (size_t)bg * plan.n_row_tiles + rt;
   float* part_base = args.partials + unit * (size_t)plan.splits * RT * rstride;
   float* mypart = part_base + (size_t)split * RT * rstride;
 #pragma unroll
@@ -120,21 +154,38 @@ __global__ void __launch_bounds__(kThreads) pass_f32_kernel(const PassArgs args)
   __threadfence();
   const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B + row0;
   combine_splits(part_base, plan.splits, RT, D, rows_valid, s_flags, grow0, args.ep, tid, kThreads);
+  if (args.step.enabled) {
+    __syncthreads();  // the recomputed cache rows are written
+    merge_tile_from_ws<D>(step_ep, grow0, rows_valid, args.inblock + unit * RT * (D + 4), tid, kThreads);
+    record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, s_M, args.step.dec_M, args.step.dec_reuse,
+                     kvh == 0 && rt == 0, tid, kThreads);
+  }
   if (tid == 0) args.counters[unit] = 0u;
 }
 
 }  // namespace
 
-cudaError_t launch_pass_f32(const PassArgs& a, cudaStream_t s) {
+template <int DC>
+cudaError_t launch_f32_dc(const PassArgs& a, cudaStream_t s) {
+  const size_t smem = f32_smem_floats(32 * DC) * sizeof(float);
+  auto kern = pass_f32_kernel<DC>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
   dim3 grid(a.plan.splits, a.plan.n_row_tiles, a.d.b * a.d.hkv);
+  kern<<<grid, kThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pass_f32(const PassArgs& a, cudaStream_t s) {
   switch (a.d.D / 32) {
-    case 1: pass_f32_kernel<1><<<grid, kThreads, 0, s>>>(a); break;
-    case 2: pass_f32_kernel<2><<<grid, kThreads, 0, s>>>(a); break;
-    case 3: pass_f32_kernel<3><<<grid, kThreads, 0, s>>>(a); break;
-    case 4: pass_f32_kernel<4><<<grid, kThreads, 0, s>>>(a); break;
+    case 1: return launch_f32_dc<1>(a, s);
+    case 2: return launch_f32_dc<2>(a, s);
+    case 3: return launch_f32_dc<3>(a, s);
+    case 4: return launch_f32_dc<4>(a, s);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace fb
