@@ -388,19 +388,22 @@ __device__ __forceinline__ void record_decisions(const GateParams& g, const Dims
 // Finish one (b, kv head, row tile) in the CTA that arrived last: merge the
 // `splits` partials in fixed split order (deterministic) and write the results.
 // Partials are [splits][RT][D + 4] fp32 (A normalised in cols 0..D-1, natural-log
-// L in col D), contiguous in global memory; they reach shared memory through 1-D
-// bulk TMA copies (chunks of as many splits as `buf` holds), together with the
-// tile's in-block slot (A_in, L_in) in a fused step.  Each thread keeps an online
-// log-space merge (the FlashBlock merge equation applied split by split) for its
-// (row, 4-column) items, then:
-//   - rows flagged for recompute: the combined (A, L) goes through `ep`
-//     (mode 0: write the cache rows; mode 1: merge with the cache into A_full);
-//   - fused step (`step_ep` != nullptr): A_full = merge(cache row, in-block row),
-//     where the cache row is the one just combined (flagged rows) or the cached
-//     one (rows of reusing heads in a mixed tile).
+// L in col D), contiguous in global memory.
+//   1. 1-D bulk TMA copies bring the partials into shared memory (chunks of as many
+//      splits as fit), together with the tile's in-block slot in a fused step;
+//      meanwhile every thread loads a share of the L values.
+//   2. Per row, the split weights w_s = e^{L_s - M} / sum_s e^{L_s - M} and the
+//      merged L = M + ln sum_s e^{L_s - M} are computed once (the FlashBlock merge
+//      equation over all splits).
+//   3. Each thread accumulates sum_s w_s A_s for its (row, 4-column) items, then
+//      - rows flagged for recompute go through `ep` (mode 0: write the cache rows;
+//        mode 1: merge with the cache into A_full);
+//      - fused step (`step_ep` != nullptr): A_full = merge(cache row, in-block
+//        row), the cache row being the one just combined (flagged rows) or the
+//        cached one (rows of reusing heads in a mixed tile).
 // Executed by threads [0, NT) with barrier `bar_id`; `buf` is `buf_bytes` of
-// 1024-byte aligned shared memory; `mbar` is an initialised mbarrier (count 1)
-// whose next phase has parity `*phase`.
+// 1024-byte aligned shared memory; `mbar` an initialised mbarrier (count 1) whose
+// next phase has parity `*phase`.
 template <int D, int RT, int NT>
 __device__ void finish_tile(const float* part, int splits, const float* inblock_slot, int rows_valid,
                             const int* s_flags, size_t grow0, const Epilogue& ep, const Epilogue* step_ep,
@@ -412,29 +415,66 @@ __device__ void finish_tile(const float* part, int splits, const float* inblock_
   constexpr int IT = (RT * D4 + NT - 1) / NT;
   const bool step = step_ep != nullptr;
   const int in_bytes = step ? (SPLIT_FLOATS * 4 + 127) / 128 * 128 : 0;
+  const int w_bytes = ((splits + 4) * RT * 4 + 127) / 128 * 128;
   float* s_in = reinterpret_cast<float*>(buf);
-  float* chunk = reinterpret_cast<float*>(buf + in_bytes);
-  const int cs = (buf_bytes - in_bytes) / (SPLIT_FLOATS * 4);
+  // [splits][RT] split weights, then per row: merged L, 1/den, and (fused step) the
+  // weights of the cache row and of the in-block row in the final merge.
+  float* sW = reinterpret_cast<float*>(buf + in_bytes);
+  float* sLf = sW + (size_t)splits * RT;
+  float* sWo = sLf + RT;
+  float* sWi = sWo + RT;
+  float* chunk = reinterpret_cast<float*>(buf + in_bytes + w_bytes);
+  const int cs = (buf_bytes - in_bytes - w_bytes) / (SPLIT_FLOATS * 4);
 
-  float m[IT], den[IT];
-  float4 acc[IT];
-#pragma unroll
-  for (int k = 0; k < IT; ++k) {
-    m[k] = -CUDART_INF_F;
-    den[k] = 0.f;
-    acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  bool ok = true;
-  for (int c0 = 0; c0 < splits && ok; c0 += cs) {
+  auto issue = [&](int c0) {
     const int nsp = min(cs, splits - c0);
     const uint32_t bytes = (uint32_t)nsp * SPLIT_FLOATS * 4;
     const bool with_in = step && c0 == 0;
-    if (tid == 0) {
-      fence_proxy_async_global();
-      mbar_arrive_expect_tx(mbar, bytes + (with_in ? (uint32_t)SPLIT_FLOATS * 4 : 0u));
-      bulk_load(chunk, part + (size_t)c0 * SPLIT_FLOATS, bytes, mbar);
-      if (with_in) bulk_load(s_in, inblock_slot, (uint32_t)SPLIT_FLOATS * 4, mbar);
-    }
+    fence_proxy_async_global();
+    mbar_arrive_expect_tx(mbar, bytes + (with_in ? (uint32_t)SPLIT_FLOATS * 4 : 0u));
+    bulk_load(chunk, part + (size_t)c0 * SPLIT_FLOATS, bytes, mbar);
+    if (with_in) bulk_load(s_in, inblock_slot, (uint32_t)SPLIT_FLOATS * 4, mbar);
+  };
+  if (tid == 0) issue(0);
+  for (int i = tid; i < splits * RT; i += NT) {
+    const int sp = i / RT, r = i - sp * RT;
+    sW[i] = __ldcg(part + (size_t)sp * SPLIT_FLOATS + (size_t)r * RS + D);
+  }
+  named_barrier_sync(bar_id, NT);
+  // Per row: M = max_s L_s (kept in sLf for now).
+  for (int r = tid; r < RT; r += NT) {
+    float M = -CUDART_INF_F;
+    for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, sW[sp * RT + r]);
+    sLf[r] = M;
+  }
+  named_barrier_sync(bar_id, NT);
+  // All (split, row) pairs in parallel: e = e^{L_s - M}.
+  for (int i = tid; i < splits * RT; i += NT) {
+    const int r = i % RT;
+    const float M = sLf[r];
+    sW[i] = M == -CUDART_INF_F ? 0.f : expf(sW[i] - M);
+  }
+  named_barrier_sync(bar_id, NT);
+  // Per row: den, merged L, and the final-merge weights of a fused step.
+  for (int r = tid; r < RT; r += NT) {
+    const float M = sLf[r];
+    float den = 0.f;
+    for (int sp = 0; sp < splits; ++sp) den += sW[sp * RT + r];
+    const float L = den > 0.f ? M + logf(den) : -CUDART_INF_F;
+    sLf[r] = L;
+    sWo[r] = den > 0.f ? 1.f / den : 0.f;  // scale of the accumulated sum_s e_s A_s
+  }
+  named_barrier_sync(bar_id, NT);
+
+  // Two accumulation chains per item, by the parity of the global split index, so
+  // that the summation order never depends on how the splits were chunked.
+  float4 acc[IT], acc1[IT];
+#pragma unroll
+  for (int k = 0; k < IT; ++k) acc[k] = acc1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  bool ok = true;
+  for (int c0 = 0; c0 < splits && ok; c0 += cs) {
+    const int nsp = min(cs, splits - c0);
+    if (c0 > 0 && tid == 0) issue(c0);
     ok = mbar_wait_bounded(mbar, *phase, err, DEV_ERR_WAIT_COMBINE);
     *phase ^= 1u;
     if (ok) {
@@ -443,31 +483,51 @@ __device__ void finish_tile(const float* part, int splits, const float* inblock_
         const int idx = tid + k * NT;
         if (idx < RT * D4) {
           const int r = idx / D4, d4 = idx - r * D4;
-          for (int s = 0; s < nsp; ++s) {
-            const float* pr = chunk + (size_t)s * SPLIT_FLOATS + (size_t)r * RS;
-            const float L = pr[D];
-            if (L == -CUDART_INF_F) continue;
-            if (L > m[k]) {
-              const float sc = m[k] == -CUDART_INF_F ? 0.f : expf(m[k] - L);
-              acc[k].x *= sc;
-              acc[k].y *= sc;
-              acc[k].z *= sc;
-              acc[k].w *= sc;
-              den[k] *= sc;
-              m[k] = L;
-            }
-            const float w = expf(L - m[k]);
-            const float4 a = *reinterpret_cast<const float4*>(pr + d4 * 4);
-            acc[k].x += w * a.x;
-            acc[k].y += w * a.y;
-            acc[k].z += w * a.z;
-            acc[k].w += w * a.w;
-            den[k] += w;
+          const float* pr = chunk + (size_t)r * RS + d4 * 4;
+          const float* wr = sW + (size_t)c0 * RT + r;
+          for (int sp = 0; sp < nsp; ++sp) {
+            const float w = wr[sp * RT];
+            const float4 x = *reinterpret_cast<const float4*>(pr + (size_t)sp * SPLIT_FLOATS);
+            float4& a = ((c0 + sp) & 1) ? acc1[k] : acc[k];
+            a.x = fmaf(w, x.x, a.x);
+            a.y = fmaf(w, x.y, a.y);
+            a.z = fmaf(w, x.z, a.z);
+            a.w = fmaf(w, x.w, a.w);
           }
         }
       }
     }
-    ok = named_barrier_and(bar_id, NT, ok);  // also: chunk buffer free again
+    ok = named_barrier_and(bar_id, NT, ok);  // also: the chunk buffer is free again
+  }
+#pragma unroll
+  for (int k = 0; k < IT; ++k) {
+    acc[k].x += acc1[k].x;
+    acc[k].y += acc1[k].y;
+    acc[k].z += acc1[k].z;
+    acc[k].w += acc1[k].w;
+  }
+  // Fused step: per row, the weights of the cache row (w_o) and of the in-block row
+  // (w_i) in A_full = w_o A_out + w_i A_in, and L_full.  Rows of reusing heads in a
+  // mixed tile take the cached (A_out, L_out) instead of the combined one.
+  if (step) {
+    for (int r = tid; r < rows_valid; r += NT) {
+      const float lo = s_flags[r] ? sLf[r] : __ldcg(step_ep->l_prev + grow0 + r);
+      const float li = s_in[(size_t)r * RS + D];
+      const float m = fmaxf(lo, li);
+      float wo = 0.f, wi = 0.f, lf = -CUDART_INF_F;
+      if (m != -CUDART_INF_F) {
+        wo = expf(lo - m);
+        wi = expf(li - m);
+        const float den = wo + wi;
+        lf = m + logf(den);
+        wo /= den;
+        wi /= den;
+      }
+      if (step_ep->l_full) step_ep->l_full[grow0 + r] = lf;
+      sWi[r] = wi;
+      sW[r] = wo;  // split weights are no longer needed
+    }
+    named_barrier_sync(bar_id, NT);
   }
 #pragma unroll
   for (int k = 0; k < IT; ++k) {
@@ -475,30 +535,18 @@ __device__ void finish_tile(const float* part, int splits, const float* inblock_
     if (idx >= RT * D4) continue;
     const int r = idx / D4, d4 = idx - r * D4;
     if (r >= rows_valid) continue;
-    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
-    float L = -CUDART_INF_F;
-    if (den[k] > 0.f) {
-      const float inv = 1.f / den[k];
-      A = make_float4(acc[k].x * inv, acc[k].y * inv, acc[k].z * inv, acc[k].w * inv);
-      L = m[k] + logf(den[k]);
-    }
+    const float sc = sWo[r];
+    const float4 A = make_float4(acc[k].x * sc, acc[k].y * sc, acc[k].z * sc, acc[k].w * sc);
     const size_t grow = grow0 + r;
-    if (s_flags[r]) epilogue4(ep, D, grow, d4, A, L);
+    if (s_flags[r]) epilogue4(ep, D, grow, d4, A, sLf[r]);
     if (step) {
       const size_t off = grow * D + (size_t)d4 * 4;
-      float4 ap = A;
-      float lp = L;
-      if (!s_flags[r]) {
-        ap = __ldcg(reinterpret_cast<const float4*>(step_ep->a_prev + off));
-        lp = __ldcg(step_ep->l_prev + grow);
-      }
+      const float4 ap = s_flags[r] ? A : __ldcg(reinterpret_cast<const float4*>(step_ep->a_prev + off));
       const float4 ai = *reinterpret_cast<const float4*>(s_in + (size_t)r * RS + d4 * 4);
-      const float li = s_in[(size_t)r * RS + D];
-      float4 af;
-      float lf;
-      merge4(ap, lp, ai, li, af, lf);
+      const float wo = sW[r], wi = sWi[r];
+      const float4 af = make_float4(wo * ap.x + wi * ai.x, wo * ap.y + wi * ai.y, wo * ap.z + wi * ai.z,
+                                    wo * ap.w + wi * ai.w);
       store4(step_ep->a_full, off, af, step_ep->out_bf16);
-      if (d4 == 0 && step_ep->l_full) step_ep->l_full[grow] = lf;
     }
   }
 }
