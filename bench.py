@@ -180,14 +180,27 @@ class DeviceWorkload:
         self.l_out = torch.full((w.batch, w.h_q, w.block), float("-inf"), **f32)
         self.a_full = torch.zeros((w.batch, w.h_q, w.block, w.head_dim), device=dev, dtype=w.torch_dtype)
         self.l_full = torch.zeros((w.batch, w.h_q, w.block), **f32)
-        n = fb.fb_workspace_bytes(self.shape)
-        self.ws = torch.zeros(((n + 15) // 16 * 16,), device=dev, dtype=torch.uint8)
+        self.sparse_layer = None
+        if w.page_size:
+            n_sel = sparse_n_select(w)
+            self.sparse_layer = fb.SparseResidualLayer(w.batch, w.h_q, w.h_kv, w.head_dim, w.block, self.k, self.v,
+                                                       n_sel, w.page_size)
+            self.ws = self.sparse_layer.ws
+        else:
+            n = fb.fb_workspace_bytes(self.shape)
+            self.ws = torch.zeros(((n + 15) // 16 * 16,), device=dev, dtype=torch.uint8)
         self.gates = [fb.make_gate(s["mask"], s["first"], w.tau, s["sim"], w.gamma or 0.0) for s in self.sched]
 
     def launches_per_step(self) -> int:
         # fb_step is one fused launch for blocks of up to 64 tokens; larger blocks
-        # take the prefix pass, the gate record and the in-block pass.
+        # take the prefix pass, the gate record and the in-block pass.  The sparse
+        # step is the page estimate, the top-k and the sparse pass.
+        if self.sparse_layer is not None:
+            return 3
         return 1 if self.w.block <= 64 else 3
+
+    def entry(self, lib):
+        return lib.fb_sparse_step if self.sparse_layer is not None else lib.fb_step
 
     def step_args(self, i: int, dec_M, dec_reuse, tau_override=None):
         """Marshalled ctypes arguments of fb_step for schedule position i."""
@@ -196,12 +209,47 @@ class DeviceWorkload:
         tau = self.w.tau if tau_override is None else tau_override
         g = fb.make_gate(s["mask"], s["first"], tau, s["sim"], self.w.gamma or 0.0)
         vp = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+        stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        if self.sparse_layer is not None:
+            sl = self.sparse_layer
+            args = (ctypes.byref(self.shape), vp(s["q"]), vp(self.k), vp(self.v), vp(s["k_blk"]), vp(s["v_blk"]),
+                    ctypes.byref(g), ctypes.byref(sl.sparse), vp(self.a_full), vp(self.l_full), vp(dec_M),
+                    vp(dec_reuse), vp(self.ws), self.ws.numel(), stream)
+            return args, g
         args = (ctypes.byref(self.shape), vp(s["q"]), vp(self.k), vp(self.v), vp(s["k_blk"]), vp(s["v_blk"]),
                 ctypes.byref(g), vp(self.a_out), vp(self.l_out), vp(self.a_full), vp(self.l_full), vp(dec_M),
-                vp(dec_reuse), vp(self.ws), self.ws.numel(), ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+                vp(dec_reuse), vp(self.ws), self.ws.numel(), stream)
         return args, g
 
+    def union_density(self):
+        """Fraction of prefix pages in the union of each KV group's selections (KV inflation)."""
+        if self.sparse_layer is None:
+            return None
+        u = self.sparse_layer.union_bits.cpu().numpy().astype("uint32")
+        ones = sum(bin(int(x)).count("1") for x in u.reshape(-1))
+        return ones / (u.shape[0] * u.shape[1] * self.sparse_layer.n_pages)
+
     def algorithmic_bytes(self):
+        if self.sparse_layer is not None:
+            return self.sparse_algorithmic_bytes()
+        return self.dense_algorithmic_bytes()
+
+    def sparse_algorithmic_bytes(self):
+        """(recompute, reuse) bytes of a sparse step: recompute reads all prefix K/V,
+        the page bounds and Q and writes the residual and the output; reuse reads the
+        union pages of each KV group (measured after the run) plus Q, the residual and
+        the block, and writes the output."""
+        w = self.w
+        q = w.batch * w.h_q * w.block * w.head_dim * w.elem_bytes
+        kvb = 2 * w.batch * w.h_kv * w.block * w.head_dim * w.elem_bytes
+        res = w.batch * w.h_q * w.block * (w.head_dim + 1) * 4
+        out = w.batch * w.h_q * w.block * (w.head_dim * w.elem_bytes + 4)
+        bounds = 2 * w.batch * w.h_kv * w.head_dim * self.sparse_layer.n_pages * w.elem_bytes
+        dens = self.union_density() or 1.0
+        return (w.prefix_bytes() + bounds + q + kvb + res + out,
+                int(w.prefix_bytes() * dens) + q + kvb + res + out)
+
+    def dense_algorithmic_bytes(self):
         """(recompute, reuse) bytes of one step: what the fused step kernel must move.
 
         Recompute: prefix K and V, Q, the block's K and V, the cache rows written
@@ -233,10 +281,11 @@ def device_arm(args, rank, world):
     npos = len(dw.sched)
     # pre-marshalled fb_step arguments per schedule position (the timed steps write
     # their decisions to per-step rows of dec_M / dec_R)
+    step_fn = dw.entry(lib)
     warm = [dw.step_args(i, wdM, wdR) for i in range(npos)]
     for i in range(Wm):
         flush()
-        st = lib.fb_step(*warm[i % npos][0])
+        st = step_fn(*warm[i % npos][0])
         assert st == 0, fb.fb_status_string(st)
     torch.cuda.synchronize()
     start = Wm  # continue the schedule where warm-up stopped
@@ -251,7 +300,7 @@ def device_arm(args, rank, world):
         for i in range(K):
             flush()                      # L2 flush between timed steps (outside the events)
             evs[i][0].record()
-            bad |= lib.fb_step(*timed[i][0])
+            bad |= step_fn(*timed[i][0])
             evs[i][1].record()
         torch.cuda.synchronize()
         wall = time.perf_counter() - t0
@@ -284,12 +333,12 @@ def device_arm(args, rank, world):
         for i in range(args.dense_steps):
             flush()
             evd[i][0].record()
-            lib.fb_step(*dense[i][0])
+            step_fn(*dense[i][0])
             evd[i][1].record()
         torch.cuda.synchronize()
         dense_ms = [e[0].elapsed_time(e[1]) for e in evd]
 
-    e2e = e2e_arm(fb, dw, K, Wm) if args.e2e else None
+    e2e = e2e_arm(fb, dw, K, Wm) if (args.e2e and dw.sparse_layer is None) else None
     res = dict(
         metric=METRIC, value=value, unit="steps/s", n_gpus=world, steps=K, warmup=Wm,
         ms_per_step=t_max / K, higher_is_better=True, scaling="weak", vs_baseline=None,
@@ -300,9 +349,11 @@ def device_arm(args, rank, world):
                     l2="flushed between timed steps, outside the step events: 256 MiB write then 256 MiB read "
                        "(the read evicts the write's dirty lines)",
                     parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
-        roofline=dict(bound="hbm", kernel=("pass_bf16_kernel" if w.dtype == "bf16" else "pass_f32_kernel")
-                      + (" (fused step: gate + prefix split-KV pass + in-block + merge), recompute launches"
-                         if w.block <= 64 else " (prefix split-KV pass)"),
+        roofline=dict(bound="hbm", kernel=("sparse step (page estimate + top-k + sparse_pass_kernel), recompute steps"
+                                           if dw.sparse_layer is not None else
+                                           ("pass_bf16_kernel" if w.dtype == "bf16" else "pass_f32_kernel")
+                                           + (" (fused step: gate + prefix split-KV pass + in-block + merge), "
+                                              "recompute launches" if w.block <= 64 else " (prefix split-KV pass)")),
                       achieved=achieved, peak=hbm, unit="GB/s",
                       frac=(achieved / hbm) if achieved else None,
                       peak_source=f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
@@ -318,12 +369,23 @@ def device_arm(args, rank, world):
                        dense_steps_per_s=(1e3 / statistics.mean(dense_ms)) if dense_ms else None,
                        wall_s=wall),
         gpu_launches=dw.launches_per_step() * K,
+        sparse=None if dw.sparse_layer is None else dict(
+            n_select=dw.sparse_layer.sparse.n_select, pages=dw.sparse_layer.n_pages, union_density=dw.union_density(),
+            reuse_step_gbs=(alg_reuse * len(reuse_steps)) / (sum(step_ms[i] for i in reuse_steps) / 1e3) / 1e9
+            if reuse_steps else None),
         clocks=clocks.summary(),
         kernel_source_sha=kernel_source_hash(),
     )
     if e2e:
         res["e2e"] = e2e
     return res
+
+
+def sparse_n_select(w: W.Workload) -> int:
+    """k = ceil(density * pages), density read as the exact decimal it is written as."""
+    from fractions import Fraction
+    pages = (w.n_prefix + w.page_size - 1) // w.page_size
+    return min(pages, max(1, math.ceil(Fraction(str(w.density)) * pages)))
 
 
 def _mean_us(ms, idx):
@@ -393,15 +455,20 @@ def oracle_steps(w: W.Workload, seed: int, budget_s: float, max_steps: int, kv_g
     """Time the CPU oracle's cached step on the workload, restricted to the first
     `kv_groups` KV-head groups (a bounded sample).  Returns (steps, seconds,
     scale) where scale converts the sample's time to a whole-layer step."""
-    import numpy as np
     from oracle import flashblock as OF
+    from oracle import sparse as OS
     k, v = W.prefix_kv(w, seed)
     hk = min(kv_groups, w.h_kv)
     hq = hk * w.group
     kk = k[:, :hk].double().numpy()
     vv = v[:, :hk].double().numpy()
     del k, v
-    st = OF.CachedBlockAttention(kk, vv, hq, 1 / math.sqrt(w.head_dim))
+    if w.page_size:
+        sp = OS.SparseResidualAttention(kk, vv, hq, 1 / math.sqrt(w.head_dim), w.page_size, w.density)
+        st = type("SparseStep", (), {"step": staticmethod(
+            lambda q, kb, vb, mask, first, tau, sim, gamma: sp.step(q, kb, vb, mask, first, tau))})()
+    else:
+        st = OF.CachedBlockAttention(kk, vv, hq, 1 / math.sqrt(w.head_dim))
     sched = list(W.block_schedule(w, seed))
     conv = [(s.q[:, :hq].double().numpy(), s.k_blk[:, :hk].double().numpy(), s.v_blk[:, :hk].double().numpy(),
              s.mask.numpy(), s.first, None if s.sim is None else s.sim[:, :hq].numpy()) for s in sched]

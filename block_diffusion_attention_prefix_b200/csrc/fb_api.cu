@@ -73,10 +73,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 struct MapKey {
   const void* base;
   long long keys, row_stride, head_stride;
-  int D, bh;
+  int D, bh, box_rows;
   bool operator==(const MapKey& o) const {
     return base == o.base && keys == o.keys && row_stride == o.row_stride && head_stride == o.head_stride &&
-           D == o.D && bh == o.bh;
+           D == o.D && bh == o.bh && box_rows == o.box_rows;
   }
 };
 constexpr int kMapCache = 16;
@@ -85,14 +85,14 @@ CUtensorMap g_map_vals[kMapCache];
 int g_map_used = 0, g_map_next = 0;
 
 int encode_kv_map_uncached(CUtensorMap* m, const void* base, int D, long long keys, long long row_stride,
-                           long long head_stride, int bh);
+                           long long head_stride, int bh, int box_rows);
 
-// 3-D map over a bf16 KV tensor: (D, keys, b*H_kv), box (64, 64, 1), 128-B swizzle.
+// 3-D map over a bf16 KV tensor: (D, keys, b*H_kv), box (64, box_rows, 1), 128-B swizzle.
 int encode_kv_map(CUtensorMap* m, const void* base, int D, long long keys, long long row_stride,
-                  long long head_stride, int bh) {
+                  long long head_stride, int bh, int box_rows = 64) {
   std::memset(m, 0, sizeof(*m));
   if (keys == 0) return FB_OK;  // never loaded
-  const MapKey key{base, keys, row_stride, head_stride, D, bh};
+  const MapKey key{base, keys, row_stride, head_stride, D, bh, box_rows};
   {
     std::lock_guard<std::mutex> lk(g_mu);
     for (int i = 0; i < g_map_used; ++i)
@@ -101,7 +101,7 @@ int encode_kv_map(CUtensorMap* m, const void* base, int D, long long keys, long 
         return FB_OK;
       }
   }
-  const int st = encode_kv_map_uncached(m, base, D, keys, row_stride, head_stride, bh);
+  const int st = encode_kv_map_uncached(m, base, D, keys, row_stride, head_stride, bh, box_rows);
   if (st != FB_OK) return st;
   std::lock_guard<std::mutex> lk(g_mu);
   const int slot = g_map_used < kMapCache ? g_map_used++ : (g_map_next++ % kMapCache);
@@ -111,11 +111,11 @@ int encode_kv_map(CUtensorMap* m, const void* base, int D, long long keys, long 
 }
 
 int encode_kv_map_uncached(CUtensorMap* m, const void* base, int D, long long keys, long long row_stride,
-                           long long head_stride, int bh) {
+                           long long head_stride, int bh, int box_rows) {
   if (!get_encoder()) return FB_ERR_CUDA;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)keys, (cuuint64_t)bh};
   cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, (cuuint64_t)head_stride * 2};
-  cuuint32_t box[3] = {64, 64, 1};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -484,6 +484,168 @@ int fb_step(const fb_shape* shape, const void* q, const void* k_cache, const voi
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Sparse attention with a cached residual.
+namespace fb {
+namespace {
+
+constexpr int kSparsePage = 16;
+
+struct SparseLayout {
+  SplitPlan plan;
+  int P, words;
+  size_t counters, part_sel, part_res, inblock, est, total;
+};
+
+int sparse_layout(const Dims& d, int sms, SparseLayout* L) {
+  L->plan = plan_split(d.R, d.D, d.N, d.b, d.hkv, FB_BF16, sms, true);
+  L->P = (int)((d.N + kSparsePage - 1) / kSparsePage);
+  L->words = (L->P + 31) / 32;
+  const size_t units = (size_t)d.b * d.hkv * L->plan.n_row_tiles;
+  const size_t part = units * L->plan.splits * L->plan.row_tile * (d.D + 4) * sizeof(float);
+  L->counters = 0;
+  L->part_sel = L->plan.counter_bytes;
+  L->part_res = L->part_sel + part;
+  L->inblock = L->part_res + part;
+  L->est = L->inblock + (units * L->plan.row_tile * (d.D + 4) * sizeof(float) + 255) / 256 * 256;
+  L->total = L->est + (size_t)d.b * d.hq * d.B * L->P * sizeof(double);
+  return FB_OK;
+}
+
+int sparse_check(const fb_shape* shape, const fb_gate* gate, const fb_sparse* sp, Dims* d, GateParams* gp) {
+  FB_TRY(resolve(shape, d));
+  if (!sp) return FB_ERR_NULL;
+  if (d->dtype != FB_BF16) return FB_ERR_DTYPE;
+  if (sp->page_size != kSparsePage) return FB_ERR_ARG;
+  if (d->N < 1 || d->B > kSmallBlockMax || d->R > 32) return FB_ERR_UNSUPPORTED;
+  const long long P = (d->N + kSparsePage - 1) / kSparsePage;
+  if (sp->n_select < 1 || sp->n_select > P) return FB_ERR_ARG;
+  if ((P + 31) / 32 > 12288) return FB_ERR_UNSUPPORTED;  // row bitmap must fit in shared memory
+  if (gate && gate->head_sim) return FB_ERR_UNSUPPORTED;  // tau gate only
+  FB_TRY(check_ptr(sp->kmin));
+  FB_TRY(check_ptr(sp->kmax));
+  FB_TRY(check_ptr(sp->sel_idx));
+  FB_TRY(check_ptr(sp->sel_bits));
+  FB_TRY(check_ptr(sp->union_bits));
+  FB_TRY(check_ptr(sp->a_res));
+  FB_TRY(check_ptr(sp->l_res));
+  if (sp->a_sel) FB_TRY(check_ptr(sp->a_sel));
+  return gate_params(gate, *d, gp);
+}
+
+int sparse_args(const Dims& d, const GateParams& gp, const fb_sparse* sp, const void* q, void* ws,
+                size_t ws_bytes, SparseArgs* a) {
+  if (!ws) return FB_ERR_WORKSPACE;
+  if (!aligned16(ws)) return FB_ERR_ALIGN;
+  const int dev = current_device();
+  if (dev < 0) return FB_ERR_CUDA;
+  const int sms = device_sms(dev);
+  uint32_t* err = device_err(dev);
+  if (!sms || !err) return FB_ERR_CUDA;
+  SparseLayout L;
+  sparse_layout(d, sms, &L);
+  if (ws_bytes < L.total) return FB_ERR_WORKSPACE;
+  if (!sparse_supported(d.D, L.plan.row_tile)) return FB_ERR_UNSUPPORTED;
+  std::memset(a, 0, sizeof(*a));
+  a->d = d;
+  a->plan = L.plan;
+  a->P = L.P;
+  a->k_sel = sp->n_select;
+  a->words = L.words;
+  a->q = q;
+  a->kmin = static_cast<const __nv_bfloat16*>(sp->kmin);
+  a->kmax = static_cast<const __nv_bfloat16*>(sp->kmax);
+  char* w = static_cast<char*>(ws);
+  a->counters = reinterpret_cast<unsigned int*>(w + L.counters);
+  a->part_sel = reinterpret_cast<float*>(w + L.part_sel);
+  a->part_res = reinterpret_cast<float*>(w + L.part_res);
+  a->inblock = reinterpret_cast<float*>(w + L.inblock);
+  a->est = reinterpret_cast<double*>(w + L.est);
+  a->sel_idx = sp->sel_idx;
+  a->sel_bits = sp->sel_bits;
+  a->union_bits = sp->union_bits;
+  a->gate = gp;
+  a->a_res = sp->a_res;
+  a->l_res = sp->l_res;
+  a->a_sel = sp->a_sel;
+  a->l_sel = sp->l_sel;
+  a->err = err;
+  return FB_OK;
+}
+
+}  // namespace
+}  // namespace fb
+
+extern "C" int fb_page_minmax(const fb_shape* shape, const void* k_cache, int page_size, void* kmin, void* kmax,
+                              fb_stream_t stream) {
+  Dims d;
+  FB_TRY(resolve(shape, &d));
+  if (d.dtype != FB_BF16) return FB_ERR_DTYPE;
+  if (page_size != kSparsePage) return FB_ERR_ARG;
+  if (d.N < 1) return FB_ERR_UNSUPPORTED;
+  FB_TRY(check_ptr(k_cache));
+  FB_TRY(check_ptr(kmin));
+  FB_TRY(check_ptr(kmax));
+  SparseArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.d = d;
+  a.P = (int)((d.N + kSparsePage - 1) / kSparsePage);
+  a.k = k_cache;
+  a.kmin_out = static_cast<__nv_bfloat16*>(kmin);
+  a.kmax_out = static_cast<__nv_bfloat16*>(kmax);
+  return cuda_status(launch_page_minmax(a, (cudaStream_t)stream));
+}
+
+extern "C" size_t fb_sparse_workspace_bytes(const fb_shape* shape, int page_size) {
+  Dims d;
+  if (resolve(shape, &d) != FB_OK || page_size != kSparsePage) return 0;
+  const int dev = current_device();
+  const int sms = dev >= 0 ? device_sms(dev) : 0;
+  SparseLayout L;
+  sparse_layout(d, sms > 0 ? sms : 148, &L);
+  return L.total;
+}
+
+extern "C" int fb_sparse_select(const fb_shape* shape, const void* q, const fb_gate* gate, const fb_sparse* sp,
+                                void* ws, size_t ws_bytes, fb_stream_t stream) {
+  Dims d;
+  GateParams gp;
+  FB_TRY(sparse_check(shape, gate, sp, &d, &gp));
+  FB_TRY(check_ptr(q));
+  SparseArgs a;
+  FB_TRY(sparse_args(d, gp, sp, q, ws, ws_bytes, &a));
+  return cuda_status(launch_sparse_select(a, (cudaStream_t)stream));
+}
+
+extern "C" int fb_sparse_step(const fb_shape* shape, const void* q, const void* k_cache, const void* v_cache,
+                              const void* k_blk, const void* v_blk, const fb_gate* gate, const fb_sparse* sp,
+                              void* a_full, float* l_full, int32_t* dec_M, uint8_t* dec_reuse, void* ws,
+                              size_t ws_bytes, fb_stream_t stream) {
+  Dims d;
+  GateParams gp;
+  FB_TRY(sparse_check(shape, gate, sp, &d, &gp));
+  FB_TRY(check_ptr(q));
+  FB_TRY(check_ptr(k_cache));
+  FB_TRY(check_ptr(v_cache));
+  FB_TRY(check_ptr(k_blk));
+  FB_TRY(check_ptr(v_blk));
+  FB_TRY(check_ptr(a_full));
+  SparseArgs a;
+  FB_TRY(sparse_args(d, gp, sp, q, ws, ws_bytes, &a));
+  a.step.enabled = 1;
+  a.step.k_blk = k_blk;
+  a.step.v_blk = v_blk;
+  a.step.a_full = a_full;
+  a.step.l_full = l_full;
+  a.step.dec_M = dec_M;
+  a.step.dec_reuse = dec_reuse;
+  CUtensorMap tk, tv;
+  FB_TRY(encode_kv_map(&tk, k_cache, d.D, d.N, d.row_stride, d.head_stride, d.b * d.hkv, kSparsePage));
+  FB_TRY(encode_kv_map(&tv, v_cache, d.D, d.N, d.row_stride, d.head_stride, d.b * d.hkv, kSparsePage));
+  FB_TRY(cuda_status(launch_sparse_select(a, (cudaStream_t)stream)));
+  return cuda_status(launch_sparse_pass(a, tk, tv, (cudaStream_t)stream));
+}
 
 // ---------------------------------------------------------------------------
 // fb_prefix_attn_noalloc: the prefix pass with its split-KV workspace in a

@@ -385,55 +385,44 @@ __device__ __forceinline__ void record_decisions(const GateParams& g, const Dims
   if (write_M && dec_M && tid == 0) dec_M[b] = M;
 }
 
-// Finish one (b, kv head, row tile) in the CTA that arrived last: merge the
-// `splits` partials in fixed split order (deterministic) and write the results.
-// Partials are [splits][RT][D + 4] fp32 (A normalised in cols 0..D-1, natural-log
-// L in col D), contiguous in global memory.
-//   1. 1-D bulk TMA copies bring the partials into shared memory (chunks of as many
-//      splits as fit), together with the tile's in-block slot in a fused step;
+// Combine the `splits` partials of one (b, kv head, row tile) in fixed split
+// order (deterministic), in the CTA that arrived last.  Partials are
+// [splits][RT][D + 4] fp32 (A normalised in cols 0..D-1, natural-log L in col D),
+// contiguous in global memory.
+//   1. 1-D bulk TMA copies bring the partials into `buf` (chunks of as many splits
+//      as fit) -- plus, with the first chunk, `in_slot` into `s_in` when given;
 //      meanwhile every thread loads a share of the L values.
 //   2. Per row, the split weights w_s = e^{L_s - M} / sum_s e^{L_s - M} and the
-//      merged L = M + ln sum_s e^{L_s - M} are computed once (the FlashBlock merge
-//      equation over all splits).
-//   3. Each thread accumulates sum_s w_s A_s for its (row, 4-column) items, then
-//      - rows flagged for recompute go through `ep` (mode 0: write the cache rows;
-//        mode 1: merge with the cache into A_full);
-//      - fused step (`step_ep` != nullptr): A_full = merge(cache row, in-block
-//        row), the cache row being the one just combined (flagged rows) or the
-//        cached one (rows of reusing heads in a mixed tile).
-// Executed by threads [0, NT) with barrier `bar_id`; `buf` is `buf_bytes` of
-// 1024-byte aligned shared memory; `mbar` an initialised mbarrier (count 1) whose
-// next phase has parity `*phase`.
+//      merged L = M + ln sum_s e^{L_s - M} (the FlashBlock merge equation over all
+//      splits) are computed once; s_L[r] gets the merged L.
+//   3. Each thread accumulates sum_s w_s A_s for its (row, 4-column) items in two
+//      chains split by the parity of the split index (order independent of the
+//      chunking); A[k] gets the result for item k = tid + k * NT.
+// Threads [0, NT), barrier `bar_id`; `buf` is `buf_bytes` of 128-byte aligned
+// shared memory; `mbar` an initialised mbarrier (count 1) whose next phase has
+// parity `*phase`.  Returns false if a bounded wait ran out (same on all threads).
 template <int D, int RT, int NT>
-__device__ void finish_tile(const float* part, int splits, const float* inblock_slot, int rows_valid,
-                            const int* s_flags, size_t grow0, const Epilogue& ep, const Epilogue* step_ep,
-                            uint8_t* buf, int buf_bytes, uint64_t* mbar, uint32_t* phase, uint32_t* err, int tid,
-                            int bar_id) {
+__device__ bool combine_regs(const float* part, int splits, const float* in_slot, float* s_in, uint8_t* buf,
+                             int buf_bytes, uint64_t* mbar, uint32_t* phase, uint32_t* err, int tid, int bar_id,
+                             float4 (&A)[(RT * (D / 4) + NT - 1) / NT], float* s_L) {
   constexpr int RS = D + 4;
   constexpr int SPLIT_FLOATS = RT * RS;
   constexpr int D4 = D / 4;
   constexpr int IT = (RT * D4 + NT - 1) / NT;
-  const bool step = step_ep != nullptr;
-  const int in_bytes = step ? (SPLIT_FLOATS * 4 + 127) / 128 * 128 : 0;
-  const int w_bytes = ((splits + 4) * RT * 4 + 127) / 128 * 128;
-  float* s_in = reinterpret_cast<float*>(buf);
-  // [splits][RT] split weights, then per row: merged L, 1/den, and (fused step) the
-  // weights of the cache row and of the in-block row in the final merge.
-  float* sW = reinterpret_cast<float*>(buf + in_bytes);
-  float* sLf = sW + (size_t)splits * RT;
-  float* sWo = sLf + RT;
-  float* sWi = sWo + RT;
-  float* chunk = reinterpret_cast<float*>(buf + in_bytes + w_bytes);
-  const int cs = (buf_bytes - in_bytes - w_bytes) / (SPLIT_FLOATS * 4);
+  const int w_bytes = ((splits + 2) * RT * 4 + 127) / 128 * 128;
+  float* sW = reinterpret_cast<float*>(buf);  // [splits][RT] weights, then [RT] 1/den
+  float* sInv = sW + (size_t)splits * RT;
+  float* chunk = reinterpret_cast<float*>(buf + w_bytes);
+  const int cs = (buf_bytes - w_bytes) / (SPLIT_FLOATS * 4);
 
   auto issue = [&](int c0) {
     const int nsp = min(cs, splits - c0);
     const uint32_t bytes = (uint32_t)nsp * SPLIT_FLOATS * 4;
-    const bool with_in = step && c0 == 0;
+    const bool with_in = in_slot != nullptr && c0 == 0;
     fence_proxy_async_global();
     mbar_arrive_expect_tx(mbar, bytes + (with_in ? (uint32_t)SPLIT_FLOATS * 4 : 0u));
     bulk_load(chunk, part + (size_t)c0 * SPLIT_FLOATS, bytes, mbar);
-    if (with_in) bulk_load(s_in, inblock_slot, (uint32_t)SPLIT_FLOATS * 4, mbar);
+    if (with_in) bulk_load(s_in, in_slot, (uint32_t)SPLIT_FLOATS * 4, mbar);
   };
   if (tid == 0) issue(0);
   for (int i = tid; i < splits * RT; i += NT) {
@@ -441,36 +430,28 @@ __device__ void finish_tile(const float* part, int splits, const float* inblock_
     sW[i] = __ldcg(part + (size_t)sp * SPLIT_FLOATS + (size_t)r * RS + D);
   }
   named_barrier_sync(bar_id, NT);
-  // Per row: M = max_s L_s (kept in sLf for now).
-  for (int r = tid; r < RT; r += NT) {
+  for (int r = tid; r < RT; r += NT) {  // per row: M = max_s L_s
     float M = -CUDART_INF_F;
     for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, sW[sp * RT + r]);
-    sLf[r] = M;
+    s_L[r] = M;
   }
   named_barrier_sync(bar_id, NT);
-  // All (split, row) pairs in parallel: e = e^{L_s - M}.
-  for (int i = tid; i < splits * RT; i += NT) {
-    const int r = i % RT;
-    const float M = sLf[r];
+  for (int i = tid; i < splits * RT; i += NT) {  // all (split, row) pairs: e = e^{L_s - M}
+    const float M = s_L[i % RT];
     sW[i] = M == -CUDART_INF_F ? 0.f : expf(sW[i] - M);
   }
   named_barrier_sync(bar_id, NT);
-  // Per row: den, merged L, and the final-merge weights of a fused step.
-  for (int r = tid; r < RT; r += NT) {
-    const float M = sLf[r];
+  for (int r = tid; r < RT; r += NT) {  // per row: den, merged L
     float den = 0.f;
     for (int sp = 0; sp < splits; ++sp) den += sW[sp * RT + r];
-    const float L = den > 0.f ? M + logf(den) : -CUDART_INF_F;
-    sLf[r] = L;
-    sWo[r] = den > 0.f ? 1.f / den : 0.f;  // scale of the accumulated sum_s e_s A_s
+    s_L[r] = den > 0.f ? s_L[r] + logf(den) : -CUDART_INF_F;
+    sInv[r] = den > 0.f ? 1.f / den : 0.f;
   }
   named_barrier_sync(bar_id, NT);
 
-  // Two accumulation chains per item, by the parity of the global split index, so
-  // that the summation order never depends on how the splits were chunked.
-  float4 acc[IT], acc1[IT];
+  float4 acc1[IT];
 #pragma unroll
-  for (int k = 0; k < IT; ++k) acc[k] = acc1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = 0; k < IT; ++k) A[k] = acc1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
   bool ok = true;
   for (int c0 = 0; c0 < splits && ok; c0 += cs) {
     const int nsp = min(cs, splits - c0);
@@ -488,7 +469,7 @@ __device__ void finish_tile(const float* part, int splits, const float* inblock_
           for (int sp = 0; sp < nsp; ++sp) {
             const float w = wr[sp * RT];
             const float4 x = *reinterpret_cast<const float4*>(pr + (size_t)sp * SPLIT_FLOATS);
-            float4& a = ((c0 + sp) & 1) ? acc1[k] : acc[k];
+            float4& a = ((c0 + sp) & 1) ? acc1[k] : A[k];
             a.x = fmaf(w, x.x, a.x);
             a.y = fmaf(w, x.y, a.y);
             a.z = fmaf(w, x.z, a.z);
@@ -501,31 +482,72 @@ __device__ void finish_tile(const float* part, int splits, const float* inblock_
   }
 #pragma unroll
   for (int k = 0; k < IT; ++k) {
-    acc[k].x += acc1[k].x;
-    acc[k].y += acc1[k].y;
-    acc[k].z += acc1[k].z;
-    acc[k].w += acc1[k].w;
+    const int idx = tid + k * NT;
+    const float sc = idx < RT * D4 ? sInv[idx / D4] : 0.f;
+    A[k] = make_float4((A[k].x + acc1[k].x) * sc, (A[k].y + acc1[k].y) * sc, (A[k].z + acc1[k].z) * sc,
+                       (A[k].w + acc1[k].w) * sc);
   }
-  // Fused step: per row, the weights of the cache row (w_o) and of the in-block row
-  // (w_i) in A_full = w_o A_out + w_i A_in, and L_full.  Rows of reusing heads in a
-  // mixed tile take the cached (A_out, L_out) instead of the combined one.
+  named_barrier_sync(bar_id, NT);  // sInv is read above; `buf` may be reused after this
+  return ok;
+}
+
+// Per-row weights of the FlashBlock merge of two (A, L) parts: w1 = e^{L1-m}/den,
+// w2 = e^{L2-m}/den and L = m + ln den (both empty: 0, 0, -inf).
+__device__ __forceinline__ void merge_weights(float l1, float l2, float& w1, float& w2, float& l) {
+  const float m = fmaxf(l1, l2);
+  if (m == -CUDART_INF_F) {
+    w1 = w2 = 0.f;
+    l = -CUDART_INF_F;
+    return;
+  }
+  w1 = expf(l1 - m);
+  w2 = expf(l2 - m);
+  const float den = w1 + w2;
+  l = m + logf(den);
+  w1 /= den;
+  w2 /= den;
+}
+
+__device__ __forceinline__ float4 wsum4(float w1, float4 a, float w2, float4 b) {
+  return make_float4(w1 * a.x + w2 * b.x, w1 * a.y + w2 * b.y, w1 * a.z + w2 * b.z, w1 * a.w + w2 * b.w);
+}
+
+// Finish one (b, kv head, row tile) of a dense pass in the CTA that arrived last:
+// combine its splits (combine_regs), then
+//   - rows flagged for recompute: the combined (A, L) goes through `ep`
+//     (mode 0: write the cache rows; mode 1: merge with the cache into A_full);
+//   - fused step (`step_ep` != nullptr): A_full = merge(cache row, in-block row),
+//     the cache row being the one just combined (flagged rows) or the cached one
+//     (rows of reusing heads in a mixed tile); the in-block rows come from the
+//     tile's slot `inblock_slot` in the workspace.
+// `buf` (1024-byte aligned, `buf_bytes`) holds the in-block slot, per-row scalars
+// and the combine's buffer.
+template <int D, int RT, int NT>
+__device__ void finish_tile(const float* part, int splits, const float* inblock_slot, int rows_valid,
+                            const int* s_flags, size_t grow0, const Epilogue& ep, const Epilogue* step_ep,
+                            uint8_t* buf, int buf_bytes, uint64_t* mbar, uint32_t* phase, uint32_t* err, int tid,
+                            int bar_id) {
+  constexpr int RS = D + 4;
+  constexpr int D4 = D / 4;
+  constexpr int IT = (RT * D4 + NT - 1) / NT;
+  const bool step = step_ep != nullptr;
+  const int in_bytes = step ? (RT * RS * 4 + 127) / 128 * 128 : 0;
+  float* s_in = reinterpret_cast<float*>(buf);
+  float* s_L = reinterpret_cast<float*>(buf + in_bytes);  // [RT] merged L, then [RT] w_o, [RT] w_i
+  float* s_wo = s_L + RT;
+  float* s_wi = s_wo + RT;
+  const int hdr = in_bytes + (3 * RT * 4 + 127) / 128 * 128;
+  float4 A[IT];
+  combine_regs<D, RT, NT>(part, splits, step ? inblock_slot : nullptr, s_in, buf + hdr, buf_bytes - hdr, mbar,
+                          phase, err, tid, bar_id, A, s_L);
   if (step) {
     for (int r = tid; r < rows_valid; r += NT) {
-      const float lo = s_flags[r] ? sLf[r] : __ldcg(step_ep->l_prev + grow0 + r);
-      const float li = s_in[(size_t)r * RS + D];
-      const float m = fmaxf(lo, li);
-      float wo = 0.f, wi = 0.f, lf = -CUDART_INF_F;
-      if (m != -CUDART_INF_F) {
-        wo = expf(lo - m);
-        wi = expf(li - m);
-        const float den = wo + wi;
-        lf = m + logf(den);
-        wo /= den;
-        wi /= den;
-      }
+      const float lo = s_flags[r] ? s_L[r] : __ldcg(step_ep->l_prev + grow0 + r);
+      float wo, wi, lf;
+      merge_weights(lo, s_in[(size_t)r * RS + D], wo, wi, lf);
       if (step_ep->l_full) step_ep->l_full[grow0 + r] = lf;
-      sWi[r] = wi;
-      sW[r] = wo;  // split weights are no longer needed
+      s_wo[r] = wo;
+      s_wi[r] = wi;
     }
     named_barrier_sync(bar_id, NT);
   }
@@ -535,18 +557,13 @@ __device__ void finish_tile(const float* part, int splits, const float* inblock_
     if (idx >= RT * D4) continue;
     const int r = idx / D4, d4 = idx - r * D4;
     if (r >= rows_valid) continue;
-    const float sc = sWo[r];
-    const float4 A = make_float4(acc[k].x * sc, acc[k].y * sc, acc[k].z * sc, acc[k].w * sc);
     const size_t grow = grow0 + r;
-    if (s_flags[r]) epilogue4(ep, D, grow, d4, A, sLf[r]);
+    if (s_flags[r]) epilogue4(ep, D, grow, d4, A[k], s_L[r]);
     if (step) {
       const size_t off = grow * D + (size_t)d4 * 4;
-      const float4 ap = s_flags[r] ? A : __ldcg(reinterpret_cast<const float4*>(step_ep->a_prev + off));
+      const float4 ap = s_flags[r] ? A[k] : __ldcg(reinterpret_cast<const float4*>(step_ep->a_prev + off));
       const float4 ai = *reinterpret_cast<const float4*>(s_in + (size_t)r * RS + d4 * 4);
-      const float wo = sW[r], wi = sWi[r];
-      const float4 af = make_float4(wo * ap.x + wi * ai.x, wo * ap.y + wi * ai.y, wo * ap.z + wi * ai.z,
-                                    wo * ap.w + wi * ai.w);
-      store4(step_ep->a_full, off, af, step_ep->out_bf16);
+      store4(step_ep->a_full, off, wsum4(s_wo[r], ap, s_wi[r], ai), step_ep->out_bf16);
     }
   }
 }

@@ -5,6 +5,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -91,6 +92,40 @@ struct PassArgs {
   float* inblock;         // workspace, fused step only
   uint32_t* err;          // device error word
 };
+
+// Page-sparse attention with a cached residual (sparse.cu).
+struct SparseArgs {
+  Dims d;                 // N = prefix tokens
+  SplitPlan plan;         // splits over 64-key (4-page) tiles
+  int P;                  // pages (16 tokens each)
+  int k_sel;              // pages selected per query row
+  int words;              // ceil(P / 32)
+  const void* q;
+  const void* k;          // prefix K (page bounds only)
+  const __nv_bfloat16* kmin;   // [b*H_kv][D][P]
+  const __nv_bfloat16* kmax;
+  __nv_bfloat16* kmin_out;     // page bounds output
+  __nv_bfloat16* kmax_out;
+  double* est;            // workspace [b*H_q*B][P]
+  int32_t* sel_idx;       // [b*H_q*B][k_sel] ascending
+  uint32_t* sel_bits;     // [b*H_q*B][words]
+  uint32_t* union_bits;   // [b*H_kv][words]
+  GateParams gate;        // tau only
+  float* a_res;           // residual cache [b, H_q, B, D] / [b, H_q, B]
+  float* l_res;
+  float* a_sel;           // optional
+  float* l_sel;
+  StepArgs step;          // in-block, A_full, L_full, decisions
+  unsigned int* counters; // workspace
+  float* part_sel;
+  float* part_res;
+  float* inblock;
+  uint32_t* err;
+};
+int sparse_supported(int D, int row_tile);
+cudaError_t launch_page_minmax(const SparseArgs& a, cudaStream_t s);
+cudaError_t launch_sparse_select(const SparseArgs& a, cudaStream_t s);
+cudaError_t launch_sparse_pass(const SparseArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s);
 
 SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int num_sms,
                      bool with_inblock = false);

@@ -66,8 +66,8 @@ struct Cfg {
   static constexpr int kSmemBytes = (kRingBytes > kScratchBytes ? kRingBytes : kScratchBytes) + 1024;
   static_assert(KW % 16 == 0, "each warp needs whole k16 steps of keys");
   static_assert(D % 64 == 0, "D must be a multiple of 64");
-  // Finisher: in-block slot + weights of up to 148 splits + at least one split's partial.
-  static_assert(kRingBytes >= 2 * kRowTile * (D + 4) * 4 + 128 + ((152 * kRowTile * 4 + 127) / 128) * 128,
+  // Finisher: in-block slot + per-row scalars + weights of up to 148 splits + one split's partial.
+  static_assert(kRingBytes >= 2 * kRowTile * (D + 4) * 4 + 256 + 3 * kRowTile * 4 + ((150 * kRowTile * 4 + 127) / 128) * 128,
                 "finisher needs the in-block slot, the weights and one split");
 };
 

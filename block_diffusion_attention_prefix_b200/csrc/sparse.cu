@@ -1,0 +1,821 @@
+// sparse.cu -- page-sparse attention with a cached residual (sm_100a).
+//
+// FlashBlock technical summary (gist.science 2602.05305), "Adaptive reuse
+// strategies / compatibility with sparse attention": the keys a sparse selector
+// leaves out are treated as the out-of-block set and their attention is cached as
+// a residual; the selected keys are attended fresh every step.  The selector is a
+// per-query top-k of 16-token pages ranked by a channel-wise min/max bound (the
+// LoSA page, gist.science 2604.12056, names QUEST as its selector):
+//     e_p = sum_d max(q_d kmin_{p,d}, q_d kmax_{p,d}),
+// summed in float64 in ascending d (each bf16 x bf16 product is exact in
+// float64, so any implementation summing in that order gets the same bits), top
+// k = ceil(density * pages) by (e desc, page asc).
+//
+// Kernels:
+//  * page_minmax_kernel: kmin / kmax [b*H_kv][D][pages] (channel-major so that
+//    the estimate reads coalesce), exact bf16.
+//  * page_estimate_kernel: e for every (row, page) of recomputing batch
+//    elements; one thread per page runs the 16 rows' float64 DFMA chains
+//    (max(q kmin, q kmax) is the product picked by the sign of q, exactly).
+//  * topk_kernel: one CTA per row: radix select of the k-th key on an
+//    order-preserving 64-bit key, tie ranks and compaction in page order ->
+//    sorted page list, row bitmap, union bitmap of the KV group (atomicOr).
+//  * sparse_pass_kernel: the TMA + mma.sync split pipeline of the dense pass
+//    with page-granular loads (16-key boxes).  Recompute step: every page, two
+//    online softmaxes per row (selected pages -> fresh part, other pages ->
+//    residual).  Reuse step: only the union pages of the KV group, selected part
+//    only (rows mask the union pages they did not select).  The finishing CTA
+//    combines the splits, writes the residual cache (recompute) and
+//    A_full = merge(merge(A_sel, A_res), A_in) with the in-block rows computed by
+//    the aux warps.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "fb_device.cuh"
+#include "fb_internal.h"
+#include "fb_ptx.cuh"
+
+namespace fb {
+namespace {
+
+using bf16 = __nv_bfloat16;
+constexpr int kPage = 16;
+constexpr int kTilePages = 4;  // 64 keys per pipeline tile
+
+__device__ __forceinline__ bool sparse_recompute(const GateParams& g, int b, int B, int* s_red) {
+  if (!g.enabled) return true;
+  const int M = block_updated_count(g.mask + (size_t)b * B, B, s_red);
+  return !tau_reuse(g, M);
+}
+
+// ------------------------------------------------------------------ page bounds
+
+template <int D>
+__global__ void __launch_bounds__(32 * (D / 16)) page_minmax_kernel(const SparseArgs a) {
+  const int lane = threadIdx.x & 31, chunk = threadIdx.x >> 5;  // 16 channels per warp
+  const int bg = blockIdx.y;
+  const int p = blockIdx.x * 32 + lane;
+  if (p >= a.P) return;
+  const bf16* kp = static_cast<const bf16*>(a.k) + (size_t)bg * a.d.head_stride +
+                   (size_t)p * kPage * a.d.row_stride + chunk * 16;
+  const long long kend = min((long long)kPage, a.d.N - (long long)p * kPage);
+  float mn[16], mx[16];
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    mn[t] = CUDART_INF_F;
+    mx[t] = -CUDART_INF_F;
+  }
+  for (int j = 0; j < kend; ++j) {
+    const uint4* src = reinterpret_cast<const uint4*>(kp + (size_t)j * a.d.row_stride);
+    const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
+    const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t]));
+      mn[2 * t] = fminf(mn[2 * t], f.x);
+      mx[2 * t] = fmaxf(mx[2 * t], f.x);
+      mn[2 * t + 1] = fminf(mn[2 * t + 1], f.y);
+      mx[2 * t + 1] = fmaxf(mx[2 * t + 1], f.y);
+    }
+  }
+  bf16* omn = a.kmin_out + (size_t)bg * D * a.P + (size_t)(chunk * 16) * a.P + p;
+  bf16* omx = a.kmax_out + (size_t)bg * D * a.P + (size_t)(chunk * 16) * a.P + p;
+#pragma unroll
+  for (int t = 0; t < 16; ++t) {
+    omn[(size_t)t * a.P] = __float2bfloat16_rn(mn[t]);  // exact: the inputs are bf16
+    omx[(size_t)t * a.P] = __float2bfloat16_rn(mx[t]);
+  }
+}
+
+// ------------------------------------------------------------------ page estimates
+
+constexpr int kEstThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kEstThreads) page_estimate_kernel(const SparseArgs a) {
+  extern __shared__ double sq[];  // [R rounded up to 16][D] float64 copies of the group's q rows
+  __shared__ int s_red[32];
+  const Dims& d = a.d;
+  const int bg = blockIdx.y, b = bg / d.hkv, kvh = bg - b * d.hkv;
+  if (!sparse_recompute(a.gate, b, d.B, s_red)) return;
+  const int R = d.R, Rp = (R + 15) / 16 * 16;
+  const int p0 = blockIdx.x * kEstThreads, p = p0 + threadIdx.x;
+  // The union of the group is rebuilt by topk_kernel: clear this chunk's words.
+  if (threadIdx.x < kEstThreads / 32) {
+    const int w = p0 / 32 + threadIdx.x;
+    if (w < a.words) a.union_bits[(size_t)bg * a.words + w] = 0u;
+  }
+  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B;
+  const bf16* qg = static_cast<const bf16*>(a.q) + grow0 * D;
+  for (int i = threadIdx.x; i < Rp * D; i += kEstThreads)
+    sq[i] = i < R * D ? (double)__bfloat162float(qg[i]) : 0.0;
+  __syncthreads();
+  if (p >= a.P) return;
+  const bf16* mn = a.kmin + (size_t)bg * D * a.P + p;
+  const bf16* mx = a.kmax + (size_t)bg * D * a.P + p;
+  for (int r0 = 0; r0 < R; r0 += 16) {
+    double acc[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) acc[j] = 0.0;
+    for (int dd = 0; dd < D; ++dd) {
+      const double kmn = (double)__bfloat162float(mn[(size_t)dd * a.P]);
+      const double kmx = (double)__bfloat162float(mx[(size_t)dd * a.P]);
+      const double* qc = sq + (size_t)r0 * D + dd;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const double qv = qc[(size_t)j * D];
+        acc[j] = fma(qv, qv >= 0.0 ? kmx : kmn, acc[j]);  // exact product, one rounding
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (r0 + j < R) a.est[(grow0 + r0 + j) * (size_t)a.P + p] = acc[j];
+  }
+}
+
+// ------------------------------------------------------------------ top-k pages
+
+constexpr int kTopkThreads = 512;
+
+// Order-preserving key: ascending key <=> descending estimate (estimates are never -0).
+__device__ __forceinline__ unsigned long long desc_key(double e) {
+  const unsigned long long u = (unsigned long long)__double_as_longlong(e);
+  const unsigned long long asc = (u >> 63) ? ~u : (u | (1ull << 63));
+  return ~asc;
+}
+
+// Exclusive scan of one int per thread over the block (kTopkThreads threads).
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  __syncthreads();
+  if (lane == 31) s_tmp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int t = lane < kTopkThreads / 32 ? s_tmp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < kTopkThreads / 32) s_tmp[lane] = t;
+  }
+  __syncthreads();
+  const int before = warp > 0 ? s_tmp[warp - 1] : 0;
+  return before + x - v;
+}
+
+__global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) {
+  extern __shared__ uint32_t s_bits[];  // [words] row bitmap
+  __shared__ unsigned hist[256];
+  __shared__ int s_tmp[32];
+  __shared__ unsigned long long s_prefix;
+  __shared__ int s_kk;
+  const Dims& d = a.d;
+  const int row = blockIdx.x;
+  const int b = row / (d.hq * d.B);
+  const int h = (row / d.B) % d.hq;
+  const int kvh = h / d.G;
+  if (!sparse_recompute(a.gate, b, d.B, s_tmp)) return;
+  const int P = a.P, tid = threadIdx.x;
+  if (a.k_sel <= 0 || P <= 0) return;
+  const int per = (P + kTopkThreads - 1) / kTopkThreads;
+  const int pb = min(P, tid * per), pe = min(P, pb + per);
+  const double* est = a.est + (size_t)row * P;
+
+  // Radix select (8 passes of 8 bits, most significant first) of the k-th smallest key.
+  unsigned long long prefix = 0, mask = 0;
+  int kk = a.k_sel;
+  for (int pass = 0; pass < 8; ++pass) {
+    const int shift = 56 - 8 * pass;
+    if (tid < 256) hist[tid] = 0u;
+    __syncthreads();
+    for (int p = pb; p < pe; ++p) {
+      const unsigned long long key = desc_key(est[p]);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      unsigned c[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = hist[tid * 8 + j];
+        sum += c[j];
+      }
+      unsigned incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (tid >= o) incl += y;
+      }
+      const unsigned excl = incl - sum;
+      const unsigned long long hit = __ballot_sync(0xffffffffu, excl < (unsigned)kk && (unsigned)kk <= incl);
+      const int owner = __ffsll((long long)hit) - 1;
+      if (tid == owner) {
+        unsigned run = excl;
+        int bin = 0;
+        for (int j = 0; j < 8; ++j) {
+          if ((unsigned)kk <= run + c[j]) {
+            bin = tid * 8 + j;
+            break;
+          }
+          run += c[j];
+        }
+        s_prefix = prefix | ((unsigned long long)bin << shift);
+        s_kk = kk - (int)run;
+      }
+    }
+    __syncthreads();
+    prefix = s_prefix;
+    kk = s_kk;
+    mask |= 0xFFull << shift;
+    __syncthreads();
+  }
+  const unsigned long long T = prefix;  // the k-th smallest key; take `kk` of the keys equal to it
+
+  // Ties to T go to the lowest pages: rank them in page order, then compact.
+  int my_eq = 0;
+  for (int p = pb; p < pe; ++p) my_eq += desc_key(est[p]) == T;
+  int eq_rank = block_exclusive_scan(my_eq, s_tmp);
+  int my_take = 0;
+  {
+    int r = eq_rank;
+    for (int p = pb; p < pe; ++p) {
+      const unsigned long long key = desc_key(est[p]);
+      const bool eq = key == T;
+      my_take += (key < T) || (eq && r < kk);
+      r += eq;
+    }
+  }
+  int pos = block_exclusive_scan(my_take, s_tmp);
+  for (int w = tid; w < a.words; w += kTopkThreads) s_bits[w] = 0u;
+  __syncthreads();
+  {
+    int r = eq_rank;
+    int32_t* out = a.sel_idx + (size_t)row * a.k_sel;
+    for (int p = pb; p < pe; ++p) {
+      const unsigned long long key = desc_key(est[p]);
+      const bool eq = key == T;
+      if ((key < T) || (eq && r < kk)) {
+        out[pos++] = p;
+        atomicOr(&s_bits[p >> 5], 1u << (p & 31));
+      }
+      r += eq;
+    }
+  }
+  __syncthreads();
+  uint32_t* rb = a.sel_bits + (size_t)row * a.words;
+  uint32_t* ub = a.union_bits + (size_t)(b * d.hkv + kvh) * a.words;
+  for (int w = tid; w < a.words; w += kTopkThreads) {
+    const uint32_t v = s_bits[w];
+    rb[w] = v;
+    if (v) atomicOr(ub + w, v);
+  }
+}
+
+// ------------------------------------------------------------------ sparse pass
+
+template <int D, int WARPS_M, int WARPS_N, int STAGES>
+struct SCfg {
+  static constexpr int kConsumerWarps = WARPS_M * WARPS_N;
+  static constexpr int kProducerWarp = kConsumerWarps;
+  static constexpr int kAuxWarp = kConsumerWarps + 1;
+  static constexpr int kThreads = 32 * (kConsumerWarps + 2);
+  static constexpr int kFinishThreads = 32 * (kConsumerWarps + 1);
+  static constexpr int kRowTile = 16 * WARPS_M;
+  static constexpr int KW = 64 / WARPS_N;
+  static constexpr int kPageBytes = kPage * D * 2;         // one page of K (or V)
+  static constexpr int kTileBytes = kTilePages * kPageBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;       // K then V
+  static constexpr int kScratchBytes = kConsumerWarps * 16 * (D + 2) * 4 * 2;  // sel and res
+  static constexpr int kRingBytes = STAGES * kStageBytes;
+  static constexpr int kSmemBytes = (kRingBytes > kScratchBytes ? kRingBytes : kScratchBytes) + 1024;
+  static_assert(KW % 16 == 0, "whole k16 steps per warp");
+  static_assert(kRingBytes >= 2 * kRowTile * (D + 4) * 4 + 1024 + ((150 * kRowTile * 4 + 127) / 128) * 128,
+                "finisher space");
+};
+
+// Byte offset of (key in tile, d) for a tile of 4 pages, each page stored as D/64
+// boxes of [16 keys x 64 d] with the 128-byte swizzle (chunk c of row r at c ^ (r % 8)).
+__device__ __forceinline__ uint32_t pswz(int key, int d, int D) {
+  const int slot = key >> 4, kr = key & 15;
+  return (uint32_t)(slot * (kPage * D * 2) + (d >> 6) * (kPage * 128) + kr * 128 +
+                    ((((d & 63) >> 3) ^ (kr & 7)) << 4) + (d & 7) * 2);
+}
+
+__device__ __forceinline__ bool sel_bit(const uint32_t* rowbits, int page) {
+  return (__ldg(rowbits + (page >> 5)) >> (page & 31)) & 1u;
+}
+
+// Online-softmax state of one 16-row fragment set (two rows per thread).
+template <int D>
+struct Acc {
+  float o[D / 8][4];
+  float m0, m1, l0, l1;
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    m0 = m1 = -CUDART_INF_F;
+    l0 = l1 = 0.f;
+  }
+};
+
+// Online softmax update + P V for one tile: `sc` holds base-2 scores (masked to
+// -inf where the key is not in this set).
+template <int D, int KW>
+__device__ __forceinline__ void softmax_pv(Acc<D>& A, float (&sc)[KW / 8][4], uint32_t sV, int wn, int lane) {
+  float mx0 = A.m0, mx1 = A.m1;
+#pragma unroll
+  for (int n = 0; n < KW / 8; ++n) {
+    mx0 = fmaxf(mx0, fmaxf(sc[n][0], sc[n][1]));
+    mx1 = fmaxf(mx1, fmaxf(sc[n][2], sc[n][3]));
+  }
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+  const float base0 = (mx0 == -CUDART_INF_F) ? 0.f : mx0;
+  const float base1 = (mx1 == -CUDART_INF_F) ? 0.f : mx1;
+  const float al0 = ex2_approx(A.m0 - base0), al1 = ex2_approx(A.m1 - base1);
+  float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+  for (int n = 0; n < KW / 8; ++n) {
+    sc[n][0] = ex2_approx(sc[n][0] - base0);
+    sc[n][1] = ex2_approx(sc[n][1] - base0);
+    sc[n][2] = ex2_approx(sc[n][2] - base1);
+    sc[n][3] = ex2_approx(sc[n][3] - base1);
+    ps0 += sc[n][0] + sc[n][1];
+    ps1 += sc[n][2] + sc[n][3];
+  }
+  A.l0 = A.l0 * al0 + ps0;
+  A.l1 = A.l1 * al1 + ps1;
+  A.m0 = mx0;
+  A.m1 = mx1;
+#pragma unroll
+  for (int dn = 0; dn < D / 8; ++dn) {
+    A.o[dn][0] *= al0;
+    A.o[dn][1] *= al0;
+    A.o[dn][2] *= al1;
+    A.o[dn][3] *= al1;
+  }
+#pragma unroll
+  for (int k2 = 0; k2 < KW / 16; ++k2) {
+    uint32_t pa[4];
+    pa[0] = pack_bf16x2(sc[2 * k2][0], sc[2 * k2][1]);
+    pa[1] = pack_bf16x2(sc[2 * k2][2], sc[2 * k2][3]);
+    pa[2] = pack_bf16x2(sc[2 * k2 + 1][0], sc[2 * k2 + 1][1]);
+    pa[3] = pack_bf16x2(sc[2 * k2 + 1][2], sc[2 * k2 + 1][3]);
+#pragma unroll
+    for (int dn = 0; dn < D / 8; dn += 2) {
+      const int key = wn * KW + k2 * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int dd = dn * 8 + (lane >> 4) * 8;
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(sV + pswz(key, dd, D), b0, b1, b2, b3);
+      mma_bf16_16816(A.o[dn], pa, b0, b1);
+      mma_bf16_16816(A.o[dn + 1], pa, b2, b3);
+    }
+  }
+}
+
+// Merge the WARPS_N key slices of each row (scratch in smem) into this CTA's
+// partial [RT][D + 4] (A normalised, natural-log L) in global memory.
+template <int D, int WARPS_M, int WARPS_N>
+__device__ void write_partial(const float* scr, float* mypart, int tid) {
+  constexpr int RT = 16 * WARPS_M, NCW = WARPS_M * WARPS_N;
+  for (int idx = tid; idx < RT * (D / 4); idx += NCW * 32) {
+    const int r = idx / (D / 4), d4 = idx - r * (D / 4);
+    const int wmr = r >> 4, rr = r & 15;
+    float M = -CUDART_INF_F;
+#pragma unroll
+    for (int x = 0; x < WARPS_N; ++x) M = fmaxf(M, scr[((size_t)(wmr * WARPS_N + x) * 16 + rr) * (D + 2) + D]);
+    float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+    float L = -CUDART_INF_F;
+    if (M != -CUDART_INF_F) {
+      float den = 0.f;
+#pragma unroll
+      for (int x = 0; x < WARPS_N; ++x) {
+        const float* w = scr + ((size_t)(wmr * WARPS_N + x) * 16 + rr) * (D + 2);
+        const float s = ex2_approx(w[D] - M);
+        den += s * w[D + 1];
+        A.x += s * w[d4 * 4 + 0];
+        A.y += s * w[d4 * 4 + 1];
+        A.z += s * w[d4 * 4 + 2];
+        A.w += s * w[d4 * 4 + 3];
+      }
+      if (den > 0.f) {
+        const float inv = 1.f / den;
+        A = make_float4(A.x * inv, A.y * inv, A.z * inv, A.w * inv);
+        L = (M + __log2f(den)) * 0.6931471805599453f;
+      } else {
+        A = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    *reinterpret_cast<float4*>(mypart + (size_t)r * (D + 4) + d4 * 4) = A;
+    if (d4 == 0) mypart[(size_t)r * (D + 4) + D] = L;
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void stash(float* scr, int warp, int lane, const Acc<D>& A) {
+  float* w = scr + (size_t)warp * 16 * (D + 2);
+  const int c = lane & 3, q0 = lane >> 2, q1 = q0 + 8;
+#pragma unroll
+  for (int dn = 0; dn < D / 8; ++dn) {
+    w[q0 * (D + 2) + dn * 8 + 2 * c] = A.o[dn][0];
+    w[q0 * (D + 2) + dn * 8 + 2 * c + 1] = A.o[dn][1];
+    w[q1 * (D + 2) + dn * 8 + 2 * c] = A.o[dn][2];
+    w[q1 * (D + 2) + dn * 8 + 2 * c + 1] = A.o[dn][3];
+  }
+  if (c == 0) {
+    w[q0 * (D + 2) + D] = A.m0;
+    w[q0 * (D + 2) + D + 1] = A.l0;
+    w[q1 * (D + 2) + D] = A.m1;
+    w[q1 * (D + 2) + D + 1] = A.l1;
+  }
+}
+
+constexpr int kBarConsumers = 1;
+constexpr int kBarFinish = 2;
+
+template <int D, int WARPS_M, int WARPS_N, int STAGES>
+__global__ void __launch_bounds__(SCfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
+    sparse_pass_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const SparseArgs args) {
+  using C = SCfg<D, WARPS_M, WARPS_N, STAGES>;
+  constexpr int NCW = C::kConsumerWarps;
+  constexpr int KW = C::KW;
+  constexpr int RT = C::kRowTile;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full_bar[STAGES];
+  __shared__ __align__(8) uint64_t empty_bar[STAGES];
+  __shared__ __align__(8) uint64_t comb_bar;
+  __shared__ int s_pages[STAGES][kTilePages];
+  __shared__ int s_flags[RT];
+  __shared__ int s_red[32];
+  __shared__ int s_last;
+  __shared__ int s_M;
+  __shared__ int s_recompute;
+  __shared__ int s_union_total;
+
+  const Dims& d = args.d;
+  const SplitPlan& plan = args.plan;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int split = blockIdx.x, rt = blockIdx.y, bg = blockIdx.z;
+  const int b = bg / d.hkv, kvh = bg - b * d.hkv;
+  const int row0 = rt * RT;
+  const int rows_valid = min(RT, d.R - row0);
+  const size_t unit = (size_t)bg * plan.n_row_tiles + rt;
+  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B + row0;
+  const bf16* q = static_cast<const bf16*>(args.q);
+
+  // Gate (tau only): every row of the batch element decides alike.
+  {
+    int M = 0;
+    bool rec = true;
+    if (args.gate.enabled) {
+      M = block_updated_count(args.gate.mask + (size_t)b * d.B, d.B, s_red);
+      rec = !tau_reuse(args.gate, M);
+    }
+    if (tid == 0) {
+      s_M = M;
+      s_recompute = rec ? 1 : 0;
+    }
+    for (int r = tid; r < RT; r += blockDim.x) s_flags[r] = (r < rows_valid && rec) ? 1 : 0;
+  }
+  // Reuse: this split's share of the union pages of the group.
+  if (tid < 32) {
+    const uint32_t* ub = args.union_bits + (size_t)bg * args.words;
+    int tot = 0;
+    for (int w = lane; w < args.words; w += 32) tot += __popc(ub[w]);
+    tot = warp_sum_int(tot);
+    if (lane == 0) s_union_total = tot;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], NCW);
+    }
+    mbar_init(&comb_bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const bool recompute = s_recompute != 0;
+  // Work in pages: recompute = all pages; reuse = the union pages, in page order.
+  const int total_pages = recompute ? args.P : s_union_total;
+  const int total_tiles = (total_pages + kTilePages - 1) / kTilePages;
+  const int tps = (total_tiles + plan.splits - 1) / plan.splits;
+  const int t_begin = min(total_tiles, split * tps), t_end = min(total_tiles, t_begin + tps);
+  const int ntiles = t_end - t_begin;
+
+  if (warp == C::kProducerWarp) {
+    // ---------------- producer: page loads into the ring ----------------
+    if (lane == 0 && ntiles > 0) {
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      const uint32_t* ub = args.union_bits + (size_t)bg * args.words;
+      int cur = t_begin * kTilePages;  // index among the pages of the work list
+      int wcur = 0, wbits = 0, seen = 0;  // union enumeration cursor
+      if (!recompute) {
+        // position the cursor on the cur-th union page
+        for (wcur = 0; wcur < args.words; ++wcur) {
+          const int c = __popc(ub[wcur]);
+          if (seen + c > cur) break;
+          seen += c;
+        }
+        wbits = wcur < args.words ? (int)ub[wcur] : 0;
+        for (int skip = cur - seen; skip > 0; --skip) wbits &= wbits - 1;
+      }
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % STAGES;
+        const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+        if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, args.err, DEV_ERR_WAIT_EMPTY)) break;
+        int pg[kTilePages];
+        int nvalid = 0;
+#pragma unroll
+        for (int j = 0; j < kTilePages; ++j) {
+          int page = -1;
+          if (cur < total_pages) {
+            if (recompute) {
+              page = cur;
+            } else {
+              while (wbits == 0 && wcur + 1 < args.words) wbits = (int)ub[++wcur];
+              page = wcur * 32 + (__ffs(wbits) - 1);
+              wbits &= wbits - 1;
+            }
+            ++cur;
+            ++nvalid;
+          }
+          pg[j] = page;
+          s_pages[s][j] = page;
+        }
+        // Every slot is loaded: an empty slot reads page P, entirely past the last key,
+        // which the TMA fills with zeros (its scores are masked; P V must not see
+        // stale shared memory).
+        (void)nvalid;
+        mbar_arrive_expect_tx(&full_bar[s], (uint32_t)kTilePages * 2u * C::kPageBytes);
+        uint8_t* st = smem + s * C::kStageBytes;
+#pragma unroll
+        for (int j = 0; j < kTilePages; ++j) {
+          const int row = (pg[j] >= 0 ? pg[j] : args.P) * kPage;
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h) {
+            tma_load_3d(st + j * C::kPageBytes + h * (kPage * 128), &tmK, &full_bar[s], h * 64, row, bg);
+            tma_load_3d(st + C::kTileBytes + j * C::kPageBytes + h * (kPage * 128), &tmV, &full_bar[s], h * 64, row,
+                        bg);
+          }
+        }
+        ++issued;
+      }
+      for (int i = max(0, issued - STAGES); i < issued; ++i)
+        mbar_wait_bounded(&full_bar[i % STAGES], (uint32_t)(i / STAGES) & 1u, args.err, DEV_ERR_WAIT_FULL);
+    }
+    return;
+  }
+
+  const size_t rs = (size_t)D + 4;
+  if (warp == C::kAuxWarp) {
+    // this split's share of the tile's in-block rows, parked in the workspace
+    const int per = (rows_valid + plan.splits - 1) / plan.splits;
+    const int r0 = min(rows_valid, split * per), r1 = min(rows_valid, r0 + per);
+    inblock_rows_to_ws<bf16, D>(d, q, static_cast<const bf16*>(args.step.k_blk),
+                                static_cast<const bf16*>(args.step.v_blk), b, kvh, row0, r0, r1,
+                                args.inblock + unit * RT * rs, 0, 1, lane);
+  } else {
+    // ---------------------------- consumers ----------------------------
+    const int wm = warp / WARPS_N, wn = warp - (warp / WARPS_N) * WARPS_N;
+    const int c = lane & 3;
+    const int r0 = wm * 16 + (lane >> 2), r1 = r0 + 8;
+    uint32_t qf[D / 16][4];
+    {
+      const bf16* qb = q + grow0 * D;
+      const bool v0 = r0 < rows_valid, v1 = r1 < rows_valid;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int col = kk * 16 + 2 * c;
+        qf[kk][0] = v0 ? *reinterpret_cast<const uint32_t*>(qb + (size_t)r0 * D + col) : 0u;
+        qf[kk][1] = v1 ? *reinterpret_cast<const uint32_t*>(qb + (size_t)r1 * D + col) : 0u;
+        qf[kk][2] = v0 ? *reinterpret_cast<const uint32_t*>(qb + (size_t)r0 * D + col + 8) : 0u;
+        qf[kk][3] = v1 ? *reinterpret_cast<const uint32_t*>(qb + (size_t)r1 * D + col + 8) : 0u;
+      }
+    }
+    const uint32_t* bits0 = args.sel_bits + (grow0 + min(r0, rows_valid - 1)) * (size_t)args.words;
+    const uint32_t* bits1 = args.sel_bits + (grow0 + min(r1, rows_valid - 1)) * (size_t)args.words;
+    Acc<D> As, Ar;
+    As.init();
+    Ar.init();
+    const float sl2 = d.scale * 1.4426950408889634f;
+    bool ok = true;
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const int s = i % STAGES;
+      if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(i / STAGES) & 1u, args.err, DEV_ERR_WAIT_FULL)) {
+        ok = false;
+        break;
+      }
+      const uint32_t sK = smem_u32(smem + s * C::kStageBytes);
+      const uint32_t sV = sK + C::kTileBytes;
+      float sc[KW / 8][4];
+#pragma unroll
+      for (int n = 0; n < KW / 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+        for (int n = 0; n < KW / 8; n += 2) {
+          const int key = wn * KW + n * 8 + (lane & 7) + ((lane >> 4) << 3);
+          const int dd = kk * 16 + ((lane >> 3) & 1) * 8;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(sK + pswz(key, dd, D), b0, b1, b2, b3);
+          mma_bf16_16816(sc[n], qf[kk], b0, b1);
+          mma_bf16_16816(sc[n + 1], qf[kk], b2, b3);
+        }
+      }
+      // Route each score to the selected or the residual set of its row.
+      float ss[KW / 8][4], sr[KW / 8][4];
+#pragma unroll
+      for (int n = 0; n < KW / 8; ++n) {
+        const int colb = wn * KW + n * 8;
+        const int page = s_pages[s][colb >> 4];
+        const bool sel0 = page >= 0 && sel_bit(bits0, page);
+        const bool sel1 = page >= 0 && sel_bit(bits1, page);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const long long key = (long long)page * kPage + (colb & 15) + 2 * c + (j & 1);
+          const bool valid = page >= 0 && key < d.N;
+          const bool sel = j < 2 ? sel0 : sel1;
+          const float v = sc[n][j] * sl2;
+          ss[n][j] = (valid && sel) ? v : -CUDART_INF_F;
+          sr[n][j] = (valid && !sel) ? v : -CUDART_INF_F;
+        }
+      }
+      softmax_pv<D, KW>(As, ss, sV, wn, lane);
+      if (recompute) softmax_pv<D, KW>(Ar, sr, sV, wn, lane);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[s]);
+    }
+    As.l0 += __shfl_xor_sync(0xffffffffu, As.l0, 1);
+    As.l0 += __shfl_xor_sync(0xffffffffu, As.l0, 2);
+    As.l1 += __shfl_xor_sync(0xffffffffu, As.l1, 1);
+    As.l1 += __shfl_xor_sync(0xffffffffu, As.l1, 2);
+    Ar.l0 += __shfl_xor_sync(0xffffffffu, Ar.l0, 1);
+    Ar.l0 += __shfl_xor_sync(0xffffffffu, Ar.l0, 2);
+    Ar.l1 += __shfl_xor_sync(0xffffffffu, Ar.l1, 1);
+    Ar.l1 += __shfl_xor_sync(0xffffffffu, Ar.l1, 2);
+    named_barrier_sync(kBarConsumers, NCW * 32);
+    float* scr_s = reinterpret_cast<float*>(smem);
+    float* scr_r = scr_s + (size_t)NCW * 16 * (D + 2);
+    stash<D>(scr_s, warp, lane, As);
+    stash<D>(scr_r, warp, lane, Ar);
+    named_barrier_sync(kBarConsumers, NCW * 32);
+    write_partial<D, WARPS_M, WARPS_N>(scr_s, args.part_sel + (unit * plan.splits + split) * RT * rs, tid);
+    if (recompute)
+      write_partial<D, WARPS_M, WARPS_N>(scr_r, args.part_res + (unit * plan.splits + split) * RT * rs, tid);
+  }
+
+  named_barrier_sync(kBarFinish, C::kFinishThreads);
+  if (tid == 0) {
+    __threadfence();
+    const unsigned prev = atomicAdd(args.counters + unit, 1u);
+    __threadfence();
+    s_last = (prev == (unsigned)plan.splits - 1u);
+  }
+  named_barrier_sync(kBarFinish, C::kFinishThreads);
+  if (!s_last) return;
+
+  // ---------------- finisher: consumers + aux ----------------
+  constexpr int NT = C::kFinishThreads;
+  constexpr int D4 = D / 4;
+  constexpr int IT = (RT * D4 + NT - 1) / NT;
+  const int ftid = warp < NCW ? tid : NCW * 32 + lane;
+  const int in_bytes = (RT * (D + 4) * 4 + 127) / 128 * 128;
+  float* s_in = reinterpret_cast<float*>(smem);
+  float* s_Ls = reinterpret_cast<float*>(smem + in_bytes);  // per row: L_sel, L_res, w_sel, w_res, w_pre, w_in
+  float* s_Lr = s_Ls + RT;
+  float* s_w = s_Lr + RT;
+  const int hdr = in_bytes + ((6 * RT * 4) + 127) / 128 * 128;
+  uint32_t phase = 0;
+  float4 Asel[IT], Ares[IT];
+  combine_regs<D, RT, NT>(args.part_sel + unit * plan.splits * RT * rs, plan.splits, args.inblock + unit * RT * rs,
+                          s_in, smem + hdr, C::kRingBytes - hdr, &comb_bar, &phase, args.err, ftid, kBarFinish, Asel,
+                          s_Ls);
+  if (recompute)
+    combine_regs<D, RT, NT>(args.part_res + unit * plan.splits * RT * rs, plan.splits, nullptr, nullptr,
+                            smem + hdr, C::kRingBytes - hdr, &comb_bar, &phase, args.err, ftid, kBarFinish, Ares,
+                            s_Lr);
+  // per-row weights: pre = merge(sel, res); full = merge(pre, in)
+  for (int r = ftid; r < rows_valid; r += NT) {
+    const size_t grow = grow0 + r;
+    const float lr = recompute ? s_Lr[r] : __ldcg(args.l_res + grow);
+    float ws, wr, lpre, wp, wi, lf;
+    merge_weights(s_Ls[r], lr, ws, wr, lpre);
+    merge_weights(lpre, s_in[(size_t)r * rs + D], wp, wi, lf);
+    s_w[4 * r + 0] = ws;
+    s_w[4 * r + 1] = wr;
+    s_w[4 * r + 2] = wp;
+    s_w[4 * r + 3] = wi;
+    if (recompute) args.l_res[grow] = s_Lr[r];
+    if (args.l_sel) args.l_sel[grow] = s_Ls[r];
+    if (args.step.l_full) args.step.l_full[grow] = lf;
+  }
+  named_barrier_sync(kBarFinish, NT);
+#pragma unroll
+  for (int k = 0; k < IT; ++k) {
+    const int idx = ftid + k * NT;
+    if (idx >= RT * D4) continue;
+    const int r = idx / D4, d4 = idx - r * D4;
+    if (r >= rows_valid) continue;
+    const size_t off = (grow0 + r) * D + (size_t)d4 * 4;
+    const float4 ar = recompute ? Ares[k] : __ldcg(reinterpret_cast<const float4*>(args.a_res + off));
+    if (recompute) *reinterpret_cast<float4*>(args.a_res + off) = ar;
+    if (args.a_sel) *reinterpret_cast<float4*>(args.a_sel + off) = Asel[k];
+    const float4 pre = wsum4(s_w[4 * r + 0], Asel[k], s_w[4 * r + 1], ar);
+    const float4 ai = *reinterpret_cast<const float4*>(s_in + (size_t)r * rs + d4 * 4);
+    store4(args.step.a_full, off, wsum4(s_w[4 * r + 2], pre, s_w[4 * r + 3], ai), 1);
+  }
+  if (args.gate.enabled) {
+    for (int r = ftid; r < rows_valid; r += NT) {
+      const int gr = row0 + r;
+      if ((r == 0 || gr % d.B == 0) && args.step.dec_reuse)
+        args.step.dec_reuse[(size_t)b * d.hq + kvh * d.G + gr / d.B] = recompute ? 0 : 1;
+    }
+    if (ftid == 0 && kvh == 0 && rt == 0 && args.step.dec_M) args.step.dec_M[b] = s_M;
+  }
+  if (tid == 0) args.counters[unit] = 0u;
+}
+
+template <int D, int WM, int WN, int STAGES>
+cudaError_t launch_sparse_cfg(const SparseArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s) {
+  using C = SCfg<D, WM, WN, STAGES>;
+  auto kern = sparse_pass_kernel<D, WM, WN, STAGES>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  dim3 grid(a.plan.splits, a.plan.n_row_tiles, a.d.b * a.d.hkv);
+  kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int sparse_supported(int D, int row_tile) { return (D == 64 || D == 128) && (row_tile == 16 || row_tile == 32); }
+
+cudaError_t launch_page_minmax(const SparseArgs& a, cudaStream_t s) {
+  dim3 grid((a.P + 31) / 32, a.d.b * a.d.hkv);
+  if (a.d.D == 128)
+    page_minmax_kernel<128><<<grid, 32 * 8, 0, s>>>(a);
+  else if (a.d.D == 64)
+    page_minmax_kernel<64><<<grid, 32 * 4, 0, s>>>(a);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sparse_select(const SparseArgs& a, cudaStream_t s) {
+  const size_t est_smem = (size_t)((a.d.R + 15) / 16 * 16) * a.d.D * sizeof(double);
+  dim3 g1((a.P + kEstThreads - 1) / kEstThreads, a.d.b * a.d.hkv);
+  cudaError_t e;
+  if (a.d.D == 128) {
+    e = cudaFuncSetAttribute(page_estimate_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)est_smem);
+    if (e != cudaSuccess) return e;
+    page_estimate_kernel<128><<<g1, kEstThreads, est_smem, s>>>(a);
+  } else {
+    e = cudaFuncSetAttribute(page_estimate_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)est_smem);
+    if (e != cudaSuccess) return e;
+    page_estimate_kernel<64><<<g1, kEstThreads, est_smem, s>>>(a);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t bits_smem = (size_t)a.words * sizeof(uint32_t);
+  if (bits_smem > 48 * 1024) {
+    e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bits_smem);
+    if (e != cudaSuccess) return e;
+  }
+  topk_kernel<<<a.d.b * a.d.hq * a.d.B, kTopkThreads, bits_smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sparse_pass(const SparseArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s) {
+  const int D = a.d.D, rt = a.plan.row_tile;
+  if (D == 128) {
+    if (rt == 16) return launch_sparse_cfg<128, 1, 4, 4>(a, tk, tv, s);
+    if (rt == 32) return launch_sparse_cfg<128, 2, 2, 4>(a, tk, tv, s);
+  } else if (D == 64) {
+    if (rt == 16) return launch_sparse_cfg<64, 1, 4, 6>(a, tk, tv, s);
+    if (rt == 32) return launch_sparse_cfg<64, 2, 2, 6>(a, tk, tv, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace fb

@@ -17,7 +17,8 @@ __all__ = [
     "FBError", "Shape", "Gate", "load", "lib_path", "make_shape", "make_gate", "FB_F32", "FB_BF16",
     "fb_version", "fb_status_string", "fb_device_error", "fb_workspace_bytes", "fb_workspace_init",
     "fb_gate_eval", "fb_prefix_attn", "fb_prefix_attn_noalloc", "fb_block_attn", "fb_merge", "fb_block_merge", "fb_step",
-    "CachedAttentionLayer", "EXPORTED",
+    "fb_page_minmax", "fb_sparse_workspace_bytes", "fb_sparse_select", "fb_sparse_step", "Sparse",
+    "SparseResidualLayer", "CachedAttentionLayer", "EXPORTED",
 ]
 
 FB_F32 = 0
@@ -50,11 +51,20 @@ class Gate(ctypes.Structure):
                 ("first_step", ctypes.c_int32), ("tau", ctypes.c_int32), ("gamma", ctypes.c_float)]
 
 
+class Sparse(ctypes.Structure):
+    """struct fb_sparse (device pointers to the page bounds and the sparse state)."""
+    _fields_ = [("page_size", ctypes.c_int32), ("n_select", ctypes.c_int32), ("kmin", ctypes.c_void_p),
+                ("kmax", ctypes.c_void_p), ("sel_idx", ctypes.c_void_p), ("sel_bits", ctypes.c_void_p),
+                ("union_bits", ctypes.c_void_p), ("a_res", ctypes.c_void_p), ("l_res", ctypes.c_void_p),
+                ("a_sel", ctypes.c_void_p), ("l_sel", ctypes.c_void_p)]
+
+
 _vp = ctypes.c_void_p
 _sz = ctypes.c_size_t
 _i = ctypes.c_int
 _PS = ctypes.POINTER(Shape)
 _PG = ctypes.POINTER(Gate)
+_PSP = ctypes.POINTER(Sparse)
 
 # name -> (restype, argtypes); the set of exported C-ABI symbols.
 EXPORTED = {
@@ -70,6 +80,10 @@ EXPORTED = {
     "fb_block_merge": (_i, [_PS, _vp, _vp, _vp, _PG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fb_step": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _PG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fb_prefix_attn_noalloc": (_i, [_PS, _vp, _vp, _vp, _PG, _vp, _vp, _vp]),
+    "fb_page_minmax": (_i, [_PS, _vp, _i, _vp, _vp, _vp]),
+    "fb_sparse_workspace_bytes": (_sz, [_PS, _i]),
+    "fb_sparse_select": (_i, [_PS, _vp, _PG, _PSP, _vp, _sz, _vp]),
+    "fb_sparse_step": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _PG, _PSP, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -199,6 +213,69 @@ def fb_prefix_attn_noalloc(shape, q, k_cache, v_cache, gate, a_out, l_out):
     _check("fb_prefix_attn_noalloc", load().fb_prefix_attn_noalloc(
         ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache), _gref(gate), _ptr(a_out), _ptr(l_out),
         _stream()))
+
+
+def fb_page_minmax(shape, k_cache, page_size, kmin, kmax):
+    _check("fb_page_minmax", load().fb_page_minmax(ctypes.byref(shape), _ptr(k_cache), int(page_size), _ptr(kmin),
+                                                   _ptr(kmax), _stream()))
+
+
+def fb_sparse_workspace_bytes(shape, page_size=16) -> int:
+    return int(load().fb_sparse_workspace_bytes(ctypes.byref(shape), int(page_size)))
+
+
+def fb_sparse_select(shape, q, gate, sparse, ws):
+    _check("fb_sparse_select", load().fb_sparse_select(ctypes.byref(shape), _ptr(q), _gref(gate),
+                                                       ctypes.byref(sparse), *_wsargs(ws), _stream()))
+
+
+def fb_sparse_step(shape, q, k_cache, v_cache, k_blk, v_blk, gate, sparse, a_full, l_full, dec_M, dec_reuse, ws):
+    _check("fb_sparse_step", load().fb_sparse_step(
+        ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_blk), _ptr(v_blk), _gref(gate),
+        ctypes.byref(sparse), _ptr(a_full), _ptr(l_full), _ptr(dec_M), _ptr(dec_reuse), *_wsargs(ws), _stream()))
+
+
+class SparseResidualLayer:
+    """Device buffers of one attention layer in sparse-residual mode, stepped through fb_sparse_step.
+
+    Owns the page bounds (computed once from the prefix keys), the frozen selection,
+    the residual cache, the outputs and the workspace.
+    """
+
+    def __init__(self, batch, h_q, h_kv, head_dim, block, k_cache, v_cache, n_select, page_size=16, scale=0.0,
+                 keep_sel=False):
+        dev = k_cache.device
+        n = k_cache.shape[2]
+        self.shape = make_shape(batch, h_q, h_kv, head_dim, block, n, k_cache.dtype, scale=scale)
+        self.k_cache, self.v_cache = k_cache, v_cache
+        self.n_pages = (n + page_size - 1) // page_size
+        words = (self.n_pages + 31) // 32
+        self.kmin = torch.empty((batch, h_kv, head_dim, self.n_pages), device=dev, dtype=k_cache.dtype)
+        self.kmax = torch.empty_like(self.kmin)
+        fb_page_minmax(self.shape, k_cache, page_size, self.kmin, self.kmax)
+        i32, f32 = dict(device=dev, dtype=torch.int32), dict(device=dev, dtype=torch.float32)
+        self.sel_idx = torch.zeros((batch, h_q, block, n_select), **i32)
+        self.sel_bits = torch.zeros((batch, h_q, block, words), **i32)
+        self.union_bits = torch.zeros((batch, h_kv, words), **i32)
+        self.a_res = torch.zeros((batch, h_q, block, head_dim), **f32)
+        self.l_res = torch.full((batch, h_q, block), float("-inf"), **f32)
+        self.a_sel = torch.zeros((batch, h_q, block, head_dim), **f32) if keep_sel else None
+        self.l_sel = torch.zeros((batch, h_q, block), **f32) if keep_sel else None
+        self.a_full = torch.zeros((batch, h_q, block, head_dim), device=dev, dtype=k_cache.dtype)
+        self.l_full = torch.zeros((batch, h_q, block), **f32)
+        self.dec_M = torch.zeros((batch,), **i32)
+        self.dec_reuse = torch.zeros((batch, h_q), device=dev, dtype=torch.uint8)
+        nbytes = fb_sparse_workspace_bytes(self.shape, page_size)
+        self.ws = torch.zeros(((nbytes + 15) // 16 * 16,), device=dev, dtype=torch.uint8)
+        p = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+        self.sparse = Sparse(page_size, n_select, p(self.kmin), p(self.kmax), p(self.sel_idx), p(self.sel_bits),
+                             p(self.union_bits), p(self.a_res), p(self.l_res), p(self.a_sel), p(self.l_sel))
+
+    def step(self, q, k_blk, v_blk, mask, first_step, tau):
+        g = make_gate(mask, first_step, tau)
+        fb_sparse_step(self.shape, q, self.k_cache, self.v_cache, k_blk, v_blk, g, self.sparse, self.a_full,
+                       self.l_full, self.dec_M, self.dec_reuse, self.ws)
+        return self.a_full
 
 
 class CachedAttentionLayer:

@@ -158,6 +158,59 @@ int fb_step(const fb_shape* shape, const void* q, const void* k_cache, const voi
             float* l_out, void* a_full, float* l_full, int32_t* dec_M, uint8_t* dec_reuse,
             void* ws, size_t ws_bytes, fb_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Sparse attention with a cached residual (FlashBlock, "Adaptive reuse
+ * strategies / compatibility with sparse attention"): the keys a sparse selector
+ * leaves out are the "out-of-block" set whose attention is cached (the
+ * residual); the selected keys are attended fresh every step:
+ *     A_full = merge(merge(A_sel, A_res), A_in).
+ * Selector (the pages name QUEST as one, without defining it; this is the plain
+ * page-bound reading): prefix pages of 16 tokens; per page and channel the
+ * min / max of K; for each query row the page estimate
+ *     e_p = sum_d max(q_d kmin_{p,d}, q_d kmax_{p,d})   (float64, ascending d)
+ * and the top n_select pages by (e desc, page asc).  On a recompute step (first
+ * step of the block, or M >= tau) the selection is redone and frozen and the
+ * residual is recomputed with the current queries; on a reuse step only the
+ * union of the KV group's selected pages is read.  Supported: bf16, head_dim 64
+ * or 128, page_size 16, block * (h_q / h_kv) <= 32, block <= 64, n_prefix >= 1,
+ * the tau gate only (head_sim must be NULL).  words = ceil(n_pages / 32),
+ * n_pages = ceil(n_prefix / 16).  All buffers are caller-owned device memory. */
+typedef struct fb_sparse {
+  int32_t page_size;      /* 16 */
+  int32_t n_select;       /* pages per query row, 1 .. n_pages */
+  const void* kmin;       /* [b, H_kv, D, n_pages] bf16 page minima (fb_page_minmax) */
+  const void* kmax;       /* [b, H_kv, D, n_pages] bf16 page maxima */
+  int32_t* sel_idx;       /* state [b, H_q, B, n_select] int32, selected pages ascending */
+  uint32_t* sel_bits;     /* state [b, H_q, B, words] bitmap of the same pages */
+  uint32_t* union_bits;   /* state [b, H_kv, words] union over the KV group's rows */
+  float* a_res;           /* state: residual cache [b, H_q, B, D] fp32 */
+  float* l_res;           /* state: [b, H_q, B] fp32, natural log */
+  float* a_sel;           /* optional output (fresh part) [b, H_q, B, D] fp32, or NULL */
+  float* l_sel;           /* optional output [b, H_q, B], or NULL */
+} fb_sparse;
+
+/* Channel-wise page bounds of the prefix keys (exact bf16 min / max over each
+ * page's real tokens; the last page may be partial). */
+int fb_page_minmax(const fb_shape* shape, const void* k_cache, int page_size, void* kmin, void* kmax,
+                   fb_stream_t stream);
+
+/* Workspace of fb_sparse_select / fb_sparse_step (split partials of both parts,
+ * in-block rows, page estimates, counters; same reuse rules as fb_workspace_bytes). */
+size_t fb_sparse_workspace_bytes(const fb_shape* shape, int page_size);
+
+/* Selection only: for batch elements whose gate says recompute, page estimates and
+ * top-k -> sel_idx, sel_bits, union_bits.  Others keep their state untouched. */
+int fb_sparse_select(const fb_shape* shape, const void* q, const fb_gate* gate, const fb_sparse* sp,
+                     void* ws, size_t ws_bytes, fb_stream_t stream);
+
+/* One denoising step in sparse mode: fb_sparse_select, then the sparse pass that
+ * writes the residual cache (recompute), A_full, L_full (nullable) and the
+ * decisions (nullable). */
+int fb_sparse_step(const fb_shape* shape, const void* q, const void* k_cache, const void* v_cache,
+                   const void* k_blk, const void* v_blk, const fb_gate* gate, const fb_sparse* sp,
+                   void* a_full, float* l_full, int32_t* dec_M, uint8_t* dec_reuse, void* ws,
+                   size_t ws_bytes, fb_stream_t stream);
+
 /* Out-of-block attention for callers that cannot allocate device memory.
  *
  * The pages have no counterpart: this is a deployment variant of fb_prefix_attn.
