@@ -139,6 +139,28 @@ class ClockSampler:
                 "samples": len(mhz), "source": "nvml"}
 
 
+# ----------------------------------------------------------------------------- ranks
+
+
+def replica_seed(seed: int, rank: int) -> int:
+    """Each rank runs its own replica of the workload, drawn from its own seed."""
+    return seed + rank
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's timed milliseconds (every rank gets it)."""
+    if world <= 1:
+        return ms
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world: int, steps_per_rank: int, t_max_ms: float) -> float:
+    """Whole-job steps/s: all ranks' steps over the slowest rank's time."""
+    return world * steps_per_rank / (t_max_ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- device arm
 
 
@@ -268,7 +290,7 @@ def device_arm(args, rank, world):
     from block_diffusion_attention_prefix_b200 import fb
     fb.load()
     w = W.get(args.workload)
-    dw = DeviceWorkload(fb, w, seed=args.seed + rank)
+    dw = DeviceWorkload(fb, w, seed=replica_seed(args.seed, rank))
     K, Wm = args.steps, args.warmup
     dev = torch.device("cuda")
     flush = L2Flush(dev)
@@ -313,12 +335,8 @@ def device_arm(args, rank, world):
     recompute_steps = [i for i in range(K) if not reuse[i].all()]
     reuse_steps = [i for i in range(K) if reuse[i].all()]
     total_ms = sum(step_ms)
-    t_max = total_ms
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_max = float(t.item())
-    value = world * K / (t_max / 1e3)
+    t_max = max_over_ranks(total_ms, world, dev)
+    value = weak_scaling_value(world, K, t_max)
     hbm, peak_kind = peaks()
     alg, alg_reuse = dw.algorithmic_bytes()
     rec_ms = [step_ms[i] for i in recompute_steps]
