@@ -342,6 +342,19 @@ def device_arm(args, rank, world):
     rec_ms = [step_ms[i] for i in recompute_steps]
     achieved = (alg * len(rec_ms)) / (sum(rec_ms) / 1e3) / 1e9 if rec_ms else None
     traffic = ncu_traffic(args.workload)
+    tensor = None
+    if w.block > 64:
+        # Large blocks (video): the passes are dense contractions.  FLOPs of a step =
+        # 4 B D (N * heads that recompute + B * H_q)  (QK^T and PV, 2 flop per MAC).
+        nrec = [int((~reuse[i]).sum()) for i in range(K)]
+        flops = [4.0 * w.block * w.head_dim * (w.n_prefix * nrec[i] + w.block * w.h_q) * w.batch for i in range(K)]
+        tflops = sum(flops) / (sum(step_ms) / 1e3) / 1e12
+        peak_t = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops_sustained"] \
+            if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else 1400.0
+        tensor = dict(bound="tensor", achieved=tflops, peak=peak_t, unit="TFLOP/s", frac=tflops / peak_t,
+                      peak_source="measured sustained cuBLAS bf16 (MEASURED_PEAKS.json bf16_tflops_sustained)",
+                      flops_per_step_mean=sum(flops) / K, traffic=None,
+                      kernel="pass_bf16_kernel (prefix pass of recomputing heads + in-block pass)")
 
     # dense-recompute reference (standard block diffusion): gate forced to recompute
     dense_ms = []
@@ -380,6 +393,7 @@ def device_arm(args, rank, world):
                       avg_launch_us=(sum(rec_ms) / len(rec_ms) * 1e3) if rec_ms else None,
                       traffic=traffic),
         breakdown=dict(recompute_steps=len(recompute_steps), reuse_steps=len(reuse_steps),
+                       recompute_heads_per_step=float((~reuse).sum()) / K,
                        recompute_step_us=_mean_us(step_ms, recompute_steps),
                        reuse_step_us=_mean_us(step_ms, reuse_steps),
                        reuse_step_alg_bytes=alg_reuse,
@@ -394,6 +408,9 @@ def device_arm(args, rank, world):
         clocks=clocks.summary(),
         kernel_source_sha=kernel_source_hash(),
     )
+    if tensor is not None:
+        res["roofline_hbm"] = res["roofline"]
+        res["roofline"] = tensor
     if e2e:
         res["e2e"] = e2e
     return res

@@ -222,6 +222,15 @@ int run_pass(const Dims& d0, long long keys, const void* q, const void* k, const
                   ? reinterpret_cast<float*>(static_cast<char*>(ws) + a.plan.counter_bytes + a.plan.partial_bytes)
                   : nullptr;
   a.err = err;
+  if (d.dtype == FB_BF16 && tc_pass_supported(d.D, d.R) && !(step && step->enabled)) {
+    // Dense contraction (>= 128 query rows per KV head): tcgen05 + TMEM, no key split.
+    CUtensorMap tq, tk, tv;
+    const long long qrows = (long long)d.b * d.hq * d.B;
+    FB_TRY(encode_kv_map(&tq, q, d.D, qrows, d.D, qrows * d.D, 1, 128));
+    FB_TRY(encode_kv_map(&tk, k, d.D, keys, row_stride, head_stride, d.b * d.hkv, 64));
+    FB_TRY(encode_kv_map(&tv, v, d.D, keys, row_stride, head_stride, d.b * d.hkv, 64));
+    return cuda_status(launch_pass_tc(a, tq, tk, tv, stream));
+  }
   if (d.dtype == FB_BF16) {
     if (!bf16_pass_supported(d.D, a.plan.row_tile)) return FB_ERR_UNSUPPORTED;
     CUtensorMap tk, tv;

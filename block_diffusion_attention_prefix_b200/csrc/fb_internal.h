@@ -135,6 +135,10 @@ cudaError_t launch_pass_f32(const PassArgs& a, cudaStream_t s);
 cudaError_t launch_pass_bf16(const PassArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                              cudaStream_t s);
 int bf16_pass_supported(int D, int row_tile);
+// tcgen05 pass (flash_tc.cu): bf16, D = 128, at least 128 query rows per KV head.
+int tc_pass_supported(int D, int R);
+cudaError_t launch_pass_tc(const PassArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           cudaStream_t s);
 
 // Small in-block pass fused with gate and merge (B <= kSmallBlockMax).
 struct SmallBlockArgs {

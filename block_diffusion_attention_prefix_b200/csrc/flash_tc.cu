@@ -1,0 +1,408 @@
+// flash_tc.cu -- attention pass on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// For passes with at least 128 query rows per KV head (video blocks: 4680 block
+// queries per head over a 31,200-token prefix and over the 4680 block keys) the
+// contraction is dense: 128 x 128 x 128 tiles on tcgen05.mma with fp32
+// accumulators in tensor memory.  Same contract as the split pass
+// (prefix_bf16.cu): (A, L) per query row over a key set -- the out-of-block part
+// over J_out, or the in-block part over J_in merged with the cache
+// (FlashBlock technical summary, gist.science 2602.05305, "Core mechanism").
+//
+// One CTA = 128 query rows of one KV group, all keys (no split), 320 threads:
+//   warp 0     TMA producer: Q once; 64-key K and V tiles into a 4-stage ring
+//              (128-byte swizzle, no multicast).
+//   warp 1     TMEM owner and MMA issuer (one thread):
+//                S_w  = Q K_j^T   (M=128, N=64 keys, K=128 d; A, B K-major)
+//                O_w += P_w V_j   (M=128, N=128 d,  K=64 keys; A = P K-major,
+//                                  B = V MN-major)
+//              for key tiles j split between two softmax warpgroups w = j % 2,
+//              so that one group's softmax overlaps the other's MMAs;
+//              completions signalled with tcgen05.commit on mbarriers.
+//   warps 2-5, 6-9  softmax warpgroups a and b, one query row per thread (TMEM
+//              lane = row): read S_w with tcgen05.ld, online softmax in base 2, P_w
+//              (bf16) into shared memory.  O_w is rescaled in TMEM only when a row's
+//              max grows by more than 2^8 (otherwise the stale max is kept; p <= 2^8
+//              is exact enough in bf16 and cannot overflow fp32).  At the end group a
+//              merges the two partial results (the FlashBlock log-space merge) and
+//              writes the cache or merges with it into A_full.
+// TMEM: 512 columns (S_a [0,64), S_b [64,128), O_a [128,256), O_b [256,384)).
+// Every mbarrier wait is time bounded; on expiry the roles fall through to the
+// common exit, which frees TMEM.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+
+#include "fb_device.cuh"
+#include "fb_internal.h"
+#include "fb_ptx.cuh"
+
+namespace fb {
+namespace {
+
+constexpr int kM = 128;
+constexpr int kKT = 64;   // keys per tile
+constexpr int kD = 128;
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kQBlock = 128 * 128;               // Q: [128 rows][128 B] per 64-column block
+constexpr int kQBytes = 2 * kQBlock;
+constexpr int kKVBlock = kKT * 128;              // K or V: [64 keys][128 B] per 64-column block
+constexpr int kKVBytes = 2 * kKVBlock;           // one 64 x 128 tile
+constexpr int kStageBytes = 2 * kKVBytes;        // K then V
+constexpr int kPBytes = 128 * kKT * 2;           // P_w: [128 rows][64 keys] bf16 = one 128-B block
+constexpr int kQOff = 0;
+constexpr int kStageOff = kQBytes;
+constexpr int kPOff = kStageOff + kStages * kStageBytes;
+constexpr int kSmemBytes = kPOff + 2 * kPBytes + 1024;
+
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2, version 1).
+// K-major: 8-row groups 1024 B apart (SBO); LBO unused (1).  MN-major: LBO is the
+// stride between 64-element blocks along M/N, SBO the stride between 8-row groups
+// along K.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulate, bf16 A and B, A K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])),
+      "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+      "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+      "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+      "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
+      "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+      "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
+      "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
+      "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
+      "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Bounded wait taken by a whole warp: every lane waits, then all agree (tcgen05.ld /
+// st are warp-collective, so a warp must never split on a timeout).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  const bool ok = mbar_wait_bounded(bar, parity, err, DEV_ERR_WAIT_FULL);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    pass_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const PassArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t q_full;
+  __shared__ __align__(8) uint64_t kv_full[kStages];
+  __shared__ __align__(8) uint64_t kv_empty[kStages];
+  __shared__ __align__(8) uint64_t s_full[2];
+  __shared__ __align__(8) uint64_t p_full[2];
+  __shared__ __align__(8) uint64_t o_done[2];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_flags[kM];
+  __shared__ int s_red[32];
+  __shared__ float s_mb[kM], s_lb[kM];  // group b's row max / sum for the final merge
+
+  const Dims& d = args.d;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rt = blockIdx.x, bg = blockIdx.y;
+  const int b = bg / d.hkv, kvh = bg - b * d.hkv;
+  const int row0 = rt * kM;
+  const int rows_valid = min(kM, d.R - row0);
+  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B + row0;
+  const int T = (int)((d.N + kKT - 1) / kKT);
+
+  if (!gate_row_flags(args.gate, d, b, kvh, row0, rows_valid, kM, s_flags, s_red)) return;
+
+  if (tid == 0) {
+    mbar_init(&q_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&s_full[w], 1);
+      mbar_init(&p_full[w], 4);
+      mbar_init(&o_done[w], 1);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&s_tmem)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const uint32_t sQ = smem_u32(smem + kQOff);
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && T > 0) {
+      prefetch_tmap(&tmQ);
+      prefetch_tmap(&tmK);
+      prefetch_tmap(&tmV);
+      mbar_arrive_expect_tx(&q_full, kQBytes);
+      for (int h = 0; h < 2; ++h) tma_load_3d(smem + kQOff + h * kQBlock, &tmQ, &q_full, h * 64, (int)grow0, 0);
+      int issued = 0;
+      for (int j = 0; j < T; ++j) {
+        const int s = j % kStages;
+        if (!mbar_wait_bounded(&kv_empty[s], ((uint32_t)(j / kStages) & 1u) ^ 1u, args.err, DEV_ERR_WAIT_EMPTY))
+          break;
+        mbar_arrive_expect_tx(&kv_full[s], kStageBytes);
+        uint8_t* st = smem + kStageOff + s * kStageBytes;
+        for (int h = 0; h < 2; ++h) {
+          tma_load_3d(st + h * kKVBlock, &tmK, &kv_full[s], h * 64, j * kKT, bg);
+          tma_load_3d(st + kKVBytes + h * kKVBlock, &tmV, &kv_full[s], h * 64, j * kKT, bg);
+        }
+        ++issued;
+      }
+      for (int j = max(0, issued - kStages); j < issued; ++j)
+        mbar_wait_bounded(&kv_full[j % kStages], (uint32_t)(j / kStages) & 1u, args.err, DEV_ERR_WAIT_FULL);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0 && T > 0) {
+      constexpr uint32_t kIdQK = idesc_bf16(kM, kKT, false);
+      constexpr uint32_t kIdPV = idesc_bf16(kM, kD, true);
+      auto issue_qk = [&](int j) -> bool {
+        if (!mbar_wait_bounded(&kv_full[j % kStages], (uint32_t)(j / kStages) & 1u, args.err, DEV_ERR_WAIT_FULL))
+          return false;
+        const uint32_t sK = smem_u32(smem + kStageOff + (j % kStages) * kStageBytes);
+        const uint32_t tS = tmem + (uint32_t)((j & 1) * kKT);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint64_t a = sdesc(sQ + (kk >> 2) * kQBlock + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc(sK + (kk >> 2) * kKVBlock + (kk & 3) * 32, 16, 1024);
+          umma(tS, a, bd, kIdQK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[j & 1]);
+        return true;
+      };
+      bool ok = mbar_wait_bounded(&q_full, 0u, args.err, DEV_ERR_WAIT_FULL);
+      if (ok) ok = issue_qk(0);
+      if (ok && T > 1) ok = issue_qk(1);
+      for (int j = 0; j < T && ok; ++j) {
+        const int w = j & 1;
+        // O_w += P_w V_j once group w has written P_w for tile j.
+        if (!mbar_wait_bounded(&p_full[w], (uint32_t)(j >> 1) & 1u, args.err, DEV_ERR_WAIT_FULL)) break;
+        tc_fence_after();
+        const uint32_t sV = smem_u32(smem + kStageOff + (j % kStages) * kStageBytes + kKVBytes);
+        const uint32_t sP = smem_u32(smem + kPOff + w * kPBytes);
+        const uint32_t tO = tmem + 128u + (uint32_t)(w * kD);
+#pragma unroll
+        for (int kk = 0; kk < kKT / 16; ++kk) {
+          const uint64_t a = sdesc(sP + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc(sV + kk * 2048, kKVBlock, 1024);
+          umma(tO, a, bd, kIdPV, (j >= 2 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&kv_empty[j % kStages]);
+        umma_commit(&o_done[w]);
+        if (j + 2 < T) ok = issue_qk(j + 2);  // S_w is free: group w has read it
+      }
+    }
+  } else {
+    // ---------------- softmax warpgroups: one query row per thread ----------------
+    const int w = (warp - 2) >> 2;  // 0 = group a (even key tiles), 1 = group b (odd)
+    const int quarter = warp & 3;   // TMEM lane quarter this warp may access
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+    const uint32_t tS = tmem + (uint32_t)(w * kKT) + lane_addr;
+    const uint32_t tO = tmem + 128u + (uint32_t)(w * kD) + lane_addr;
+    const float sl2 = d.scale * 1.4426950408889634f;
+    const int ntiles = T > w ? (T - w + 1) / 2 : 0;
+    float m_used = -CUDART_INF_F, l = 0.f;
+    bool ok = true;
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const int j = 2 * i + w;
+      if (!warp_wait(&s_full[w], (uint32_t)i & 1u, args.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[kKT];
+#pragma unroll
+      for (int c = 0; c < kKT / 32; ++c) {
+        float v[32];
+        tmem_ld32(tS + c * 32, v);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) s[c * 32 + t] = v[t];
+      }
+      tmem_wait_ld();
+      const long long kleft = d.N - (long long)j * kKT;
+      float mt = -CUDART_INF_F;
+#pragma unroll
+      for (int c = 0; c < kKT; ++c) {
+        s[c] = c < kleft ? s[c] * sl2 : -CUDART_INF_F;
+        mt = fmaxf(mt, s[c]);
+      }
+      if (i > 0) {  // PV of this group's previous tile must be done: P_w is overwritten, O_w may be rescaled
+        if (!warp_wait(&o_done[w], (uint32_t)(i - 1) & 1u, args.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+      }
+      if (mt != -CUDART_INF_F && (m_used == -CUDART_INF_F || mt > m_used + 8.f)) {
+        const float alpha = m_used == -CUDART_INF_F ? 0.f : ex2_approx(m_used - mt);
+        l *= alpha;
+        if (i > 0) {
+#pragma unroll
+          for (int c = 0; c < kD / 32; ++c) {
+            float v[32];
+            tmem_ld32(tO + c * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int t = 0; t < 32; ++t) v[t] *= alpha;
+            tmem_st32(tO + c * 32, v);
+          }
+          tmem_wait_st();
+        }
+        m_used = mt;
+      }
+      const float base = m_used == -CUDART_INF_F ? 0.f : m_used;
+      float ps = 0.f;
+      uint8_t* prow = smem + kPOff + w * kPBytes + r * 128;
+#pragma unroll
+      for (int ch = 0; ch < kKT / 8; ++ch) {  // 8 chunks of 8 keys
+        float p[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          p[t] = ex2_approx(s[ch * 8 + t] - base);
+          ps += p[t];
+        }
+        uint4 u;
+        u.x = pack_bf16x2(p[0], p[1]);
+        u.y = pack_bf16x2(p[2], p[3]);
+        u.z = pack_bf16x2(p[4], p[5]);
+        u.w = pack_bf16x2(p[6], p[7]);
+        *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = u;
+      }
+      l += ps;
+      fence_proxy_async_smem();  // P visible to the tensor core (async proxy)
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[w]);
+    }
+    if (ok && ntiles > 0) {
+      ok = warp_wait(&o_done[w], (uint32_t)(ntiles - 1) & 1u, args.err);
+      tc_fence_after();
+    }
+    const bool has = ok && ntiles > 0;  // warp-uniform
+    if (w == 1) {
+      s_mb[r] = has ? m_used : -CUDART_INF_F;
+      s_lb[r] = has ? l : 0.f;
+    }
+    named_barrier_sync(1, 256);
+    if (w == 0) {
+      // Merge the two groups' partial results row by row, then the epilogue.
+      const float ma = has ? m_used : -CUDART_INF_F, la = has ? l : 0.f;
+      const float mb = s_mb[r], lb = s_lb[r];
+      const bool has_b = T > 1;  // group b's O holds data (warp-uniform)
+      const float M = fmaxf(ma, mb);
+      const float wa = (M == -CUDART_INF_F || ma == -CUDART_INF_F) ? 0.f : ex2_approx(ma - M);
+      const float wb = (M == -CUDART_INF_F || mb == -CUDART_INF_F) ? 0.f : ex2_approx(mb - M);
+      const float lt = wa * la + wb * lb;
+      const bool row_has = lt > 0.f;
+      const float inv = row_has ? 1.f / lt : 0.f;
+      const float L = row_has ? (M + __log2f(lt)) * 0.6931471805599453f : -CUDART_INF_F;
+      const bool mine = r < rows_valid && s_flags[r];
+#pragma unroll
+      for (int c = 0; c < kD / 32; ++c) {
+        float va[32], vb[32];
+        if (has) tmem_ld32(tO + c * 32, va);
+        if (has_b) tmem_ld32(tmem + 128u + kD + lane_addr + c * 32, vb);
+        if (has || has_b) tmem_wait_ld();
+        if (!mine) continue;
+#pragma unroll
+        for (int t = 0; t < 32; t += 4) {
+          float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (row_has) {
+            const float fa = wa * inv, fb2 = wb * inv;
+            A.x = (has ? fa * va[t] : 0.f) + (has_b ? fb2 * vb[t] : 0.f);
+            A.y = (has ? fa * va[t + 1] : 0.f) + (has_b ? fb2 * vb[t + 1] : 0.f);
+            A.z = (has ? fa * va[t + 2] : 0.f) + (has_b ? fb2 * vb[t + 2] : 0.f);
+            A.w = (has ? fa * va[t + 3] : 0.f) + (has_b ? fb2 * vb[t + 3] : 0.f);
+          }
+          epilogue4(args.ep, kD, grow0 + r, (c * 32 + t) / 4, A, L);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+}  // namespace
+
+int tc_pass_supported(int D, int R) { return D == kD && R >= kM; }
+
+cudaError_t launch_pass_tc(const PassArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           cudaStream_t s) {
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(pass_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  dim3 grid((a.d.R + kM - 1) / kM, a.d.b * a.d.hkv);
+  pass_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace fb

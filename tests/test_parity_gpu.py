@@ -394,3 +394,48 @@ def test_fused_step_equals_two_call_path(fb, name, B):
         torch.cuda.synchronize()
         for x, y in zip(A, Bt):
             assert torch.equal(x, y), f"step {s.index}"
+
+
+# --------------------------------------------------------------------------- tcgen05 pass (>= 128 rows per KV head)
+
+
+@pytest.mark.parametrize("hq,hkv,B,N", [
+    (1, 1, 128, 128),      # exactly one row tile and one key tile
+    (2, 2, 128, 1000),     # ragged key tail
+    (4, 2, 65, 4097),      # R = 130: two row tiles, the second with 2 rows; GQA
+    (1, 1, 300, 0),        # empty prefix
+    (1, 1, 200, 50),       # fewer keys than one tile
+    (8, 2, 40, 2000),      # R = 160: row tiles straddle query heads
+])
+def test_prefix_tc(fb, hq, hkv, B, N):
+    prefix_case(fb, "bf16", 1, hq, hkv, 128, B, N, seed=hq * 100 + B + N)
+
+
+def test_prefix_tc_batched_strided(fb):
+    # batch 2, row stride 192 and head stride with spare capacity, 2 x 128 rows per KV head
+    prefix_case(fb, "bf16", 2, 4, 2, 128, 64, 3000, seed=44, row_stride=192, cap=3100)
+
+
+def test_prefix_tc_gated_heads(fb):
+    # per-head gate with 256 rows per head: reusing heads keep their cache rows bit for bit
+    b, hq, hkv, D, B, N = 1, 6, 6, 128, 256, 3000
+    q = rand((b, hq, B, D), torch.bfloat16, seed=31)
+    k = rand((b, hkv, N, D), torch.bfloat16, 0.5, 32)
+    v = rand((b, hkv, N, D), torch.bfloat16, 1.0, 33)
+    sh = fb.make_shape(b, hq, hkv, D, B, N, "bf16")
+    sim = torch.tensor([[0.1, 0.9, 0.2, 0.8, 0.6, 0.3]])
+    mask = torch.zeros((b, B), dtype=torch.uint8)
+    a0 = torch.randn((b, hq, B, D)).cuda()
+    l0 = torch.randn((b, hq, B)).cuda()
+    a, l = a0.clone(), l0.clone()
+    ws = workspace(fb, sh)
+    fb.fb_prefix_attn(sh, q.cuda(), k.cuda(), v.cuda(), fb.make_gate(mask.cuda(), False, 1, sim.cuda(), 0.5), a, l, ws)
+    torch.cuda.synchronize()
+    assert fb.fb_device_error() == 0
+    A, L = OF.prefix_attention(f64(q), f64(k), f64(v), 1 / math.sqrt(D))
+    for h in range(hq):
+        if float(sim[0, h]) > 0.5:
+            assert torch.equal(a[0, h], a0[0, h]) and torch.equal(l[0, h], l0[0, h])
+        else:
+            close(f64(a[0, h]), A[0, h], 2e-2, f"A h={h}")
+            close(f64(l[0, h]), L[0, h], 2e-2, f"L h={h}")
