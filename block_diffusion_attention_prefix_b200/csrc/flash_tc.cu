@@ -278,13 +278,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 32; ++t) s[c * 32 + t] = v[t];
       }
       tmem_wait_ld();
+      // Raw scores; the scale (> 0) is applied in the exponent.  Keys past the end
+      // (only in the last tile) are masked.
       const long long kleft = d.N - (long long)j * kKT;
-      float mt = -CUDART_INF_F;
+      if (kleft < kKT) {
 #pragma unroll
-      for (int c = 0; c < kKT; ++c) {
-        s[c] = c < kleft ? s[c] * sl2 : -CUDART_INF_F;
-        mt = fmaxf(mt, s[c]);
+        for (int c = 0; c < kKT; ++c) s[c] = c < kleft ? s[c] : -CUDART_INF_F;
       }
+      float mx0 = s[0], mx1 = s[1];
+#pragma unroll
+      for (int c = 2; c < kKT; c += 2) {
+        mx0 = fmaxf(mx0, s[c]);
+        mx1 = fmaxf(mx1, s[c + 1]);
+      }
+      const float mt = fmaxf(mx0, mx1) * sl2;
       if (i > 0) {  // PV of this group's previous tile must be done: P_w is overwritten, O_w may be rescaled
         if (!warp_wait(&o_done[w], (uint32_t)(i - 1) & 1u, args.err)) {
           ok = false;
@@ -309,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         m_used = mt;
       }
-      const float base = m_used == -CUDART_INF_F ? 0.f : m_used;
+      const float nbase = m_used == -CUDART_INF_F ? 0.f : -m_used;
       float ps = 0.f;
       uint8_t* prow = smem + kPOff + w * kPBytes + r * 128;
 #pragma unroll
@@ -317,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float p[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
-          p[t] = ex2_approx(s[ch * 8 + t] - base);
+          p[t] = ex2_approx(fmaf(s[ch * 8 + t], sl2, nbase));
           ps += p[t];
         }
         uint4 u;
