@@ -369,6 +369,19 @@ def device_arm(args, rank, world):
         torch.cuda.synchronize()
         dense_ms = [e[0].elapsed_time(e[1]) for e in evd]
 
+    # Launch floor: the same event pair around libfb's smallest kernel (the gate
+    # alone: one CTA per batch element) after the same L2 flush.
+    floor = []
+    for i in range(64):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fb.fb_gate_eval(dw.shape, dw.gates[i % npos], wdM, wdR)
+        e1.record()
+        floor.append((e0, e1))
+    torch.cuda.synchronize()
+    floor_us = statistics.median(a.elapsed_time(b) for a, b in floor) * 1e3
+
     e2e = e2e_arm(fb, dw, K, Wm) if (args.e2e and dw.sparse_layer is None) else None
     res = dict(
         metric=METRIC, value=value, unit="steps/s", n_gpus=world, steps=K, warmup=Wm,
@@ -397,6 +410,7 @@ def device_arm(args, rank, world):
                        recompute_step_us=_mean_us(step_ms, recompute_steps),
                        reuse_step_us=_mean_us(step_ms, reuse_steps),
                        reuse_step_alg_bytes=alg_reuse,
+                       launch_floor_us=floor_us,
                        dense_recompute_step_us=(statistics.mean(dense_ms) * 1e3) if dense_ms else None,
                        dense_steps_per_s=(1e3 / statistics.mean(dense_ms)) if dense_ms else None,
                        wall_s=wall),

@@ -91,7 +91,10 @@ __global__ void __launch_bounds__(32 * (D / 16)) page_minmax_kernel(const Sparse
 
 // ------------------------------------------------------------------ page estimates
 
-constexpr int kEstThreads = 256;
+constexpr int kEstPages = 256;  // pages per CTA
+constexpr int kEstRowLanes = 2; // threads per page, each taking every other chunk of rows
+constexpr int kEstRows = 8;     // rows per chunk
+constexpr int kEstThreads = kEstPages * kEstRowLanes;
 
 template <int D>
 __global__ void __launch_bounds__(kEstThreads) page_estimate_kernel(const SparseArgs a) {
@@ -101,9 +104,10 @@ __global__ void __launch_bounds__(kEstThreads) page_estimate_kernel(const Sparse
   const int bg = blockIdx.y, b = bg / d.hkv, kvh = bg - b * d.hkv;
   if (!sparse_recompute(a.gate, b, d.B, s_red)) return;
   const int R = d.R, Rp = (R + 15) / 16 * 16;
-  const int p0 = blockIdx.x * kEstThreads, p = p0 + threadIdx.x;
+  const int p0 = blockIdx.x * kEstPages, p = p0 + (threadIdx.x % kEstPages);
+  const int rlane = threadIdx.x / kEstPages;
   // The union of the group is rebuilt by topk_kernel: clear this chunk's words.
-  if (threadIdx.x < kEstThreads / 32) {
+  if (threadIdx.x < kEstPages / 32) {
     const int w = p0 / 32 + threadIdx.x;
     if (w < a.words) a.union_bits[(size_t)bg * a.words + w] = 0u;
   }
@@ -115,22 +119,32 @@ __global__ void __launch_bounds__(kEstThreads) page_estimate_kernel(const Sparse
   if (p >= a.P) return;
   const bf16* mn = a.kmin + (size_t)bg * D * a.P + p;
   const bf16* mx = a.kmax + (size_t)bg * D * a.P + p;
-  for (int r0 = 0; r0 < R; r0 += 16) {
-    double acc[16];
+  for (int r0 = rlane * kEstRows; r0 < R; r0 += kEstRows * kEstRowLanes) {
+    double acc[kEstRows];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) acc[j] = 0.0;
-    for (int dd = 0; dd < D; ++dd) {
-      const double kmn = (double)__bfloat162float(mn[(size_t)dd * a.P]);
-      const double kmx = (double)__bfloat162float(mx[(size_t)dd * a.P]);
-      const double* qc = sq + (size_t)r0 * D + dd;
+    for (int j = 0; j < kEstRows; ++j) acc[j] = 0.0;
+    for (int d0 = 0; d0 < D; d0 += 8) {
+      // Loads of 8 channels' bounds first (memory-level parallelism), then the
+      // DFMA chains in ascending d.
+      float kn[8], kx[8];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const double qv = qc[(size_t)j * D];
-        acc[j] = fma(qv, qv >= 0.0 ? kmx : kmn, acc[j]);  // exact product, one rounding
+      for (int t = 0; t < 8; ++t) {
+        kn[t] = __bfloat162float(__ldg(mn + (size_t)(d0 + t) * a.P));
+        kx[t] = __bfloat162float(__ldg(mx + (size_t)(d0 + t) * a.P));
+      }
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const double kmn = (double)kn[t], kmx = (double)kx[t];
+        const double* qc = sq + (size_t)r0 * D + d0 + t;
+#pragma unroll
+        for (int j = 0; j < kEstRows; ++j) {
+          const double qv = qc[(size_t)j * D];
+          acc[j] = fma(qv, qv >= 0.0 ? kmx : kmn, acc[j]);  // exact product, one rounding
+        }
       }
     }
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
+    for (int j = 0; j < kEstRows; ++j)
       if (r0 + j < R) a.est[(grow0 + r0 + j) * (size_t)a.P + p] = acc[j];
   }
 }
@@ -172,6 +186,18 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_tmp) {
   return before + x - v;
 }
 
+// KEYS_IN_REGS: each thread holds its (at most 8) keys in registers; otherwise they
+// are recomputed from the estimates in global memory at every pass.
+template <int REG>
+struct KeyCache {
+  unsigned long long k[REG > 0 ? REG : 1];
+  __device__ __forceinline__ void load(const double* est, int pb, int n) {
+#pragma unroll
+    for (int t = 0; t < (REG > 0 ? REG : 1); ++t) k[t] = (REG > 0 && t < n) ? desc_key(est[pb + t]) : ~0ull;
+  }
+};
+
+template <int REG>
 __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) {
   extern __shared__ uint32_t s_bits[];  // [words] row bitmap
   __shared__ unsigned hist[256];
@@ -188,7 +214,13 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
   if (a.k_sel <= 0 || P <= 0) return;
   const int per = (P + kTopkThreads - 1) / kTopkThreads;
   const int pb = min(P, tid * per), pe = min(P, pb + per);
+  const int n = pe - pb;
   const double* est = a.est + (size_t)row * P;
+  KeyCache<REG> kc;
+  kc.load(est, pb, n);
+  // key of the t-th page of this thread (t < n)
+#define FB_KEY(t) (REG > 0 ? kc.k[(t)] : desc_key(est[pb + (t)]))
+#define FB_FOR_MINE(t) _Pragma("unroll") for (int t = 0; t < (REG > 0 ? REG : 1); ++t) if (REG > 0 ? (t < n) : false)
 
   // Radix select (8 passes of 8 bits, most significant first) of the k-th smallest key.
   unsigned long long prefix = 0, mask = 0;
@@ -197,9 +229,16 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
     const int shift = 56 - 8 * pass;
     if (tid < 256) hist[tid] = 0u;
     __syncthreads();
-    for (int p = pb; p < pe; ++p) {
-      const unsigned long long key = desc_key(est[p]);
-      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    if (REG > 0) {
+      FB_FOR_MINE(t) {
+        const unsigned long long key = FB_KEY(t);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
+    } else {
+      for (int t = 0; t < n; ++t) {
+        const unsigned long long key = FB_KEY(t);
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      }
     }
     __syncthreads();
     if (tid < 32) {
@@ -242,13 +281,17 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
 
   // Ties to T go to the lowest pages: rank them in page order, then compact.
   int my_eq = 0;
-  for (int p = pb; p < pe; ++p) my_eq += desc_key(est[p]) == T;
-  int eq_rank = block_exclusive_scan(my_eq, s_tmp);
+  if (REG > 0) {
+    FB_FOR_MINE(t) my_eq += FB_KEY(t) == T;
+  } else {
+    for (int t = 0; t < n; ++t) my_eq += FB_KEY(t) == T;
+  }
+  const int eq_rank = block_exclusive_scan(my_eq, s_tmp);
   int my_take = 0;
   {
     int r = eq_rank;
-    for (int p = pb; p < pe; ++p) {
-      const unsigned long long key = desc_key(est[p]);
+    for (int t = 0; t < n; ++t) {
+      const unsigned long long key = REG > 0 ? desc_key(est[pb + t]) : FB_KEY(t);
       const bool eq = key == T;
       my_take += (key < T) || (eq && r < kk);
       r += eq;
@@ -260,7 +303,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
   {
     int r = eq_rank;
     int32_t* out = a.sel_idx + (size_t)row * a.k_sel;
-    for (int p = pb; p < pe; ++p) {
+    for (int t = 0; t < n; ++t) {
+      const int p = pb + t;
       const unsigned long long key = desc_key(est[p]);
       const bool eq = key == T;
       if ((key < T) || (eq && r < kk)) {
@@ -270,6 +314,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
       r += eq;
     }
   }
+#undef FB_KEY
+#undef FB_FOR_MINE
   __syncthreads();
   uint32_t* rb = a.sel_bits + (size_t)row * a.words;
   uint32_t* ub = a.union_bits + (size_t)(b * d.hkv + kvh) * a.words;
@@ -785,7 +831,7 @@ cudaError_t launch_page_minmax(const SparseArgs& a, cudaStream_t s) {
 
 cudaError_t launch_sparse_select(const SparseArgs& a, cudaStream_t s) {
   const size_t est_smem = (size_t)((a.d.R + 15) / 16 * 16) * a.d.D * sizeof(double);
-  dim3 g1((a.P + kEstThreads - 1) / kEstThreads, a.d.b * a.d.hkv);
+  dim3 g1((a.P + kEstPages - 1) / kEstPages, a.d.b * a.d.hkv);
   cudaError_t e;
   if (a.d.D == 128) {
     e = cudaFuncSetAttribute(page_estimate_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)est_smem);
@@ -798,11 +844,13 @@ cudaError_t launch_sparse_select(const SparseArgs& a, cudaStream_t s) {
   }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const size_t bits_smem = (size_t)a.words * sizeof(uint32_t);
+  const bool regs = a.P <= 8 * kTopkThreads;
+  auto kern = regs ? topk_kernel<8> : topk_kernel<0>;
   if (bits_smem > 48 * 1024) {
-    e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bits_smem);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bits_smem);
     if (e != cudaSuccess) return e;
   }
-  topk_kernel<<<a.d.b * a.d.hq * a.d.B, kTopkThreads, bits_smem, s>>>(a);
+  kern<<<a.d.b * a.d.hq * a.d.B, kTopkThreads, bits_smem, s>>>(a);
   return cudaGetLastError();
 }
 
