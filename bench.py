@@ -354,7 +354,7 @@ def device_arm(args, rank, world):
         tensor = dict(bound="tensor", achieved=tflops, peak=peak_t, unit="TFLOP/s", frac=tflops / peak_t,
                       peak_source="measured sustained cuBLAS bf16 (MEASURED_PEAKS.json bf16_tflops_sustained)",
                       flops_per_step_mean=sum(flops) / K, traffic=None,
-                      kernel="pass_bf16_kernel (prefix pass of recomputing heads + in-block pass)")
+                      kernel="pass_tc_kernel (tcgen05: prefix pass of recomputing heads + in-block pass)")
 
     # dense-recompute reference (standard block diffusion): gate forced to recompute
     dense_ms = []
@@ -395,7 +395,8 @@ def device_arm(args, rank, world):
                     parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
         roofline=dict(bound="hbm", kernel=("sparse step (page estimate + top-k + sparse_pass_kernel), recompute steps"
                                            if dw.sparse_layer is not None else
-                                           ("pass_bf16_kernel" if w.dtype == "bf16" else "pass_f32_kernel")
+                                           (("pass_tc_kernel" if w.block > 64 and w.head_dim == 128 else "pass_bf16_kernel")
+                                            if w.dtype == "bf16" else "pass_f32_kernel")
                                            + (" (fused step: gate + prefix split-KV pass + in-block + merge), "
                                               "recompute launches" if w.block <= 64 else " (prefix split-KV pass)")),
                       achieved=achieved, peak=hbm, unit="GB/s",

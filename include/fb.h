@@ -69,7 +69,7 @@ typedef enum fb_status {
 typedef enum fb_dtype { FB_F32 = 0, FB_BF16 = 1 } fb_dtype;
 
 /* Problem sizes of one attention layer.  head_dim must be 64 or 128 for bf16 and
- * a multiple of 32 up to 256 for fp32.  kv_row_stride / kv_head_stride of 0 mean
+ * a multiple of 32 up to 128 for fp32.  kv_row_stride / kv_head_stride of 0 mean
  * "contiguous" (head_dim and n_prefix * kv_row_stride).  scale of 0 means
  * 1/sqrt(head_dim) (the pages leave the temperature open; this is the standard one). */
 typedef struct fb_shape {
