@@ -395,8 +395,8 @@ def device_arm(args, rank, world):
                     parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
         roofline=dict(bound="hbm", kernel=("sparse step (page estimate + top-k + sparse_pass_kernel), recompute steps"
                                            if dw.sparse_layer is not None else
-                                           (("pass_tc_kernel" if w.block > 64 and w.head_dim == 128 else "pass_bf16_kernel")
-                                            if w.dtype == "bf16" else "pass_f32_kernel")
+                                           (("pass_tc_kernel" if w.group * w.block > 16 and w.head_dim == 128
+                                             else "pass_bf16_kernel") if w.dtype == "bf16" else "pass_f32_kernel")
                                            + (" (fused step: gate + prefix split-KV pass + in-block + merge), "
                                               "recompute launches" if w.block <= 64 else " (prefix split-KV pass)")),
                       achieved=achieved, peak=hbm, unit="GB/s",

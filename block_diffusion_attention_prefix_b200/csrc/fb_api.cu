@@ -222,8 +222,8 @@ int run_pass(const Dims& d0, long long keys, const void* q, const void* k, const
                   ? reinterpret_cast<float*>(static_cast<char*>(ws) + a.plan.counter_bytes + a.plan.partial_bytes)
                   : nullptr;
   a.err = err;
-  if (d.dtype == FB_BF16 && tc_pass_supported(d.D, d.R) && !(step && step->enabled)) {
-    // Dense contraction (>= 128 query rows per KV head): tcgen05 + TMEM, no key split.
+  if (a.plan.tc) {
+    // Dense contraction (more than 16 query rows per KV head): tcgen05 + TMEM.
     CUtensorMap tq, tk, tv;
     const long long qrows = (long long)d.b * d.hq * d.B;
     FB_TRY(encode_kv_map(&tq, q, d.D, qrows, d.D, qrows * d.D, 1, 128));
@@ -249,11 +249,15 @@ size_t pass_bytes(const Dims& d, long long keys, bool with_inblock = false) {
 
 }  // namespace
 
-SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int num_sms, bool with_inblock) {
+SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int num_sms, bool with_inblock,
+                     bool allow_tc) {
   SplitPlan p;
   std::memset(&p, 0, sizeof(p));
   if (dtype == FB_BF16) {
-    p.row_tile = R <= 16 ? 16 : (R <= 32 ? 32 : 64);
+    // More than 16 packed query rows per KV head make the tiles a real dense
+    // contraction: tcgen05 (M = 128, rows past the tile padded); otherwise mma.sync.
+    p.tc = (allow_tc && D == 128 && R > 16) ? 1 : 0;
+    p.row_tile = p.tc ? (R <= 32 ? 32 : (R <= 64 ? 64 : 128)) : (R <= 16 ? 16 : (R <= 32 ? 32 : 64));
     p.key_tile = 64;
   } else {
     p.row_tile = 16;
@@ -264,6 +268,14 @@ SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int n
   const long long units = (long long)b * hkv * p.n_row_tiles;
   const long long total_tiles = (N + p.key_tile - 1) / p.key_tile;
   long long target = (long long)num_sms * ctas_per_sm;
+  if (p.tc && p.row_tile == 128 && !with_inblock && units >= target) {
+    // Enough row tiles to fill the GPU: one CTA per row tile over all keys, no combine.
+    p.tc = 2;
+    p.splits = 1;
+    p.tiles_per_split = (int)total_tiles;
+    p.counter_bytes = 256;  // unused; keeps the workspace non-empty
+    return p;
+  }
   long long splits = units > 0 ? target / units : 1;
   if (splits < 1) splits = 1;
   if (total_tiles > 0 && splits > total_tiles) splits = total_tiles;
@@ -274,7 +286,7 @@ SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int n
     p.tiles_per_split = 0;
     p.splits = 1;
   }
-  p.counter_bytes = ((size_t)units * 4 + 255) / 256 * 256;
+  p.counter_bytes = ((size_t)units * 2 * 4 + 255) / 256 * 256;
   p.partial_bytes = (size_t)units * p.splits * p.row_tile * (D + 4) * sizeof(float);
   p.inblock_bytes = with_inblock ? (size_t)units * p.row_tile * (D + 4) * sizeof(float) : 0;
   return p;
@@ -508,7 +520,7 @@ struct SparseLayout {
 };
 
 int sparse_layout(const Dims& d, int sms, SparseLayout* L) {
-  L->plan = plan_split(d.R, d.D, d.N, d.b, d.hkv, FB_BF16, sms, true);
+  L->plan = plan_split(d.R, d.D, d.N, d.b, d.hkv, FB_BF16, sms, true, false);
   L->P = (int)((d.N + kSparsePage - 1) / kSparsePage);
   L->words = (L->P + 31) / 32;
   const size_t units = (size_t)d.b * d.hkv * L->plan.n_row_tiles;

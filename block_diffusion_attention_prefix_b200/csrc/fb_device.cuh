@@ -101,21 +101,37 @@ __device__ __forceinline__ void store4(void* base, size_t idx, float4 v, int bf1
   }
 }
 
+// The merge equation for one row, in the one rounding order every dense merge of
+// the library uses (so a fused step and the separate calls agree bit for bit):
+// m = max(L1, L2), w_i = e^{L_i - m}, A = (w1 A1 + w2 A2) / (w1 + w2),
+// L = m + ln(w1 + w2).
+struct MergeRow {
+  float w1, w2, rden, l;
+};
+__device__ __forceinline__ MergeRow merge_row(float l1, float l2) {
+  const float m = fmaxf(l1, l2);
+  MergeRow w;
+  w.w1 = m == -CUDART_INF_F ? 0.f : expf(l1 - m);
+  w.w2 = m == -CUDART_INF_F ? 0.f : expf(l2 - m);
+  const float den = w.w1 + w.w2;
+  w.rden = den > 0.f ? 1.f / den : 0.f;
+  w.l = den > 0.f ? m + logf(den) : -CUDART_INF_F;
+  return w;
+}
+__device__ __forceinline__ float merge_val(const MergeRow& w, float a1, float a2) {
+  return fmaf(w.w1, a1, w.w2 * a2) * w.rden;
+}
+
 // The merge equation on one float4 of a row: (A1, L1) and (A2, L2) -> (A, L).
 __device__ __forceinline__ void merge4(float4 a1, float l1, float4 a2, float l2, float4& a, float& l) {
-  const float m = fmaxf(l1, l2);
-  if (m == -CUDART_INF_F) {
+  const MergeRow w = merge_row(l1, l2);
+  l = w.l;
+  if (w.l == -CUDART_INF_F) {
     a = make_float4(0.f, 0.f, 0.f, 0.f);
-    l = -CUDART_INF_F;
     return;
   }
-  const float w1 = expf(l1 - m), w2 = expf(l2 - m);  // exp(-inf) = 0
-  const float inv = 1.f / (w1 + w2);
-  a.x = (w1 * a1.x + w2 * a2.x) * inv;
-  a.y = (w1 * a1.y + w2 * a2.y) * inv;
-  a.z = (w1 * a1.z + w2 * a2.z) * inv;
-  a.w = (w1 * a1.w + w2 * a2.w) * inv;
-  l = m + logf(w1 + w2);
+  a = make_float4(merge_val(w, a1.x, a2.x), merge_val(w, a1.y, a2.y), merge_val(w, a1.z, a2.z),
+                  merge_val(w, a1.w, a2.w));
 }
 
 // Epilogue for one float4 (cols d4*4 .. d4*4+3) of global row `grow` (index into
@@ -307,20 +323,16 @@ __device__ void inblock_rows(const Dims& d, const T* q, const T* k_blk, const T*
       if (lane == 0) ep.l_dst[grow] = L;
       continue;
     }
-    const float m = fmaxf(lp, L);
-    const float wp = m == -CUDART_INF_F ? 0.f : expf(lp - m);
-    const float wi = m == -CUDART_INF_F ? 0.f : expf(L - m);
-    const float den = wp + wi;
-    const float rden = den > 0.f ? 1.f / den : 0.f;
+    const MergeRow w = merge_row(lp, L);
 #pragma unroll
     for (int t = 0; t < DC; ++t) {
-      const float v = (wp * ap[t] + wi * a[t]) * rden;
+      const float v = merge_val(w, ap[t], a[t]);
       if (ep.out_bf16)
         static_cast<__nv_bfloat16*>(ep.a_full)[off + t] = __float2bfloat16_rn(v);
       else
         static_cast<float*>(ep.a_full)[off + t] = v;
     }
-    if (lane == 0 && ep.l_full) ep.l_full[grow] = den > 0.f ? m + logf(den) : -CUDART_INF_F;
+    if (lane == 0 && ep.l_full) ep.l_full[grow] = w.l;
   }
 }
 
@@ -365,6 +377,26 @@ __device__ void merge_tile_from_ws(const Epilogue& ep, size_t grow0, int rows_va
     store4(ep.a_full, off, af, ep.out_bf16);
     if (d4 == 0 && ep.l_full) ep.l_full[grow] = lf;
   }
+}
+
+// Rows [r0, r1) of a tile assigned to split `split` for the in-block pass.
+__device__ __forceinline__ void split_rows(int rows_valid, int splits, int split, int& r0, int& r1) {
+  const int per = (rows_valid + splits - 1) / splits;
+  r0 = min(rows_valid, split * per);
+  r1 = min(rows_valid, r0 + per);
+}
+
+__device__ __forceinline__ Epilogue step_epilogue(const PassArgs& args) {
+  Epilogue ep;
+  ep.mode = 1;
+  ep.a_dst = nullptr;
+  ep.l_dst = nullptr;
+  ep.a_prev = args.ep.a_dst;
+  ep.l_prev = args.ep.l_dst;
+  ep.a_full = args.step.a_full;
+  ep.l_full = args.step.l_full;
+  ep.out_bf16 = 1;
+  return ep;
 }
 
 // Record the gate's decisions for the rows of one tile: dec_reuse[b, h] for every
@@ -512,59 +544,151 @@ __device__ __forceinline__ float4 wsum4(float w1, float4 a, float w2, float4 b) 
   return make_float4(w1 * a.x + w2 * b.x, w1 * a.y + w2 * b.y, w1 * a.z + w2 * b.z, w1 * a.w + w2 * b.w);
 }
 
-// Finish one (b, kv head, row tile) of a dense pass in the CTA that arrived last:
-// combine its splits (combine_regs), then
-//   - rows flagged for recompute: the combined (A, L) goes through `ep`
-//     (mode 0: write the cache rows; mode 1: merge with the cache into A_full);
-//   - fused step (`step_ep` != nullptr): A_full = merge(cache row, in-block row),
-//     the cache row being the one just combined (flagged rows) or the cached one
-//     (rows of reusing heads in a mixed tile); the in-block rows come from the
-//     tile's slot `inblock_slot` in the workspace.
-// `buf` (1024-byte aligned, `buf_bytes`) holds the in-block slot, per-row scalars
-// and the combine's buffer.
-template <int D, int RT, int NT>
-__device__ void finish_tile(const float* part, int splits, const float* inblock_slot, int rows_valid,
-                            const int* s_flags, size_t grow0, const Epilogue& ep, const Epilogue* step_ep,
-                            uint8_t* buf, int buf_bytes, uint64_t* mbar, uint32_t* phase, uint32_t* err, int tid,
-                            int bar_id) {
+// Split-KV combine spread over the split CTAs of one (b, kv head, row tile)
+// (`unit`).  Called by the threads [0, NT) of every split CTA once its partial
+// ([RT][D + 4] fp32, A normalised, natural-log L) and its share of the in-block
+// rows are in the workspace.  The launch is cooperative -- every CTA of the grid
+// is resident -- so a CTA may wait for the other splits of its tile:
+//   1. arrive on arrive[0] (release); wait (acquire, bounded) until all `splits`
+//      CTAs have arrived; depart on depart[0] -- the last to depart resets both
+//      counters for the next launch;
+//   2. bring rows [r0, r1) of every split's partial (the rows whose in-block part
+//      this CTA computed), and those in-block rows, into shared memory with one
+//      1-D bulk copy per split;
+//   3. per row (one warp): M = max_s L_s, e_s = e^{L_s - M}, den = sum_s e_s (a
+//      fixed warp tree), L = M + ln den -- the FlashBlock merge equation over all
+//      splits; per item sum_s e_s A_s in split order, times 1/den.  The order is
+//      fixed, so the result does not depend on timing;
+//   4. epilogue: rows flagged for recompute go through `ep`; in a fused step
+//      (`step_ep`) A_full = merge(cache row, in-block row), the cache row being the
+//      one just combined (flagged rows) or the cached one (rows of reusing heads).
+// `sbuf` (1024-byte aligned, `sbuf_bytes`) is idle shared memory; `mbar` an
+// initialised mbarrier (count 1) whose phases this function alone uses, next
+// parity `*phase`; barrier `bar_id` over NT threads.
+template <int D, int NT>
+__device__ void coop_finish_rows(const float* part, int splits, int RT, int r0, int r1, const float* inblock_slot,
+                                 const int* s_flags, size_t grow0, const Epilogue& ep, const Epilogue* step_ep,
+                                 uint8_t* sbuf, int sbuf_bytes, uint64_t* mbar, uint32_t* phase,
+                                 unsigned int* arrive, unsigned int* depart, uint32_t* err, int tid, int bar_id) {
   constexpr int RS = D + 4;
   constexpr int D4 = D / 4;
-  constexpr int IT = (RT * D4 + NT - 1) / NT;
+  constexpr int NW = NT / 32;
+  const int n = r1 - r0 > 0 ? r1 - r0 : 0;
   const bool step = step_ep != nullptr;
-  const int in_bytes = step ? (RT * RS * 4 + 127) / 128 * 128 : 0;
-  float* s_in = reinterpret_cast<float*>(buf);
-  float* s_L = reinterpret_cast<float*>(buf + in_bytes);  // [RT] merged L, then [RT] w_o, [RT] w_i
-  float* s_wo = s_L + RT;
-  float* s_wi = s_wo + RT;
-  const int hdr = in_bytes + (3 * RT * 4 + 127) / 128 * 128;
-  float4 A[IT];
-  combine_regs<D, RT, NT>(part, splits, step ? inblock_slot : nullptr, s_in, buf + hdr, buf_bytes - hdr, mbar,
-                          phase, err, tid, bar_id, A, s_L);
-  if (step) {
-    for (int r = tid; r < rows_valid; r += NT) {
-      const float lo = s_flags[r] ? s_L[r] : __ldcg(step_ep->l_prev + grow0 + r);
-      float wo, wi, lf;
-      merge_weights(lo, s_in[(size_t)r * RS + D], wo, wi, lf);
-      if (step_ep->l_full) step_ep->l_full[grow0 + r] = lf;
-      s_wo[r] = wo;
-      s_wi[r] = wi;
+  // Shared layout: [splits][n][RS] partial rows | [n][RS] in-block rows | [n][splits] e_s | 5 x [n] row scalars.
+  const size_t a_floats = (size_t)splits * n * RS;
+  const size_t in_floats = step ? (size_t)n * RS : 0;
+  float* sA = reinterpret_cast<float*>(sbuf);
+  float* sIn = sA + a_floats;
+  float* sE = sIn + in_floats;
+  float* sL = sE + (size_t)n * splits;
+  float* sInv = sL + n;
+  float* sWo = sInv + n;  // fused step: the merge of the cache row with the in-block row
+  float* sWi = sWo + n;
+  float* sWr = sWi + n;
+  const bool staged = (a_floats + in_floats + (size_t)n * splits + 5 * (size_t)n) * 4 <= (size_t)sbuf_bytes;
+  fence_proxy_async_smem();         // generic writes to `sbuf` before the bulk copies land there
+  named_barrier_sync(bar_id, NT);  // this CTA's partial and in-block rows are written
+  bool ok = true;
+  unsigned int dep = 0;
+  if (tid == 0) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(arrive) : "memory");
+    ok = wait_count_bounded(arrive, (unsigned)splits, err, DEV_ERR_WAIT_PEERS);
+    dep = atomicAdd(depart, 1u);  // result checked at the end
+    if (ok && staged && n > 0) {
+      fence_proxy_async_global();  // the partials were written through the generic proxy
+      const uint32_t row_bytes = (uint32_t)n * RS * 4;
+      mbar_arrive_expect_tx(mbar, row_bytes * (uint32_t)(splits + (step ? 1 : 0)));
+      for (int sp = 0; sp < splits; ++sp)
+        bulk_load(sA + (size_t)sp * n * RS, part + ((size_t)sp * RT + r0) * RS, row_bytes, mbar);
+      if (step) bulk_load(sIn, inblock_slot + (size_t)r0 * RS, row_bytes, mbar);
+    }
+  }
+  ok = named_barrier_and(bar_id, NT, ok);
+  if (ok && n > 0) {
+    if (staged) {
+      ok = mbar_wait_bounded(mbar, *phase, err, DEV_ERR_WAIT_COMBINE);
+      *phase ^= 1u;
+    }
+    ok = named_barrier_and(bar_id, NT, ok);
+    // Source rows: shared memory when staged, else the workspace itself (L2).
+    auto ld1 = [&](int sp, int rr) -> float {
+      return staged ? sA[((size_t)sp * n + rr) * RS + D] : __ldcg(part + ((size_t)sp * RT + r0 + rr) * RS + D);
+    };
+    auto ld4 = [&](int sp, int rr, int d4) -> float4 {
+      return staged ? reinterpret_cast<const float4*>(sA + ((size_t)sp * n + rr) * RS)[d4]
+                    : __ldcg(reinterpret_cast<const float4*>(part + ((size_t)sp * RT + r0 + rr) * RS) + d4);
+    };
+    auto in1 = [&](int rr) -> float {
+      return staged ? sIn[(size_t)rr * RS + D] : __ldcg(inblock_slot + (size_t)(r0 + rr) * RS + D);
+    };
+    auto in4 = [&](int rr, int d4) -> float4 {
+      return staged ? reinterpret_cast<const float4*>(sIn + (size_t)rr * RS)[d4]
+                    : __ldcg(reinterpret_cast<const float4*>(inblock_slot + (size_t)(r0 + rr) * RS) + d4);
+    };
+    const int warp = tid >> 5, lane = tid & 31;
+    for (int rr = warp; rr < n && ok; rr += NW) {
+      float M = -CUDART_INF_F;
+      for (int sp = lane; sp < splits; sp += 32) M = fmaxf(M, ld1(sp, rr));
+      M = warp_max(M);
+      float den = 0.f;
+      for (int sp = lane; sp < splits; sp += 32) {
+        const float e = M == -CUDART_INF_F ? 0.f : expf(ld1(sp, rr) - M);
+        sE[(size_t)rr * splits + sp] = e;
+        den += e;
+      }
+      den = warp_sum(den);
+      if (lane == 0) {
+        const int r = r0 + rr;
+        const float L = den > 0.f ? M + logf(den) : -CUDART_INF_F;
+        sL[rr] = L;
+        sInv[rr] = den > 0.f ? 1.f / den : 0.f;
+        if (step) {
+          const float lo = s_flags[r] ? L : __ldcg(step_ep->l_prev + grow0 + r);
+          const MergeRow w = merge_row(lo, in1(rr));
+          if (step_ep->l_full) step_ep->l_full[grow0 + r] = w.l;
+          sWo[rr] = w.w1;
+          sWi[rr] = w.w2;
+          sWr[rr] = w.rden;
+        }
+      }
     }
     named_barrier_sync(bar_id, NT);
-  }
-#pragma unroll
-  for (int k = 0; k < IT; ++k) {
-    const int idx = tid + k * NT;
-    if (idx >= RT * D4) continue;
-    const int r = idx / D4, d4 = idx - r * D4;
-    if (r >= rows_valid) continue;
-    const size_t grow = grow0 + r;
-    if (s_flags[r]) epilogue4(ep, D, grow, d4, A[k], s_L[r]);
-    if (step) {
-      const size_t off = grow * D + (size_t)d4 * 4;
-      const float4 ap = s_flags[r] ? A[k] : __ldcg(reinterpret_cast<const float4*>(step_ep->a_prev + off));
-      const float4 ai = *reinterpret_cast<const float4*>(s_in + (size_t)r * RS + d4 * 4);
-      store4(step_ep->a_full, off, wsum4(s_wo[r], ap, s_wi[r], ai), step_ep->out_bf16);
+    for (int idx = tid; idx < n * D4 && ok; idx += NT) {
+      const int rr = idx / D4, d4 = idx - rr * D4;
+      const int r = r0 + rr;
+      const float* er = sE + (size_t)rr * splits;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sp = 0; sp < splits; ++sp) {
+        const float w = er[sp];
+        const float4 x = ld4(sp, rr, d4);
+        a.x = fmaf(w, x.x, a.x);
+        a.y = fmaf(w, x.y, a.y);
+        a.z = fmaf(w, x.z, a.z);
+        a.w = fmaf(w, x.w, a.w);
+      }
+      const float sc = sInv[rr];
+      const float4 A = make_float4(a.x * sc, a.y * sc, a.z * sc, a.w * sc);
+      const size_t grow = grow0 + r;
+      if (s_flags[r]) epilogue4(ep, D, grow, d4, A, sL[rr]);
+      if (step) {
+        const size_t off = grow * D + (size_t)d4 * 4;
+        const float4 ap = s_flags[r] ? A : __ldcg(reinterpret_cast<const float4*>(step_ep->a_prev + off));
+        const float4 ai = in4(rr, d4);
+        MergeRow w;
+        w.w1 = sWo[rr];
+        w.w2 = sWi[rr];
+        w.rden = sWr[rr];
+        store4(step_ep->a_full, off,
+               make_float4(merge_val(w, ap.x, ai.x), merge_val(w, ap.y, ai.y), merge_val(w, ap.z, ai.z),
+                           merge_val(w, ap.w, ai.w)),
+               step_ep->out_bf16);
+      }
     }
+  }
+  if (tid == 0 && dep == (unsigned)splits - 1u) {  // every split has seen the full count
+    *arrive = 0u;
+    *depart = 0u;
   }
 }
 

@@ -44,7 +44,8 @@ struct SplitPlan {
   int key_tile;         // keys per pipeline tile
   int splits;           // CTAs along the key axis per (b, kv head, row tile)
   int tiles_per_split;  // key tiles per split
-  size_t counter_bytes; // arrival counters, one per (b, kv head, row tile), 256-B padded
+  int tc;               // 0: mma.sync / CUDA-core pass; 1: tcgen05 split pass; 2: tcgen05, one CTA per row tile
+  size_t counter_bytes; // arrival then departure counters, one each per (b, kv head, row tile), 256-B padded
   size_t partial_bytes; // [b*hkv][n_row_tiles][splits][row_tile][D + 4] fp32
   size_t inblock_bytes; // fused step only: [b*hkv][n_row_tiles][row_tile][D + 4] fp32 (A_in, L_in)
   size_t total() const { return counter_bytes + partial_bytes + inblock_bytes; }
@@ -128,15 +129,14 @@ cudaError_t launch_sparse_select(const SparseArgs& a, cudaStream_t s);
 cudaError_t launch_sparse_pass(const SparseArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s);
 
 SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int num_sms,
-                     bool with_inblock = false);
+                     bool with_inblock = false, bool allow_tc = true);
 
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_pass_f32(const PassArgs& a, cudaStream_t s);
 cudaError_t launch_pass_bf16(const PassArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                              cudaStream_t s);
 int bf16_pass_supported(int D, int row_tile);
-// tcgen05 pass (flash_tc.cu): bf16, D = 128, at least 128 query rows per KV head.
-int tc_pass_supported(int D, int R);
+// tcgen05 pass (flash_tc.cu): bf16, D = 128, more than 16 query rows per KV head.
 cudaError_t launch_pass_tc(const PassArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            cudaStream_t s);
 

@@ -16,6 +16,7 @@ enum : uint32_t {
   DEV_ERR_WAIT_FULL = 1,   // consumer gave up waiting for a TMA tile
   DEV_ERR_WAIT_EMPTY = 2,  // producer gave up waiting for a free stage
   DEV_ERR_WAIT_COMBINE = 3, // last CTA gave up waiting for its partials copy
+  DEV_ERR_WAIT_PEERS = 4,   // a split CTA gave up waiting for the other splits of its tile
 };
 
 // 2 s: far above any legitimate wait (a tile load takes microseconds).
@@ -73,6 +74,22 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (err) atomicCAS(err, 0u, code);
+      return false;
+    }
+  }
+}
+
+// Wait until the global counter *p reaches `target` (acquire), at most kWaitLimitNs.
+// Only for counters that CTAs of the same (cooperative) launch increment.
+__device__ __forceinline__ bool wait_count_bounded(const unsigned int* p, unsigned int target, uint32_t* err,
+                                                   uint32_t code) {
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    if (v >= target) return true;
     if (globaltimer_ns() - t0 > kWaitLimitNs) {
       if (err) atomicCAS(err, 0u, code);
       return false;

@@ -1,14 +1,23 @@
 // flash_tc.cu -- attention pass on the 5th-generation tensor cores (tcgen05 + TMEM).
 //
-// For passes with at least 128 query rows per KV head (video blocks: 4680 block
-// queries per head over a 31,200-token prefix and over the 4680 block keys) the
-// contraction is dense: 128 x 128 x 128 tiles on tcgen05.mma with fp32
-// accumulators in tensor memory.  Same contract as the split pass
-// (prefix_bf16.cu): (A, L) per query row over a key set -- the out-of-block part
-// over J_out, or the in-block part over J_in merged with the cache
-// (FlashBlock technical summary, gist.science 2602.05305, "Core mechanism").
+// Used when more than 16 query rows share a KV head (GQA packing: B x G rows), so
+// the tiles are a real dense contraction: 128 x 64 x 128 score tiles and
+// 128 x 128 x 64 output tiles on tcgen05.mma with fp32 accumulators in tensor
+// memory.  Same contract as the mma.sync pass (prefix_bf16.cu): (A, L) per query
+// row over a key set -- the out-of-block part over J_out, or the in-block part
+// over J_in -- and, in a fused step, the in-block rows, the merge with the cache
+// and the decision record (FlashBlock technical summary, gist.science
+// 2602.05305, "Core mechanism" and "Adaptive reuse strategies").
 //
-// One CTA = 128 query rows of one KV group, all keys (no split), 320 threads:
+// A CTA owns a row tile of RT = 32, 64 or 128 rows of one KV group (the MMA is
+// always M = 128; TMEM lanes past RT are padding whose softmax is skipped) and
+//   SPLIT:  one key range of the split-KV grid (splits, row tiles, b * H_kv).  It
+//           writes a normalised partial; once all splits of the tile have arrived
+//           (cooperative launch: all CTAs resident), each split CTA combines its
+//           share of the rows in fixed split order (deterministic) and runs the
+//           epilogue -- small blocks, where row tiles alone cannot fill the GPU;
+//   !SPLIT: all keys, epilogue directly (large blocks: video, 4680 rows per head).
+// 352 threads:
 //   warp 0     TMA producer: Q once; 64-key K and V tiles into a 4-stage ring
 //              (128-byte swizzle, no multicast).
 //   warp 1     TMEM owner and MMA issuer (one thread):
@@ -23,8 +32,8 @@
 //              (bf16) into shared memory.  O_w is rescaled in TMEM only when a row's
 //              max grows by more than 2^8 (otherwise the stale max is kept; p <= 2^8
 //              is exact enough in bf16 and cannot overflow fp32).  At the end group a
-//              merges the two partial results (the FlashBlock log-space merge) and
-//              writes the cache or merges with it into A_full.
+//              merges the two partial results (the FlashBlock log-space merge).
+//   warp 10    fused step: this split's share of the tile's in-block rows.
 // TMEM: 512 columns (S_a [0,64), S_b [64,128), O_a [128,256), O_b [256,384)).
 // Every mbarrier wait is time bounded; on expiry the roles fall through to the
 // common exit, which frees TMEM.
@@ -44,7 +53,10 @@ constexpr int kM = 128;
 constexpr int kKT = 64;   // keys per tile
 constexpr int kD = 128;
 constexpr int kStages = 4;
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;  // 11 warps
+constexpr int kAuxWarp = 10;
+constexpr int kBarSoftmax = 1;  // the 8 softmax warps
+constexpr int kBarFinish = 2;   // every warp (split combine)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kQBlock = 128 * 128;               // Q: [128 rows][128 B] per 64-column block
 constexpr int kQBytes = 2 * kQBlock;
@@ -56,6 +68,7 @@ constexpr int kQOff = 0;
 constexpr int kStageOff = kQBytes;
 constexpr int kPOff = kStageOff + kStages * kStageBytes;
 constexpr int kSmemBytes = kPOff + 2 * kPBytes + 1024;
+constexpr int kBufBytes = kSmemBytes - 1024;  // all of it, reused by the split combine
 
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2, version 1).
 // K-major: 8-row groups 1024 B apart (SBO); LBO unused (1).  MN-major: LBO is the
@@ -133,9 +146,13 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint32
   return __all_sync(0xffffffffu, ok);
 }
 
+template <int RT, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     pass_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const PassArgs args) {
+  static_assert(RT % 32 == 0 && RT <= kM, "row tile: whole TMEM lane quarters of the 128-row accumulator");
+  constexpr int kRealWarps = RT / 32;  // softmax warps per group whose TMEM lanes hold tile rows
+  using bf16 = __nv_bfloat16;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t q_full;
@@ -144,21 +161,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ __align__(8) uint64_t s_full[2];
   __shared__ __align__(8) uint64_t p_full[2];
   __shared__ __align__(8) uint64_t o_done[2];
+  __shared__ __align__(8) uint64_t fin_bar;
   __shared__ uint32_t s_tmem;
-  __shared__ int s_flags[kM];
+  __shared__ int s_flags[RT];
   __shared__ int s_red[32];
-  __shared__ float s_mb[kM], s_lb[kM];  // group b's row max / sum for the final merge
+  __shared__ int s_M;
+  __shared__ float s_mb[RT], s_lb[RT];  // group b's row max / sum for the final merge
 
   const Dims& d = args.d;
+  const SplitPlan& plan = args.plan;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int rt = blockIdx.x, bg = blockIdx.y;
+  const int split = SPLIT ? (int)blockIdx.x : 0;
+  const int rt = SPLIT ? (int)blockIdx.y : (int)blockIdx.x;
+  const int bg = SPLIT ? (int)blockIdx.z : (int)blockIdx.y;
   const int b = bg / d.hkv, kvh = bg - b * d.hkv;
-  const int row0 = rt * kM;
-  const int rows_valid = min(kM, d.R - row0);
+  const int row0 = rt * RT;
+  const int rows_valid = min(RT, d.R - row0);
   const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B + row0;
-  const int T = (int)((d.N + kKT - 1) / kKT);
+  const size_t unit = (size_t)bg * plan.n_row_tiles + rt;
+  const long long key_begin = SPLIT ? (long long)split * plan.tiles_per_split * kKT : 0;
+  const long long key_end = SPLIT ? min(d.N, key_begin + (long long)plan.tiles_per_split * kKT) : d.N;
+  const int T = key_end > key_begin ? (int)((key_end - key_begin + kKT - 1) / kKT) : 0;
+  const bf16* q = static_cast<const bf16*>(args.q);
+  const bf16* k_blk = static_cast<const bf16*>(args.step.k_blk);
+  const bf16* v_blk = static_cast<const bf16*>(args.step.v_blk);
 
-  if (!gate_row_flags(args.gate, d, b, kvh, row0, rows_valid, kM, s_flags, s_red)) return;
+  if (!gate_row_flags(args.gate, d, b, kvh, row0, rows_valid, RT, s_flags, s_red, &s_M)) {
+    // Every row of this tile reuses its cache: no K/V is read.  In a fused step the
+    // tile's CTAs still produce the step's output from the cache.
+    if (SPLIT && args.step.enabled) {
+      int r0, r1;
+      split_rows(rows_valid, plan.splits, split, r0, r1);
+      inblock_rows<bf16, kD>(d, q, k_blk, v_blk, b, kvh, row0, r0, r1, step_epilogue(args), warp, kThreads / 32,
+                             lane);
+      if (split == 0)
+        record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, s_M, args.step.dec_M,
+                         args.step.dec_reuse, kvh == 0 && rt == 0, tid, kThreads);
+    }
+    return;
+  }
 
   if (tid == 0) {
     mbar_init(&q_full, 1);
@@ -168,9 +209,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&s_full[w], 1);
-      mbar_init(&p_full[w], 4);
+      mbar_init(&p_full[w], kRealWarps);
       mbar_init(&o_done[w], 1);
     }
+    mbar_init(&fin_bar, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -200,9 +242,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         mbar_arrive_expect_tx(&kv_full[s], kStageBytes);
         uint8_t* st = smem + kStageOff + s * kStageBytes;
+        const int key0 = (int)(key_begin + (long long)j * kKT);
         for (int h = 0; h < 2; ++h) {
-          tma_load_3d(st + h * kKVBlock, &tmK, &kv_full[s], h * 64, j * kKT, bg);
-          tma_load_3d(st + kKVBytes + h * kKVBlock, &tmV, &kv_full[s], h * 64, j * kKT, bg);
+          tma_load_3d(st + h * kKVBlock, &tmK, &kv_full[s], h * 64, key0, bg);
+          tma_load_3d(st + kKVBytes + h * kKVBlock, &tmV, &kv_full[s], h * 64, key0, bg);
         }
         ++issued;
       }
@@ -250,16 +293,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j + 2 < T) ok = issue_qk(j + 2);  // S_w is free: group w has read it
       }
     }
+  } else if (warp == kAuxWarp) {
+    // ---------------- aux warp: this split's share of the in-block rows ----------------
+    if (SPLIT && args.step.enabled) {
+      int r0, r1;
+      split_rows(rows_valid, plan.splits, split, r0, r1);
+      inblock_rows_to_ws<bf16, kD>(d, q, k_blk, v_blk, b, kvh, row0, r0, r1, args.inblock + unit * RT * (kD + 4),
+                                   0, 1, lane);
+    }
   } else {
     // ---------------- softmax warpgroups: one query row per thread ----------------
     const int w = (warp - 2) >> 2;  // 0 = group a (even key tiles), 1 = group b (odd)
     const int quarter = warp & 3;   // TMEM lane quarter this warp may access
+    const bool real = quarter < kRealWarps;  // warp-uniform: lanes past the row tile are padding
     const int r = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem + (uint32_t)(w * kKT) + lane_addr;
     const uint32_t tO = tmem + 128u + (uint32_t)(w * kD) + lane_addr;
     const float sl2 = d.scale * 1.4426950408889634f;
-    const int ntiles = T > w ? (T - w + 1) / 2 : 0;
+    const int ntiles = (real && T > w) ? (T - w + 1) / 2 : 0;
     float m_used = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int i = 0; i < ntiles && ok; ++i) {
@@ -279,8 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tmem_wait_ld();
       // Raw scores; the scale (> 0) is applied in the exponent.  Keys past the end
-      // (only in the last tile) are masked.
-      const long long kleft = d.N - (long long)j * kKT;
+      // of the range (only in its last tile) are masked.
+      const long long kleft = key_end - key_begin - (long long)j * kKT;
       if (kleft < kKT) {
 #pragma unroll
         for (int c = 0; c < kKT; ++c) s[c] = c < kleft ? s[c] : -CUDART_INF_F;
@@ -345,13 +397,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
     }
     const bool has = ok && ntiles > 0;  // warp-uniform
-    if (w == 1) {
+    if (w == 1 && real) {
       s_mb[r] = has ? m_used : -CUDART_INF_F;
       s_lb[r] = has ? l : 0.f;
     }
-    named_barrier_sync(1, 256);
-    if (w == 0) {
-      // Merge the two groups' partial results row by row, then the epilogue.
+    named_barrier_sync(kBarSoftmax, 256);
+    if (w == 0 && real) {
+      // Merge the two groups' partial results row by row (the FlashBlock merge).
       const float ma = has ? m_used : -CUDART_INF_F, la = has ? l : 0.f;
       const float mb = s_mb[r], lb = s_lb[r];
       const bool has_b = T > 1;  // group b's O holds data (warp-uniform)
@@ -362,7 +414,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool row_has = lt > 0.f;
       const float inv = row_has ? 1.f / lt : 0.f;
       const float L = row_has ? (M + __log2f(lt)) * 0.6931471805599453f : -CUDART_INF_F;
-      const bool mine = r < rows_valid && s_flags[r];
+      // SPLIT: this CTA's partial row (A normalised, L natural) into the workspace,
+      // for every row of the tile; otherwise the epilogue for recomputed rows.
+      float* prow = SPLIT ? args.partials + ((unit * plan.splits + split) * RT + r) * (size_t)(kD + 4) : nullptr;
+      const bool mine = SPLIT ? true : (r < rows_valid && s_flags[r]);
 #pragma unroll
       for (int c = 0; c < kD / 32; ++c) {
         float va[32], vb[32];
@@ -380,9 +435,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             A.z = (has ? fa * va[t + 2] : 0.f) + (has_b ? fb2 * vb[t + 2] : 0.f);
             A.w = (has ? fa * va[t + 3] : 0.f) + (has_b ? fb2 * vb[t + 3] : 0.f);
           }
-          epilogue4(args.ep, kD, grow0 + r, (c * 32 + t) / 4, A, L);
+          if (SPLIT)
+            *reinterpret_cast<float4*>(prow + c * 32 + t) = A;
+          else
+            epilogue4(args.ep, kD, grow0 + r, (c * 32 + t) / 4, A, L);
         }
       }
+      if (SPLIT) prow[kD] = L;
     }
   }
   tc_fence_before();
@@ -391,25 +450,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
+  if constexpr (SPLIT) {
+    // Every split CTA combines its share of the tile's rows once all splits have
+    // arrived (cooperative launch); the shared memory is idle now.
+    int r0, r1;
+    split_rows(rows_valid, plan.splits, split, r0, r1);
+    const Epilogue sep = step_epilogue(args);
+    const size_t nunits = (size_t)d.b * d.hkv * plan.n_row_tiles;
+    uint32_t fin_phase = 0;
+    coop_finish_rows<kD, kThreads>(args.partials + unit * plan.splits * RT * (kD + 4), plan.splits, RT, r0, r1,
+                                   args.step.enabled ? args.inblock + unit * RT * (kD + 4) : nullptr, s_flags,
+                                   grow0, args.ep, args.step.enabled ? &sep : nullptr, smem, kBufBytes, &fin_bar,
+                                   &fin_phase, args.counters + unit, args.counters + nunits + unit, args.err, tid,
+                                   kBarFinish);
+    if (args.step.enabled && split == 0)
+      record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, s_M, args.step.dec_M, args.step.dec_reuse,
+                       kvh == 0 && rt == 0, tid, kThreads);
+  }
 }
 
-}  // namespace
-
-int tc_pass_supported(int D, int R) { return D == kD && R >= kM; }
-
-cudaError_t launch_pass_tc(const PassArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                           cudaStream_t s) {
+template <int RT, bool SPLIT>
+cudaError_t launch_tc(const PassArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                      cudaStream_t s) {
+  auto kern = pass_tc_kernel<RT, SPLIT>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(pass_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  dim3 grid((a.d.R + kM - 1) / kM, a.d.b * a.d.hkv);
-  pass_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(tq, tk, tv, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = SPLIT ? dim3(a.plan.splits, a.plan.n_row_tiles, a.d.b * a.d.hkv)
+                      : dim3(a.plan.n_row_tiles, a.d.b * a.d.hkv);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // the split CTAs of a tile wait for one another
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = (SPLIT && a.plan.splits > 1) ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, a);
+}
+
+}  // namespace
+
+cudaError_t launch_pass_tc(const PassArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                           cudaStream_t s) {
+  if (a.plan.tc == 2) return a.plan.row_tile == kM ? launch_tc<kM, false>(a, tq, tk, tv, s) : cudaErrorInvalidValue;
+  switch (a.plan.row_tile) {
+    case 32: return launch_tc<32, true>(a, tq, tk, tv, s);
+    case 64: return launch_tc<64, true>(a, tq, tk, tv, s);
+    case 128: return launch_tc<128, true>(a, tq, tk, tv, s);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 }  // namespace fb

@@ -17,16 +17,16 @@
 //    warp (wm, wn) owns query rows [16 wm, 16 wm + 16) and keys
 //    [wn * KW, (wn + 1) * KW) of every tile; Q stays in registers; the online
 //    softmax (running max / sum in base 2) stays in registers.
-//  * At the end, warps of the same rows merge in shared memory, the CTA writes
-//    its partial (A normalised, L natural) to the workspace, and the last CTA to
-//    arrive on the (b, kv head, row tile) counter merges all splits in fixed
-//    order (deterministic) and runs the epilogue (write the cache, or merge with
-//    the cache into A_full).  The counter is reset by that CTA.  The combine
-//    brings the partials into the (now idle) ring with 1-D bulk TMA copies.
+//  * At the end, warps of the same rows merge in shared memory and the CTA writes
+//    its partial (A normalised, L natural) to the workspace.  The launch is
+//    cooperative (every CTA resident), so the split CTAs of a (b, kv head, row
+//    tile) wait for one another on a counter and then each combines its share of
+//    the tile's rows over all splits in fixed order (deterministic) and runs the
+//    epilogue (write the cache, or merge with the cache into A_full).
 //  * Fused step (small blocks): the in-block rows of a tile are spread over its
-//    split CTAs (aux warps) and parked in the workspace; the finishing CTA merges
-//    them with the combined cache rows into A_full and records the decisions, so
-//    a denoising step is one launch.  When every row of a tile reuses the cache,
+//    split CTAs (aux warps), the same rows each CTA combines, so each CTA also
+//    merges them with the combined cache rows into A_full; split 0 records the
+//    decisions, so a denoising step is one launch.  When every row of a tile reuses the cache,
 //    its CTAs read no K/V at all: they merge their in-block rows with the cache.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -66,34 +66,15 @@ struct Cfg {
   static constexpr int kSmemBytes = (kRingBytes > kScratchBytes ? kRingBytes : kScratchBytes) + 1024;
   static_assert(KW % 16 == 0, "each warp needs whole k16 steps of keys");
   static_assert(D % 64 == 0, "D must be a multiple of 64");
-  // Finisher: in-block slot + per-row scalars + weights of up to 148 splits + one split's partial.
-  static_assert(kRingBytes >= 2 * kRowTile * (D + 4) * 4 + 256 + 3 * kRowTile * 4 + ((150 * kRowTile * 4 + 127) / 128) * 128,
-                "finisher needs the in-block slot, the weights and one split");
+  // The combine stages (rows x (splits + 1)) partial rows, rows <= ceil(RT / splits):
+  // at most 2 RT + 149 rows for up to 148 splits (it reads the workspace directly
+  // when they do not fit).
+  static_assert(kRingBytes >= (2 * kRowTile + 149) * (D + 4) * 4 + 8192, "combine staging");
 };
 
 // Barrier ids: 0 = whole CTA, 1 = consumer warps, 2 = consumer + aux warps.
 constexpr int kBarConsumers = 1;
 constexpr int kBarFinish = 2;
-
-// Rows [r0, r1) of a tile assigned to split `split` for the in-block pass.
-__device__ __forceinline__ void split_rows(int rows_valid, int splits, int split, int& r0, int& r1) {
-  const int per = (rows_valid + splits - 1) / splits;
-  r0 = min(rows_valid, split * per);
-  r1 = min(rows_valid, r0 + per);
-}
-
-__device__ __forceinline__ Epilogue step_epilogue(const PassArgs& args) {
-  Epilogue ep;
-  ep.mode = 1;
-  ep.a_dst = nullptr;
-  ep.l_dst = nullptr;
-  ep.a_prev = args.ep.a_dst;
-  ep.l_prev = args.ep.l_dst;
-  ep.a_full = args.step.a_full;
-  ep.l_full = args.step.l_full;
-  ep.out_bf16 = 1;
-  return ep;
-}
 
 template <int D, int WARPS_M, int WARPS_N, int STAGES>
 __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
@@ -109,10 +90,9 @@ __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t full_bar[STAGES];
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
-  __shared__ __align__(8) uint64_t comb_bar;
+  __shared__ __align__(8) uint64_t fin_bar;
   __shared__ int s_flags[RT];
   __shared__ int s_red[32];
-  __shared__ int s_last;
   __shared__ int s_M;
 
   const Dims& d = args.d;
@@ -156,7 +136,7 @@ __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], NCW);
     }
-    mbar_init(&comb_bar, 1);
+    mbar_init(&fin_bar, 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -380,28 +360,22 @@ __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
     }
   }
 
-  // ------------- consumers + aux: arrive; the last CTA finishes the tile -------------
-  named_barrier_sync(kBarFinish, C::kFinishThreads);
-  if (tid == 0) {
-    __threadfence();  // release this CTA's partial and in-block rows (cumulative over the barrier)
-    const unsigned prev = atomicAdd(args.counters + unit, 1u);
-    __threadfence();  // acquire the other CTAs' writes when last
-    s_last = (prev == (unsigned)plan.splits - 1u);
-  }
-  named_barrier_sync(kBarFinish, C::kFinishThreads);
-  if (!s_last) return;
+  // ---- consumers + aux: once every split has arrived, combine this CTA's share of the rows ----
   // Finisher threads are the consumer warps and the aux warp: number them 0..kFinishThreads-1.
   const int ftid = warp < NCW ? tid : NCW * 32 + lane;
-  uint32_t comb_phase = 0;
+  int r0, r1;
+  split_rows(rows_valid, plan.splits, split, r0, r1);
   const Epilogue sep = step_epilogue(args);
-  finish_tile<D, RT, C::kFinishThreads>(args.partials + unit * plan.splits * RT * (D + 4), plan.splits,
-                                        args.step.enabled ? args.inblock + unit * RT * (D + 4) : nullptr,
-                                        rows_valid, s_flags, grow0, args.ep, args.step.enabled ? &sep : nullptr,
-                                        smem, C::kRingBytes, &comb_bar, &comb_phase, args.err, ftid, kBarFinish);
-  if (args.step.enabled)
+  const size_t nunits = (size_t)d.b * d.hkv * plan.n_row_tiles;
+  uint32_t fin_phase = 0;
+  coop_finish_rows<D, C::kFinishThreads>(args.partials + unit * plan.splits * RT * (D + 4), plan.splits, RT, r0, r1,
+                                         args.step.enabled ? args.inblock + unit * RT * (D + 4) : nullptr, s_flags,
+                                         grow0, args.ep, args.step.enabled ? &sep : nullptr, smem, C::kRingBytes,
+                                         &fin_bar, &fin_phase, args.counters + unit, args.counters + nunits + unit,
+                                         args.err, ftid, kBarFinish);
+  if (args.step.enabled && split == 0)
     record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, s_M, args.step.dec_M, args.step.dec_reuse,
                      kvh == 0 && rt == 0, ftid, C::kFinishThreads);
-  if (tid == 0) args.counters[unit] = 0u;
 }
 
 template <int D, int WM, int WN, int STAGES>
@@ -416,9 +390,17 @@ cudaError_t launch_cfg(const PassArgs& a, const CUtensorMap& tk, const CUtensorM
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  dim3 grid(a.plan.splits, a.plan.n_row_tiles, a.d.b * a.d.hkv);
-  kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(tk, tv, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.plan.splits, a.plan.n_row_tiles, a.d.b * a.d.hkv);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // the split CTAs of a tile wait for one another
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.plan.splits > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, tk, tv, a);
 }
 
 }  // namespace

@@ -133,7 +133,7 @@ def test_prefix_f32(fb, N, D, hq, hkv, B):
 
 @pytest.mark.parametrize("N", [0, 1, 63, 64, 65, 1000, 4097])
 @pytest.mark.parametrize("D,hq,hkv,B", [(128, 32, 8, 4), (128, 8, 2, 16), (64, 8, 4, 8), (128, 3, 3, 3),
-                                        (64, 4, 2, 37)])
+                                        (64, 4, 2, 37), (128, 8, 2, 8)])
 def test_prefix_bf16(fb, N, D, hq, hkv, B):
     prefix_case(fb, "bf16", 1, hq, hkv, D, B, N, seed=N * 7 + D + B)
 
@@ -352,7 +352,8 @@ def test_video_gamma_full_size_sampled(fb):
     dict(name="dlm8b_b4", n_prefix=5000, seed=7),
     dict(name="dlm8b_b4", n_prefix=0, seed=8),                          # empty prefix
     dict(name="dlm8b_b4", n_prefix=3001, block=37, tau=10, seed=9),     # heads straddle row tiles
-    dict(name="dlm8b_b16", n_prefix=4000, block=64, tau=20, seed=10),   # 4 row tiles of 64
+    dict(name="dlm8b_b16", n_prefix=4000, block=64, tau=20, seed=10),   # 256 rows per KV head: 2 row tiles
+    dict(name="dlm8b_b4", n_prefix=3000, block=8, tau=3, seed=14),      # 32 rows per KV head
     dict(name="tiny_f32", n_prefix=777, block=33, h_q=4, h_kv=2, tau=9, seed=11),
 ])
 def test_fused_step_schedules(fb, variant):
@@ -396,7 +397,7 @@ def test_fused_step_equals_two_call_path(fb, name, B):
             assert torch.equal(x, y), f"step {s.index}"
 
 
-# --------------------------------------------------------------------------- tcgen05 pass (>= 128 rows per KV head)
+# --------------------------------------------------------------------------- tcgen05 pass (> 16 rows per KV head)
 
 
 @pytest.mark.parametrize("hq,hkv,B,N", [
@@ -406,6 +407,9 @@ def test_fused_step_equals_two_call_path(fb, name, B):
     (1, 1, 300, 0),        # empty prefix
     (1, 1, 200, 50),       # fewer keys than one tile
     (8, 2, 40, 2000),      # R = 160: row tiles straddle query heads
+    (1, 1, 128, 7296),     # 114 key tiles: the most splits a 128-row tile combines
+    (1, 1, 128, 7327),     # same with a ragged tail
+    (12, 12, 1600, 700),   # 13 row tiles x 12 heads fill the GPU: one CTA per row tile, no split
 ])
 def test_prefix_tc(fb, hq, hkv, B, N):
     prefix_case(fb, "bf16", 1, hq, hkv, 128, B, N, seed=hq * 100 + B + N)

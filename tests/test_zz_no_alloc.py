@@ -52,8 +52,9 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(fb):
 
 
 def test_noalloc_rejects_shapes_beyond_the_static_array(fb):
-    # the video layer's prefix pass needs about 30 MB of split partials: more than 8 MiB
-    b, hq, hkv, D, B, N = 1, 12, 12, 128, 4680, 31200
+    # a dLM-8B-like layer with 64-token blocks (256 query rows per KV head) needs
+    # about 9.7 MB of split partials for its prefix pass: more than 8 MiB
+    b, hq, hkv, D, B, N = 1, 32, 8, 128, 64, 32768
     shape = fb.make_shape(b, hq, hkv, D, B, N, "bf16")
     assert fb.fb_workspace_bytes(shape) > 8 << 20
     q = torch.zeros((b, hq, B, D), dtype=torch.bfloat16, device="cuda")
