@@ -382,6 +382,28 @@ def device_arm(args, rank, world):
     torch.cuda.synchronize()
     floor_us = statistics.median(a.elapsed_time(b) for a, b in floor) * 1e3
 
+    # Block transition (once per block, after its last step): fb_append_block of one
+    # block into a cache with room, with the page-bound refresh in sparse mode.
+    n0, cap = 64, 64 + w.block
+    kc = torch.zeros((w.batch, w.h_kv, cap, w.head_dim), device=dev, dtype=w.torch_dtype)
+    vc = torch.zeros_like(kc)
+    kb = torch.randn((w.batch, w.h_kv, w.block, w.head_dim), device=dev).to(w.torch_dtype)
+    tsh = fb.make_shape(w.batch, w.h_q, w.h_kv, w.head_dim, w.block, n0, w.dtype, kv_head_stride=cap * w.head_dim)
+    kmn = kmx = None
+    if dw.sparse_layer is not None:
+        kmn = torch.zeros((w.batch, w.h_kv, w.head_dim, (cap + 15) // 16), device=dev, dtype=w.torch_dtype)
+        kmx = torch.zeros_like(kmn)
+    trans = []
+    for i in range(32):
+        flush()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fb.fb_append_block(tsh, kc, vc, kb, kb, 16, kmn, kmx)
+        e1.record()
+        trans.append((e0, e1))
+    torch.cuda.synchronize()
+    trans_us = statistics.median(a.elapsed_time(b) for a, b in trans) * 1e3
+
     e2e = e2e_arm(fb, dw, K, Wm) if (args.e2e and dw.sparse_layer is None) else None
     res = dict(
         metric=METRIC, value=value, unit="steps/s", n_gpus=world, steps=K, warmup=Wm,
@@ -412,6 +434,7 @@ def device_arm(args, rank, world):
                        reuse_step_us=_mean_us(step_ms, reuse_steps),
                        reuse_step_alg_bytes=alg_reuse,
                        launch_floor_us=floor_us,
+                       block_transition_us=trans_us,
                        dense_recompute_step_us=(statistics.mean(dense_ms) * 1e3) if dense_ms else None,
                        dense_steps_per_s=(1e3 / statistics.mean(dense_ms)) if dense_ms else None,
                        wall_s=wall),

@@ -9,6 +9,10 @@
 //    mechanism" merge equation and "Adaptive reuse strategies" gates.)
 //  * gate_kernel: the gate alone (M^{s+1} and the per-head decisions).
 //  * merge_kernel: the merge equation alone, elementwise, 16-byte vectors.
+//  * append_block_kernel: the block transition -- once a block's last step is
+//    done its tokens belong to the prefix: their K/V rows are copied to the end
+//    of the prefix cache (the prefix J_out grows by B; FlashBlock technical
+//    summary, "1. Problem definition").
 //
 // The in-block scores are B x B per head (B <= 64): CUDA cores, fp32 math.
 #include <cuda_bf16.h>
@@ -75,6 +79,24 @@ __global__ void merge_kernel(const Dims d, const float* a1, const float* l1, con
   }
 }
 
+// Block transition: one CTA per (b, KV head) copies the block's B rows of K and V
+// into cache rows [N, N + B) (16-byte vectors; rows of the cache may be padded).
+__global__ void append_block_kernel(const Dims d, uint8_t* k_cache, uint8_t* v_cache, const uint8_t* k_blk,
+                                    const uint8_t* v_blk, int elem_bytes) {
+  const int bg = blockIdx.x;
+  const int vec_per_row = d.D * elem_bytes / 16;
+  const size_t n = (size_t)d.B * vec_per_row;
+  const size_t src0 = (size_t)bg * d.B * d.D * elem_bytes;
+  const size_t dst0 = ((size_t)bg * d.head_stride + (size_t)d.N * d.row_stride) * elem_bytes;
+  for (size_t i = threadIdx.x; i < 2 * n; i += blockDim.x) {
+    const bool isv = i >= n;
+    const size_t j = isv ? i - n : i;
+    const size_t row = j / vec_per_row, c = j - row * vec_per_row;
+    const uint4 x = __ldg(reinterpret_cast<const uint4*>((isv ? v_blk : k_blk) + src0 + row * d.D * elem_bytes) + c);
+    reinterpret_cast<uint4*>((isv ? v_cache : k_cache) + dst0 + row * d.row_stride * elem_bytes)[c] = x;
+  }
+}
+
 template <typename T>
 cudaError_t launch_small_t(const SmallBlockArgs& a, cudaStream_t s) {
   dim3 grid(a.d.hq, a.d.b);
@@ -97,6 +119,14 @@ cudaError_t launch_small_block(const SmallBlockArgs& a, cudaStream_t s) {
 cudaError_t launch_gate_eval(const Dims& d, const GateParams& g, int32_t* dec_M, uint8_t* dec_reuse,
                              cudaStream_t s) {
   gate_kernel<<<d.b, 128, 0, s>>>(d, g, dec_M, dec_reuse);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_block(const Dims& d, void* k_cache, void* v_cache, const void* k_blk, const void* v_blk,
+                                cudaStream_t s) {
+  append_block_kernel<<<d.b * d.hkv, 256, 0, s>>>(d, static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache),
+                                                   static_cast<const uint8_t*>(k_blk),
+                                                   static_cast<const uint8_t*>(v_blk), d.dtype == 1 ? 2 : 4);
   return cudaGetLastError();
 }
 

@@ -534,6 +534,14 @@ int sparse_layout(const Dims& d, int sms, SparseLayout* L) {
   return FB_OK;
 }
 
+// Pages the K cache's row capacity holds (the page stride of the bounds layout):
+// rows r with r * row_stride + D <= head_stride, at least N.
+int page_capacity(const Dims& d) {
+  long long rows = d.row_stride > 0 ? (d.head_stride - d.D) / d.row_stride + 1 : d.N;
+  if (rows < d.N) rows = d.N;
+  return (int)((rows + kSparsePage - 1) / kSparsePage);
+}
+
 int sparse_check(const fb_shape* shape, const fb_gate* gate, const fb_sparse* sp, Dims* d, GateParams* gp) {
   FB_TRY(resolve(shape, d));
   if (!sp) return FB_ERR_NULL;
@@ -572,6 +580,7 @@ int sparse_args(const Dims& d, const GateParams& gp, const fb_sparse* sp, const 
   a->d = d;
   a->plan = L.plan;
   a->P = L.P;
+  a->Pcap = page_capacity(d);
   a->k_sel = sp->n_select;
   a->words = L.words;
   a->q = q;
@@ -612,6 +621,44 @@ extern "C" int fb_page_minmax(const fb_shape* shape, const void* k_cache, int pa
   std::memset(&a, 0, sizeof(a));
   a.d = d;
   a.P = (int)((d.N + kSparsePage - 1) / kSparsePage);
+  a.Pcap = page_capacity(d);
+  a.p_first = 0;
+  a.k = k_cache;
+  a.kmin_out = static_cast<__nv_bfloat16*>(kmin);
+  a.kmax_out = static_cast<__nv_bfloat16*>(kmax);
+  return cuda_status(launch_page_minmax(a, (cudaStream_t)stream));
+}
+
+extern "C" int fb_append_block(const fb_shape* shape, void* k_cache, void* v_cache, const void* k_blk,
+                               const void* v_blk, int page_size, void* kmin, void* kmax, fb_stream_t stream) {
+  Dims d;
+  FB_TRY(resolve(shape, &d));
+  if (!shape->kv_head_stride) return FB_ERR_SHAPE;  // a contiguous cache has no room to grow
+  // Row capacity per head: rows r with r * row_stride + D <= head_stride.
+  const long long cap = (d.head_stride - d.D) / d.row_stride + 1;
+  if (d.N + d.B > cap || d.N + d.B > (1LL << 31) - 64) return FB_ERR_SHAPE;
+  FB_TRY(check_ptr(k_cache));
+  FB_TRY(check_ptr(v_cache));
+  FB_TRY(check_ptr(k_blk));
+  FB_TRY(check_ptr(v_blk));
+  const bool bounds = kmin || kmax;
+  if (bounds) {
+    if (d.dtype != FB_BF16) return FB_ERR_DTYPE;
+    if (page_size != kSparsePage) return FB_ERR_ARG;
+    FB_TRY(check_ptr(kmin));
+    FB_TRY(check_ptr(kmax));
+  }
+  FB_TRY(cuda_status(launch_append_block(d, k_cache, v_cache, k_blk, v_blk, (cudaStream_t)stream)));
+  if (!bounds) return FB_OK;
+  // Page bounds of the grown prefix: only the pages the new rows fall in change
+  // (the first may be a partial page that already holds old rows).
+  SparseArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.d = d;
+  a.d.N = d.N + d.B;
+  a.P = (int)((a.d.N + kSparsePage - 1) / kSparsePage);
+  a.Pcap = page_capacity(a.d);
+  a.p_first = (int)(d.N / kSparsePage);
   a.k = k_cache;
   a.kmin_out = static_cast<__nv_bfloat16*>(kmin);
   a.kmax_out = static_cast<__nv_bfloat16*>(kmax);

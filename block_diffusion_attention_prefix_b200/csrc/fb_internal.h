@@ -99,11 +99,13 @@ struct SparseArgs {
   Dims d;                 // N = prefix tokens
   SplitPlan plan;         // splits over 64-key (4-page) tiles
   int P;                  // pages (16 tokens each)
+  int Pcap;               // page stride of the bounds layout: pages the K cache's capacity holds
+  int p_first;            // page_minmax: first page to (re)compute
   int k_sel;              // pages selected per query row
   int words;              // ceil(P / 32)
   const void* q;
   const void* k;          // prefix K (page bounds only)
-  const __nv_bfloat16* kmin;   // [b*H_kv][D][P]
+  const __nv_bfloat16* kmin;   // [b*H_kv][D][Pcap], pages [0, P) valid
   const __nv_bfloat16* kmax;
   __nv_bfloat16* kmin_out;     // page bounds output
   __nv_bfloat16* kmax_out;
@@ -156,5 +158,8 @@ cudaError_t launch_gate_eval(const Dims& d, const GateParams& g, int32_t* dec_M,
                              cudaStream_t s);
 cudaError_t launch_merge(const Dims& d, const float* a1, const float* l1, const float* a2,
                          const float* l2, void* a_full, float* l_full, cudaStream_t s);
+// Block transition: copy the block's K/V ([b, H_kv, B, D]) into cache rows [N, N + B).
+cudaError_t launch_append_block(const Dims& d, void* k_cache, void* v_cache, const void* k_blk, const void* v_blk,
+                                cudaStream_t s);
 
 }  // namespace fb

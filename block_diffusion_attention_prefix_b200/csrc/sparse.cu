@@ -12,8 +12,10 @@
 // k = ceil(density * pages) by (e desc, page asc).
 //
 // Kernels:
-//  * page_minmax_kernel: kmin / kmax [b*H_kv][D][pages] (channel-major so that
-//    the estimate reads coalesce), exact bf16.
+//  * page_minmax_kernel: kmin / kmax [b*H_kv][D][page capacity] (channel-major
+//    so that the estimate reads coalesce; the page stride is what the K cache's
+//    row capacity holds, so a growing prefix keeps its layout), exact bf16; pages
+//    [p_first, P), so a block transition refreshes only the pages it touched.
 //  * page_estimate_kernel: e for every (row, page) of recomputing batch
 //    elements; one thread per page runs the 16 rows' float64 DFMA chains
 //    (max(q kmin, q kmax) is the product picked by the sign of q, exactly).
@@ -56,7 +58,7 @@ template <int D>
 __global__ void __launch_bounds__(32 * (D / 16)) page_minmax_kernel(const SparseArgs a) {
   const int lane = threadIdx.x & 31, chunk = threadIdx.x >> 5;  // 16 channels per warp
   const int bg = blockIdx.y;
-  const int p = blockIdx.x * 32 + lane;
+  const int p = a.p_first + blockIdx.x * 32 + lane;
   if (p >= a.P) return;
   const bf16* kp = static_cast<const bf16*>(a.k) + (size_t)bg * a.d.head_stride +
                    (size_t)p * kPage * a.d.row_stride + chunk * 16;
@@ -80,12 +82,12 @@ __global__ void __launch_bounds__(32 * (D / 16)) page_minmax_kernel(const Sparse
       mx[2 * t + 1] = fmaxf(mx[2 * t + 1], f.y);
     }
   }
-  bf16* omn = a.kmin_out + (size_t)bg * D * a.P + (size_t)(chunk * 16) * a.P + p;
-  bf16* omx = a.kmax_out + (size_t)bg * D * a.P + (size_t)(chunk * 16) * a.P + p;
+  bf16* omn = a.kmin_out + (size_t)bg * D * a.Pcap + (size_t)(chunk * 16) * a.Pcap + p;
+  bf16* omx = a.kmax_out + (size_t)bg * D * a.Pcap + (size_t)(chunk * 16) * a.Pcap + p;
 #pragma unroll
   for (int t = 0; t < 16; ++t) {
-    omn[(size_t)t * a.P] = __float2bfloat16_rn(mn[t]);  // exact: the inputs are bf16
-    omx[(size_t)t * a.P] = __float2bfloat16_rn(mx[t]);
+    omn[(size_t)t * a.Pcap] = __float2bfloat16_rn(mn[t]);  // exact: the inputs are bf16
+    omx[(size_t)t * a.Pcap] = __float2bfloat16_rn(mx[t]);
   }
 }
 
@@ -117,8 +119,8 @@ __global__ void __launch_bounds__(kEstThreads) page_estimate_kernel(const Sparse
     sq[i] = i < R * D ? (double)__bfloat162float(qg[i]) : 0.0;
   __syncthreads();
   if (p >= a.P) return;
-  const bf16* mn = a.kmin + (size_t)bg * D * a.P + p;
-  const bf16* mx = a.kmax + (size_t)bg * D * a.P + p;
+  const bf16* mn = a.kmin + (size_t)bg * D * a.Pcap + p;
+  const bf16* mx = a.kmax + (size_t)bg * D * a.Pcap + p;
   for (int r0 = rlane * kEstRows; r0 < R; r0 += kEstRows * kEstRowLanes) {
     double acc[kEstRows];
 #pragma unroll
@@ -129,8 +131,8 @@ __global__ void __launch_bounds__(kEstThreads) page_estimate_kernel(const Sparse
       float kn[8], kx[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
-        kn[t] = __bfloat162float(__ldg(mn + (size_t)(d0 + t) * a.P));
-        kx[t] = __bfloat162float(__ldg(mx + (size_t)(d0 + t) * a.P));
+        kn[t] = __bfloat162float(__ldg(mn + (size_t)(d0 + t) * a.Pcap));
+        kx[t] = __bfloat162float(__ldg(mx + (size_t)(d0 + t) * a.Pcap));
       }
 #pragma unroll
       for (int t = 0; t < 8; ++t) {
@@ -819,7 +821,8 @@ cudaError_t launch_sparse_cfg(const SparseArgs& a, const CUtensorMap& tk, const 
 int sparse_supported(int D, int row_tile) { return (D == 64 || D == 128) && (row_tile == 16 || row_tile == 32); }
 
 cudaError_t launch_page_minmax(const SparseArgs& a, cudaStream_t s) {
-  dim3 grid((a.P + 31) / 32, a.d.b * a.d.hkv);
+  if (a.P <= a.p_first) return cudaSuccess;
+  dim3 grid((a.P - a.p_first + 31) / 32, a.d.b * a.d.hkv);
   if (a.d.D == 128)
     page_minmax_kernel<128><<<grid, 32 * 8, 0, s>>>(a);
   else if (a.d.D == 64)

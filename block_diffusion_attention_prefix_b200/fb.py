@@ -17,7 +17,7 @@ __all__ = [
     "FBError", "Shape", "Gate", "load", "lib_path", "make_shape", "make_gate", "FB_F32", "FB_BF16",
     "fb_version", "fb_status_string", "fb_device_error", "fb_workspace_bytes", "fb_workspace_init",
     "fb_gate_eval", "fb_prefix_attn", "fb_prefix_attn_noalloc", "fb_block_attn", "fb_merge", "fb_block_merge", "fb_step",
-    "fb_page_minmax", "fb_sparse_workspace_bytes", "fb_sparse_select", "fb_sparse_step", "Sparse",
+    "fb_page_minmax", "fb_append_block", "fb_sparse_workspace_bytes", "fb_sparse_select", "fb_sparse_step", "Sparse",
     "SparseResidualLayer", "CachedAttentionLayer", "EXPORTED",
 ]
 
@@ -81,6 +81,7 @@ EXPORTED = {
     "fb_step": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _PG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fb_prefix_attn_noalloc": (_i, [_PS, _vp, _vp, _vp, _PG, _vp, _vp, _vp]),
     "fb_page_minmax": (_i, [_PS, _vp, _i, _vp, _vp, _vp]),
+    "fb_append_block": (_i, [_PS, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
     "fb_sparse_workspace_bytes": (_sz, [_PS, _i]),
     "fb_sparse_select": (_i, [_PS, _vp, _PG, _PSP, _vp, _sz, _vp]),
     "fb_sparse_step": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _PG, _PSP, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -220,6 +221,12 @@ def fb_page_minmax(shape, k_cache, page_size, kmin, kmax):
                                                    _ptr(kmax), _stream()))
 
 
+def fb_append_block(shape, k_cache, v_cache, k_blk, v_blk, page_size=16, kmin=None, kmax=None):
+    _check("fb_append_block", load().fb_append_block(ctypes.byref(shape), _ptr(k_cache), _ptr(v_cache), _ptr(k_blk),
+                                                     _ptr(v_blk), int(page_size), _ptr(kmin), _ptr(kmax),
+                                                     _stream()))
+
+
 def fb_sparse_workspace_bytes(shape, page_size=16) -> int:
     return int(load().fb_sparse_workspace_bytes(ctypes.byref(shape), int(page_size)))
 
@@ -243,14 +250,19 @@ class SparseResidualLayer:
     """
 
     def __init__(self, batch, h_q, h_kv, head_dim, block, k_cache, v_cache, n_select, page_size=16, scale=0.0,
-                 keep_sel=False):
+                 keep_sel=False, n_prefix=None):
+        # k_cache / v_cache [b, H_kv, capacity, D]; n_prefix (default: capacity) rows are the prefix.
         dev = k_cache.device
-        n = k_cache.shape[2]
-        self.shape = make_shape(batch, h_q, h_kv, head_dim, block, n, k_cache.dtype, scale=scale)
+        cap = k_cache.shape[2]
+        n = cap if n_prefix is None else int(n_prefix)
+        self.shape = make_shape(batch, h_q, h_kv, head_dim, block, n, k_cache.dtype, scale=scale,
+                                kv_head_stride=0 if n_prefix is None else cap * head_dim)
         self.k_cache, self.v_cache = k_cache, v_cache
+        self.page_size = page_size
         self.n_pages = (n + page_size - 1) // page_size
         words = (self.n_pages + 31) // 32
-        self.kmin = torch.empty((batch, h_kv, head_dim, self.n_pages), device=dev, dtype=k_cache.dtype)
+        page_cap = (cap + page_size - 1) // page_size
+        self.kmin = torch.empty((batch, h_kv, head_dim, page_cap), device=dev, dtype=k_cache.dtype)
         self.kmax = torch.empty_like(self.kmin)
         fb_page_minmax(self.shape, k_cache, page_size, self.kmin, self.kmax)
         i32, f32 = dict(device=dev, dtype=torch.int32), dict(device=dev, dtype=torch.float32)
@@ -277,6 +289,27 @@ class SparseResidualLayer:
                        self.l_full, self.dec_M, self.dec_reuse, self.ws)
         return self.a_full
 
+    def finish_block(self, k_blk, v_blk, n_select):
+        """Block transition: append the block's K/V to the prefix, refresh the page
+        bounds it touched, and size the selection state for the grown prefix."""
+        fb_append_block(self.shape, self.k_cache, self.v_cache, k_blk, v_blk, self.page_size, self.kmin, self.kmax)
+        sh = self.shape
+        self.shape = make_shape(sh.batch, sh.h_q, sh.h_kv, sh.head_dim, sh.block, sh.n_prefix + sh.block, sh.dtype,
+                                kv_row_stride=sh.kv_row_stride, kv_head_stride=sh.kv_head_stride, scale=sh.scale)
+        self.n_pages = (self.shape.n_prefix + self.page_size - 1) // self.page_size
+        words = (self.n_pages + 31) // 32
+        b, hq, B = sh.batch, sh.h_q, sh.block
+        dev = self.k_cache.device
+        self.sel_idx = torch.zeros((b, hq, B, n_select), device=dev, dtype=torch.int32)
+        self.sel_bits = torch.zeros((b, hq, B, words), device=dev, dtype=torch.int32)
+        self.union_bits = torch.zeros((b, sh.h_kv, words), device=dev, dtype=torch.int32)
+        nbytes = fb_sparse_workspace_bytes(self.shape, self.page_size)
+        self.ws = torch.zeros(((nbytes + 15) // 16 * 16,), device=dev, dtype=torch.uint8)
+        sp = self.sparse
+        self.sparse = Sparse(sp.page_size, n_select, sp.kmin, sp.kmax, self.sel_idx.data_ptr(),
+                             self.sel_bits.data_ptr(), self.union_bits.data_ptr(), sp.a_res, sp.l_res, sp.a_sel,
+                             sp.l_sel)
+
 
 class CachedAttentionLayer:
     """Device buffers of one attention layer's FlashBlock state, stepped through fb_step.
@@ -286,10 +319,13 @@ class CachedAttentionLayer:
     """
 
     def __init__(self, batch, h_q, h_kv, head_dim, block, k_cache: torch.Tensor, v_cache: torch.Tensor,
-                 scale: float = 0.0, device=None):
+                 scale: float = 0.0, device=None, n_prefix=None):
+        # k_cache / v_cache [b, H_kv, capacity, D]; n_prefix (default: capacity) rows are the prefix.
         dev = k_cache.device if device is None else device
         self.dtype = k_cache.dtype
-        self.shape = make_shape(batch, h_q, h_kv, head_dim, block, k_cache.shape[2], k_cache.dtype, scale=scale)
+        cap = k_cache.shape[2]
+        self.shape = make_shape(batch, h_q, h_kv, head_dim, block, cap if n_prefix is None else int(n_prefix),
+                                k_cache.dtype, scale=scale, kv_head_stride=0 if n_prefix is None else cap * head_dim)
         self.k_cache, self.v_cache = k_cache, v_cache
         f32 = dict(device=dev, dtype=torch.float32)
         self.a_out = torch.zeros((batch, h_q, block, head_dim), **f32)
@@ -306,3 +342,14 @@ class CachedAttentionLayer:
         fb_step(self.shape, q, self.k_cache, self.v_cache, k_blk, v_blk, g, self.a_out, self.l_out,
                 self.a_full, self.l_full, self.dec_M, self.dec_reuse, self.ws)
         return self.a_full
+
+    def finish_block(self, k_blk, v_blk):
+        """Block transition: append the block's K/V to the prefix (the cache needs the
+        capacity); the next block starts with first_step=True."""
+        fb_append_block(self.shape, self.k_cache, self.v_cache, k_blk, v_blk)
+        sh = self.shape
+        self.shape = make_shape(sh.batch, sh.h_q, sh.h_kv, sh.head_dim, sh.block, sh.n_prefix + sh.block, sh.dtype,
+                                kv_row_stride=sh.kv_row_stride, kv_head_stride=sh.kv_head_stride, scale=sh.scale)
+        nbytes = fb_workspace_bytes(self.shape)
+        if nbytes > self.ws.numel():
+            self.ws = torch.zeros(((nbytes + 15) // 16 * 16,), device=self.ws.device, dtype=torch.uint8)

@@ -188,6 +188,13 @@ def block_schedule(w: Workload, seed: int, steps: Optional[int] = None) -> Itera
                    mask=mask, sim=sim)
 
 
+def generation_schedule(w: Workload, seed: int, blocks: int, steps: Optional[int] = None):
+    """Several consecutive blocks (inputs only): a list per block of its denoising
+    steps.  Block t draws from seed + 7919 * t; the block's keys and values as of its
+    last step are what joins the prefix when the block is finished."""
+    return [list(block_schedule(w, seed + 7919 * t, steps)) for t in range(blocks)]
+
+
 def default_scale(head_dim: int) -> float:
     """Softmax temperature used when the caller passes 0: 1/sqrt(D)."""
     return 1.0 / math.sqrt(head_dim)

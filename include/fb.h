@@ -178,8 +178,12 @@ int fb_step(const fb_shape* shape, const void* q, const void* k_cache, const voi
 typedef struct fb_sparse {
   int32_t page_size;      /* 16 */
   int32_t n_select;       /* pages per query row, 1 .. n_pages */
-  const void* kmin;       /* [b, H_kv, D, n_pages] bf16 page minima (fb_page_minmax) */
-  const void* kmax;       /* [b, H_kv, D, n_pages] bf16 page maxima */
+  const void* kmin;       /* [b, H_kv, D, page_cap] bf16 page minima (fb_page_minmax), pages
+                             [0, n_pages) valid; page_cap = ceil(cap / page_size) with cap the
+                             K cache's row capacity per head (rows r with
+                             r * kv_row_stride + head_dim <= kv_head_stride; = n_prefix for a
+                             contiguous cache), so the layout survives fb_append_block */
+  const void* kmax;       /* same layout, page maxima */
   int32_t* sel_idx;       /* state [b, H_q, B, n_select] int32, selected pages ascending */
   uint32_t* sel_bits;     /* state [b, H_q, B, words] bitmap of the same pages */
   uint32_t* union_bits;   /* state [b, H_kv, words] union over the KV group's rows */
@@ -193,6 +197,27 @@ typedef struct fb_sparse {
  * page's real tokens; the last page may be partial). */
 int fb_page_minmax(const fb_shape* shape, const void* k_cache, int page_size, void* kmin, void* kmax,
                    fb_stream_t stream);
+
+/* Block transition (after the last denoising step of a block): the block's tokens
+ * join the prefix.  FlashBlock technical summary (gist.science 2602.05305),
+ * "1. Problem definition": attention splits into the current block J_in and the
+ * tokens outside it, J_out, which are the earlier blocks -- so when a block is
+ * finished its keys and values are appended to the prefix cache and the next
+ * block's J_out is one block longer.
+ *
+ * shape->n_prefix is N before the call; k_blk / v_blk ([b, H_kv, B, D], the block's
+ * keys and values as of its last step) are copied into cache rows [N, N + B) of
+ * every (b, KV head).  The cache must have room: shape->kv_head_stride must be
+ * given (non-zero) and hold at least N + B rows of kv_row_stride (FB_ERR_SHAPE
+ * otherwise).  When kmin / kmax are non-NULL (bf16, page_size 16; layout as in
+ * fb_sparse, with the page stride of the capacity) the page bounds of the pages
+ * the new rows fall in are recomputed over their real tokens; other pages keep
+ * theirs.  Afterwards the caller uses n_prefix = N + B.  The cached (A_out,
+ * L_out) of the finished block is stale for the next block, whose step 0
+ * recomputes it (first_step).  All pointers caller-owned device memory,
+ * 16-byte aligned; asynchronous on `stream`. */
+int fb_append_block(const fb_shape* shape, void* k_cache, void* v_cache, const void* k_blk, const void* v_blk,
+                    int page_size, void* kmin, void* kmax, fb_stream_t stream);
 
 /* Workspace of fb_sparse_select / fb_sparse_step (split partials of both parts,
  * in-block rows, page estimates, counters; same reuse rules as fb_workspace_bytes). */

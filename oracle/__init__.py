@@ -22,6 +22,7 @@ Modules:
 * :mod:`oracle.attention`  -- softmax attention over a key set as (A, L), and the merge.
 * :mod:`oracle.flashblock` -- the tau / gamma gates and the stateful cached step.
 * :mod:`oracle.sparse`     -- page bounds, top-k page selection and the residual split.
+* :mod:`oracle.transition` -- the block transition: a finished block joins the prefix.
 
 Pins: every function here is pinned by ``tests/test_oracle_*.py`` against
 library routines (torch float64 SDPA, logsumexp, full sorts), closed forms and

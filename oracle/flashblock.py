@@ -150,3 +150,11 @@ class CachedBlockAttention:
         a_full, l_full = merge(self.a_out, self.l_out, a_in, l_in)
         return StepResult(M=M, reuse=reuse, a_full=a_full, l_full=l_full,
                           a_out=self.a_out.copy(), l_out=self.l_out.copy())
+
+    def finish_block(self, k_blk, v_blk) -> None:
+        """Block transition (:mod:`oracle.transition`): the block's K/V join the
+        prefix; the next block starts afresh (first step recomputes)."""
+        from .transition import append_block
+        self.k, self.v = append_block(self.k, self.v, k_blk, v_blk)
+        self.a_out = None
+        self.l_out = None

@@ -132,6 +132,7 @@ class SparseResidualAttention:
         self.v = np.asarray(v_cache, dtype=np.float64)
         b, hk, N, D = self.k.shape
         self.h_q, self.scale, self.page = h_q, scale, page
+        self.density = density
         self.N = N
         self.P = n_pages(N, page)
         self.k_sel = n_selected(N, page, density)
@@ -178,3 +179,20 @@ class SparseResidualAttention:
         return SparseStepResult(M=M, reuse=reuse, sel=self.sel.copy(), union=union,
                                 a_full=a_full, l_full=l_full, a_res=self.a_res.copy(),
                                 l_res=self.l_res.copy(), a_sel=a_sel, l_sel=l_sel)
+
+    def finish_block(self, k_blk, v_blk) -> None:
+        """Block transition (:mod:`oracle.transition`, readings T1-T3): the block's
+        K/V join the prefix, the page bounds the new rows touch are refreshed, k
+        follows the grown page count, and the next block starts afresh."""
+        from .transition import append_block, update_page_minmax
+        n_old = self.N
+        self.k, self.v = append_block(self.k, self.v, k_blk, v_blk)
+        b, hk, N, D = self.k.shape
+        self.bounds = [[update_page_minmax(*self.bounds[bi][g], self.k[bi, g], n_old, self.page)
+                        for g in range(hk)] for bi in range(b)]
+        self.N = N
+        self.P = n_pages(N, self.page)
+        self.k_sel = n_selected(N, self.page, self.density)
+        self.sel = None
+        self.a_res = None
+        self.l_res = None

@@ -10,10 +10,12 @@ import pytest
 import oracle.attention as OA
 import oracle.flashblock as OF
 import oracle.sparse as OS
+import oracle.transition as OT
 
 from tests import test_oracle_attention as TA
 from tests import test_oracle_flashblock as TF
 from tests import test_oracle_sparse as TS
+from tests import test_oracle_transition as TT
 
 _orig_attend = OA.attend
 _orig_merge = OA.merge
@@ -84,6 +86,21 @@ def _select_high_tie(est, k_sel):
     return out
 
 
+_orig_update = OT.update_page_minmax
+_orig_append = OT.append_block
+
+
+def _update_skips_partial_page(kmin, kmax, k_grown, n_old, page):
+    # starts at the first page after the old rows, leaving a partial page stale
+    return _orig_update(kmin, kmax, k_grown, -(-n_old // page) * page, page) if n_old % page else \
+        _orig_update(kmin, kmax, k_grown, n_old, page)
+
+
+def _append_block_first(k_cache, v_cache, k_blk, v_blk):
+    # block placed before the prefix instead of after it
+    return _orig_append(k_blk, v_blk, k_cache, v_cache)
+
+
 PINS_ATTN = [
     lambda: TA.test_attend_matches_torch_sdpa_and_logsumexp(3, 7, 16, 0.25),
     lambda: TA.test_golden_attention_cases(),
@@ -94,6 +111,10 @@ PINS_GATE = [lambda: TF.test_golden_gate_cases()]
 PINS_SPARSE = [lambda: TS.test_page_estimate_bounds_every_score_in_page(),
                lambda: TS.test_select_pages_matches_full_lexsort(0),
                lambda: TS.test_select_ties_prefer_lower_page()]
+
+PINS_TRANSITION = [lambda: TT.test_incremental_page_bounds_equal_recomputed(17, 4),
+                   lambda: TT.test_appended_prefix_is_old_prefix_then_block(37, 5),
+                   lambda: TT.test_generation_first_steps_are_dense_over_all_earlier_blocks()]
 
 MUTANTS = [
     ("merge: denominator drops w_in", [(OA, "merge"), (OF, "merge"), (OS, "merge")], _merge_den_drop, PINS_ATTN),
@@ -106,6 +127,9 @@ MUTANTS = [
     ("gamma gate: >= instead of >", [(OF, "gamma_reuse")], _gamma_ge, PINS_GATE),
     ("page bound: min instead of max", [(OS, "page_estimates")], _est_min, PINS_SPARSE),
     ("top-k: ties to the higher page", [(OS, "select_pages")], _select_high_tie, PINS_SPARSE),
+    ("transition: partial page left stale", [(OT, "update_page_minmax")], _update_skips_partial_page,
+     PINS_TRANSITION),
+    ("transition: block before the prefix", [(OT, "append_block")], _append_block_first, PINS_TRANSITION),
 ]
 
 
@@ -124,5 +148,5 @@ def test_pins_catch_planted_mistake(monkeypatch, name, targets, mutant, pins):
 
 
 def test_pins_pass_on_unmutated_oracle():
-    for pin in PINS_ATTN + PINS_GATE + PINS_SPARSE:
+    for pin in PINS_ATTN + PINS_GATE + PINS_SPARSE + PINS_TRANSITION:
         pin()
