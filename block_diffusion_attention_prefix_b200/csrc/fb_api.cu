@@ -711,8 +711,11 @@ extern "C" int fb_sparse_step(const fb_shape* shape, const void* q, const void* 
   CUtensorMap tk, tv;
   FB_TRY(encode_kv_map(&tk, k_cache, d.D, d.N, d.row_stride, d.head_stride, d.b * d.hkv, kSparsePage));
   FB_TRY(encode_kv_map(&tv, v_cache, d.D, d.N, d.row_stride, d.head_stride, d.b * d.hkv, kSparsePage));
+  CUtensorMap tk4, tv4;
+  FB_TRY(encode_kv_map(&tk4, k_cache, d.D, d.N, d.row_stride, d.head_stride, d.b * d.hkv, 4 * kSparsePage));
+  FB_TRY(encode_kv_map(&tv4, v_cache, d.D, d.N, d.row_stride, d.head_stride, d.b * d.hkv, 4 * kSparsePage));
   FB_TRY(cuda_status(launch_sparse_select(a, (cudaStream_t)stream)));
-  return cuda_status(launch_sparse_pass(a, tk, tv, (cudaStream_t)stream));
+  return cuda_status(launch_sparse_pass(a, tk, tv, tk4, tv4, (cudaStream_t)stream));
 }
 
 // ---------------------------------------------------------------------------

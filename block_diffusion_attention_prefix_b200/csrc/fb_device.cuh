@@ -417,133 +417,6 @@ __device__ __forceinline__ void record_decisions(const GateParams& g, const Dims
   if (write_M && dec_M && tid == 0) dec_M[b] = M;
 }
 
-// Combine the `splits` partials of one (b, kv head, row tile) in fixed split
-// order (deterministic), in the CTA that arrived last.  Partials are
-// [splits][RT][D + 4] fp32 (A normalised in cols 0..D-1, natural-log L in col D),
-// contiguous in global memory.
-//   1. 1-D bulk TMA copies bring the partials into `buf` (chunks of as many splits
-//      as fit) -- plus, with the first chunk, `in_slot` into `s_in` when given;
-//      meanwhile every thread loads a share of the L values.
-//   2. Per row, the split weights w_s = e^{L_s - M} / sum_s e^{L_s - M} and the
-//      merged L = M + ln sum_s e^{L_s - M} (the FlashBlock merge equation over all
-//      splits) are computed once; s_L[r] gets the merged L.
-//   3. Each thread accumulates sum_s w_s A_s for its (row, 4-column) items in two
-//      chains split by the parity of the split index (order independent of the
-//      chunking); A[k] gets the result for item k = tid + k * NT.
-// Threads [0, NT), barrier `bar_id`; `buf` is `buf_bytes` of 128-byte aligned
-// shared memory; `mbar` an initialised mbarrier (count 1) whose next phase has
-// parity `*phase`.  Returns false if a bounded wait ran out (same on all threads).
-template <int D, int RT, int NT>
-__device__ bool combine_regs(const float* part, int splits, const float* in_slot, float* s_in, uint8_t* buf,
-                             int buf_bytes, uint64_t* mbar, uint32_t* phase, uint32_t* err, int tid, int bar_id,
-                             float4 (&A)[(RT * (D / 4) + NT - 1) / NT], float* s_L) {
-  constexpr int RS = D + 4;
-  constexpr int SPLIT_FLOATS = RT * RS;
-  constexpr int D4 = D / 4;
-  constexpr int IT = (RT * D4 + NT - 1) / NT;
-  const int w_bytes = ((splits + 2) * RT * 4 + 127) / 128 * 128;
-  float* sW = reinterpret_cast<float*>(buf);  // [splits][RT] weights, then [RT] 1/den
-  float* sInv = sW + (size_t)splits * RT;
-  float* chunk = reinterpret_cast<float*>(buf + w_bytes);
-  const int cs = (buf_bytes - w_bytes) / (SPLIT_FLOATS * 4);
-
-  auto issue = [&](int c0) {
-    const int nsp = min(cs, splits - c0);
-    const uint32_t bytes = (uint32_t)nsp * SPLIT_FLOATS * 4;
-    const bool with_in = in_slot != nullptr && c0 == 0;
-    fence_proxy_async_global();
-    mbar_arrive_expect_tx(mbar, bytes + (with_in ? (uint32_t)SPLIT_FLOATS * 4 : 0u));
-    bulk_load(chunk, part + (size_t)c0 * SPLIT_FLOATS, bytes, mbar);
-    if (with_in) bulk_load(s_in, in_slot, (uint32_t)SPLIT_FLOATS * 4, mbar);
-  };
-  if (tid == 0) issue(0);
-  for (int i = tid; i < splits * RT; i += NT) {
-    const int sp = i / RT, r = i - sp * RT;
-    sW[i] = __ldcg(part + (size_t)sp * SPLIT_FLOATS + (size_t)r * RS + D);
-  }
-  named_barrier_sync(bar_id, NT);
-  for (int r = tid; r < RT; r += NT) {  // per row: M = max_s L_s
-    float M = -CUDART_INF_F;
-    for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, sW[sp * RT + r]);
-    s_L[r] = M;
-  }
-  named_barrier_sync(bar_id, NT);
-  for (int i = tid; i < splits * RT; i += NT) {  // all (split, row) pairs: e = e^{L_s - M}
-    const float M = s_L[i % RT];
-    sW[i] = M == -CUDART_INF_F ? 0.f : expf(sW[i] - M);
-  }
-  named_barrier_sync(bar_id, NT);
-  for (int r = tid; r < RT; r += NT) {  // per row: den, merged L
-    float den = 0.f;
-    for (int sp = 0; sp < splits; ++sp) den += sW[sp * RT + r];
-    s_L[r] = den > 0.f ? s_L[r] + logf(den) : -CUDART_INF_F;
-    sInv[r] = den > 0.f ? 1.f / den : 0.f;
-  }
-  named_barrier_sync(bar_id, NT);
-
-  float4 acc1[IT];
-#pragma unroll
-  for (int k = 0; k < IT; ++k) A[k] = acc1[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  bool ok = true;
-  for (int c0 = 0; c0 < splits && ok; c0 += cs) {
-    const int nsp = min(cs, splits - c0);
-    if (c0 > 0 && tid == 0) issue(c0);
-    ok = mbar_wait_bounded(mbar, *phase, err, DEV_ERR_WAIT_COMBINE);
-    *phase ^= 1u;
-    if (ok) {
-#pragma unroll
-      for (int k = 0; k < IT; ++k) {
-        const int idx = tid + k * NT;
-        if (idx < RT * D4) {
-          const int r = idx / D4, d4 = idx - r * D4;
-          const float* pr = chunk + (size_t)r * RS + d4 * 4;
-          const float* wr = sW + (size_t)c0 * RT + r;
-          for (int sp = 0; sp < nsp; ++sp) {
-            const float w = wr[sp * RT];
-            const float4 x = *reinterpret_cast<const float4*>(pr + (size_t)sp * SPLIT_FLOATS);
-            float4& a = ((c0 + sp) & 1) ? acc1[k] : A[k];
-            a.x = fmaf(w, x.x, a.x);
-            a.y = fmaf(w, x.y, a.y);
-            a.z = fmaf(w, x.z, a.z);
-            a.w = fmaf(w, x.w, a.w);
-          }
-        }
-      }
-    }
-    ok = named_barrier_and(bar_id, NT, ok);  // also: the chunk buffer is free again
-  }
-#pragma unroll
-  for (int k = 0; k < IT; ++k) {
-    const int idx = tid + k * NT;
-    const float sc = idx < RT * D4 ? sInv[idx / D4] : 0.f;
-    A[k] = make_float4((A[k].x + acc1[k].x) * sc, (A[k].y + acc1[k].y) * sc, (A[k].z + acc1[k].z) * sc,
-                       (A[k].w + acc1[k].w) * sc);
-  }
-  named_barrier_sync(bar_id, NT);  // sInv is read above; `buf` may be reused after this
-  return ok;
-}
-
-// Per-row weights of the FlashBlock merge of two (A, L) parts: w1 = e^{L1-m}/den,
-// w2 = e^{L2-m}/den and L = m + ln den (both empty: 0, 0, -inf).
-__device__ __forceinline__ void merge_weights(float l1, float l2, float& w1, float& w2, float& l) {
-  const float m = fmaxf(l1, l2);
-  if (m == -CUDART_INF_F) {
-    w1 = w2 = 0.f;
-    l = -CUDART_INF_F;
-    return;
-  }
-  w1 = expf(l1 - m);
-  w2 = expf(l2 - m);
-  const float den = w1 + w2;
-  l = m + logf(den);
-  w1 /= den;
-  w2 /= den;
-}
-
-__device__ __forceinline__ float4 wsum4(float w1, float4 a, float w2, float4 b) {
-  return make_float4(w1 * a.x + w2 * b.x, w1 * a.y + w2 * b.y, w1 * a.z + w2 * b.z, w1 * a.w + w2 * b.w);
-}
-
 // Split-KV combine spread over the split CTAs of one (b, kv head, row tile)
 // (`unit`).  Called by the threads [0, NT) of every split CTA once its partial
 // ([RT][D + 4] fp32, A normalised, natural-log L) and its share of the in-block

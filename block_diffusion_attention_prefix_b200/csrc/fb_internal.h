@@ -128,7 +128,9 @@ struct SparseArgs {
 int sparse_supported(int D, int row_tile);
 cudaError_t launch_page_minmax(const SparseArgs& a, cudaStream_t s);
 cudaError_t launch_sparse_select(const SparseArgs& a, cudaStream_t s);
-cudaError_t launch_sparse_pass(const SparseArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s);
+// tk / tv: 16-row boxes (one page); tk4 / tv4: 64-row boxes (four consecutive pages).
+cudaError_t launch_sparse_pass(const SparseArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                               const CUtensorMap& tk4, const CUtensorMap& tv4, cudaStream_t s);
 
 SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int num_sms,
                      bool with_inblock = false, bool allow_tc = true);

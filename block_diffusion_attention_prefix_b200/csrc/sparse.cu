@@ -23,14 +23,17 @@
 //    order-preserving 64-bit key, tie ranks and compaction in page order ->
 //    sorted page list, row bitmap, union bitmap of the KV group (atomicOr).
 //  * sparse_pass_kernel: the TMA + mma.sync split pipeline of the dense pass
-//    with page-granular loads (16-key boxes).  Recompute step: every page, two
-//    online softmaxes per row (selected pages -> fresh part, other pages ->
-//    residual).  Reuse step: only the union pages of the KV group, selected part
-//    only (rows mask the union pages they did not select).  The finishing CTA
-//    combines the splits, writes the residual cache (recompute) and
-//    A_full = merge(merge(A_sel, A_res), A_in) with the in-block rows computed by
-//    the aux warps.
+//    with page-granular loads (four consecutive pages as one 64-key box, other
+//    pages as 16-key boxes).  Recompute step: every page, both online softmaxes
+//    per row from one score tile (selected pages -> fresh part, other pages ->
+//    residual; one exponential per score).  Reuse step: only the union pages of
+//    the KV group, selected part only (rows mask the union pages they did not
+//    select).  Cooperative launch: once all splits of a tile have arrived, each
+//    split CTA combines its own rows of both parts, writes the residual cache
+//    (recompute) and A_full = merge(merge(A_sel, A_res), A_in) with the in-block
+//    rows its aux warp computed.
 #include <cuda.h>
+#include <type_traits>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <math_constants.h>
@@ -45,6 +48,7 @@ namespace {
 using bf16 = __nv_bfloat16;
 constexpr int kPage = 16;
 constexpr int kTilePages = 4;  // 64 keys per pipeline tile
+constexpr int kBitsWords = 4096;  // shared words for the tile rows' selection bitmaps (16 KB)
 
 __device__ __forceinline__ bool sparse_recompute(const GateParams& g, int b, int B, int* s_red) {
   if (!g.enabled) return true;
@@ -350,16 +354,15 @@ struct SCfg {
                 "finisher space");
 };
 
-// Byte offset of (key in tile, d) for a tile of 4 pages, each page stored as D/64
-// boxes of [16 keys x 64 d] with the 128-byte swizzle (chunk c of row r at c ^ (r % 8)).
+// Byte offset of (key in tile, d) for a tile of 4 pages (64 keys) stored as D/64
+// boxes of [64 keys x 64 d] with the 128-byte swizzle (chunk c of row r at c ^ (r % 8)).
+// Page j of the tile is keys [16 j, 16 j + 16): a 16-row box at offset 2048 j of each
+// 64-column half has the same swizzle phase as rows of one 64-row box, so four
+// consecutive pages can arrive as one box per half and single pages as small boxes.
 __device__ __forceinline__ uint32_t pswz(int key, int d, int D) {
-  const int slot = key >> 4, kr = key & 15;
-  return (uint32_t)(slot * (kPage * D * 2) + (d >> 6) * (kPage * 128) + kr * 128 +
-                    ((((d & 63) >> 3) ^ (kr & 7)) << 4) + (d & 7) * 2);
-}
-
-__device__ __forceinline__ bool sel_bit(const uint32_t* rowbits, int page) {
-  return (__ldg(rowbits + (page >> 5)) >> (page & 31)) & 1u;
+  (void)D;
+  return (uint32_t)((d >> 6) * (kTilePages * kPage * 128) + key * 128 + ((((d & 63) >> 3) ^ (key & 7)) << 4) +
+                    (d & 7) * 2);
 }
 
 // Online-softmax state of one 16-row fragment set (two rows per thread).
@@ -432,6 +435,99 @@ __device__ __forceinline__ void softmax_pv(Acc<D>& A, float (&sc)[KW / 8][4], ui
   }
 }
 
+// Recompute steps: both online softmaxes -- the selected and the residual key sets
+// of each row -- from one score tile.  `sc` holds base-2 scores (-inf where the key
+// is past the end), `sel` says which set each score belongs to; one exponential per
+// score (against its own set's running max) and two P V products that share every
+// V fragment.
+template <int D, int KW>
+__device__ __forceinline__ void softmax_pv_dual(Acc<D>& As, Acc<D>& Ar, float (&sc)[KW / 8][4],
+                                                const bool (&sel)[KW / 8][4], uint32_t sV, int wn, int lane) {
+  float ms0 = As.m0, ms1 = As.m1, mr0 = Ar.m0, mr1 = Ar.m1;
+#pragma unroll
+  for (int n = 0; n < KW / 8; ++n) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float v = sc[n][j];
+      if (j < 2) {
+        if (sel[n][j]) ms0 = fmaxf(ms0, v); else mr0 = fmaxf(mr0, v);
+      } else {
+        if (sel[n][j]) ms1 = fmaxf(ms1, v); else mr1 = fmaxf(mr1, v);
+      }
+    }
+  }
+#pragma unroll
+  for (int x = 1; x <= 2; x <<= 1) {
+    ms0 = fmaxf(ms0, __shfl_xor_sync(0xffffffffu, ms0, x));
+    ms1 = fmaxf(ms1, __shfl_xor_sync(0xffffffffu, ms1, x));
+    mr0 = fmaxf(mr0, __shfl_xor_sync(0xffffffffu, mr0, x));
+    mr1 = fmaxf(mr1, __shfl_xor_sync(0xffffffffu, mr1, x));
+  }
+  const float bs0 = (ms0 == -CUDART_INF_F) ? 0.f : ms0, bs1 = (ms1 == -CUDART_INF_F) ? 0.f : ms1;
+  const float br0 = (mr0 == -CUDART_INF_F) ? 0.f : mr0, br1 = (mr1 == -CUDART_INF_F) ? 0.f : mr1;
+  const float as0 = ex2_approx(As.m0 - bs0), as1 = ex2_approx(As.m1 - bs1);
+  const float ar0 = ex2_approx(Ar.m0 - br0), ar1 = ex2_approx(Ar.m1 - br1);
+  float pss0 = 0.f, pss1 = 0.f, psr0 = 0.f, psr1 = 0.f;
+  float ps[KW / 8][4], pr[KW / 8][4];
+#pragma unroll
+  for (int n = 0; n < KW / 8; ++n) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bool s_ = sel[n][j];
+      const float base = j < 2 ? (s_ ? bs0 : br0) : (s_ ? bs1 : br1);
+      const float p = ex2_approx(sc[n][j] - base);
+      ps[n][j] = s_ ? p : 0.f;
+      pr[n][j] = s_ ? 0.f : p;
+    }
+    pss0 += ps[n][0] + ps[n][1];
+    pss1 += ps[n][2] + ps[n][3];
+    psr0 += pr[n][0] + pr[n][1];
+    psr1 += pr[n][2] + pr[n][3];
+  }
+  As.l0 = As.l0 * as0 + pss0;
+  As.l1 = As.l1 * as1 + pss1;
+  Ar.l0 = Ar.l0 * ar0 + psr0;
+  Ar.l1 = Ar.l1 * ar1 + psr1;
+  As.m0 = ms0;
+  As.m1 = ms1;
+  Ar.m0 = mr0;
+  Ar.m1 = mr1;
+#pragma unroll
+  for (int dn = 0; dn < D / 8; ++dn) {
+    As.o[dn][0] *= as0;
+    As.o[dn][1] *= as0;
+    As.o[dn][2] *= as1;
+    As.o[dn][3] *= as1;
+    Ar.o[dn][0] *= ar0;
+    Ar.o[dn][1] *= ar0;
+    Ar.o[dn][2] *= ar1;
+    Ar.o[dn][3] *= ar1;
+  }
+#pragma unroll
+  for (int k2 = 0; k2 < KW / 16; ++k2) {
+    uint32_t pa[4], pb[4];
+    pa[0] = pack_bf16x2(ps[2 * k2][0], ps[2 * k2][1]);
+    pa[1] = pack_bf16x2(ps[2 * k2][2], ps[2 * k2][3]);
+    pa[2] = pack_bf16x2(ps[2 * k2 + 1][0], ps[2 * k2 + 1][1]);
+    pa[3] = pack_bf16x2(ps[2 * k2 + 1][2], ps[2 * k2 + 1][3]);
+    pb[0] = pack_bf16x2(pr[2 * k2][0], pr[2 * k2][1]);
+    pb[1] = pack_bf16x2(pr[2 * k2][2], pr[2 * k2][3]);
+    pb[2] = pack_bf16x2(pr[2 * k2 + 1][0], pr[2 * k2 + 1][1]);
+    pb[3] = pack_bf16x2(pr[2 * k2 + 1][2], pr[2 * k2 + 1][3]);
+#pragma unroll
+    for (int dn = 0; dn < D / 8; dn += 2) {
+      const int key = wn * KW + k2 * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int dd = dn * 8 + (lane >> 4) * 8;
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(sV + pswz(key, dd, D), b0, b1, b2, b3);
+      mma_bf16_16816(As.o[dn], pa, b0, b1);
+      mma_bf16_16816(As.o[dn + 1], pa, b2, b3);
+      mma_bf16_16816(Ar.o[dn], pb, b0, b1);
+      mma_bf16_16816(Ar.o[dn + 1], pb, b2, b3);
+    }
+  }
+}
+
 // Merge the WARPS_N key slices of each row (scratch in smem) into this CTA's
 // partial [RT][D + 4] (A normalised, natural-log L) in global memory.
 template <int D, int WARPS_M, int WARPS_N>
@@ -492,9 +588,170 @@ __device__ __forceinline__ void stash(float* scr, int warp, int lane, const Acc<
 constexpr int kBarConsumers = 1;
 constexpr int kBarFinish = 2;
 
+// Split combine of the sparse pass, spread over the split CTAs of one (b, KV head,
+// row tile) `unit` (the launch is cooperative: all CTAs resident).  Called by the
+// threads [0, NT) of every split CTA once its partials (selected set; residual set
+// on recompute steps) and its in-block rows are in the workspace.  Each CTA waits
+// (bounded) for the other splits, pulls rows [r0, r1) of every split's partials and
+// its in-block rows into shared memory (one bulk copy per split and set), and then:
+//   A_sel, L_sel (and A_res, L_res on recompute) over all splits -- the FlashBlock
+//   merge equation with the split weights e_s = e^{L_s - M}, a fixed warp-tree sum;
+//   recompute: the residual cache is written; reuse: it is read;
+//   A_full = merge(merge(A_sel, A_res), A_in).
+template <int D, int NT>
+__device__ void sparse_coop_rows(const SparseArgs& args, size_t unit, int RT, int r0, int r1, size_t grow0,
+                                 bool recompute, uint8_t* sbuf, int sbuf_bytes, uint64_t* mbar, int tid,
+                                 int bar_id) {
+  constexpr int RS = D + 4;
+  constexpr int D4 = D / 4;
+  constexpr int NW = NT / 32;
+  const int splits = args.plan.splits;
+  const int n = r1 - r0 > 0 ? r1 - r0 : 0;
+  const int nsets = recompute ? 2 : 1;
+  const float* part[2] = {args.part_sel + unit * splits * RT * RS, args.part_res + unit * splits * RT * RS};
+  const float* pin = args.inblock + unit * RT * RS;
+  const size_t nd = (size_t)splits * n * RS;  // floats of one set's staged rows
+  float* sA = reinterpret_cast<float*>(sbuf);  // [nsets][splits][n][RS]
+  float* sIn = sA + nsets * nd;                 // [n][RS]
+  float* sE = sIn + (size_t)n * RS;             // [nsets][n][splits]
+  float* sL = sE + (size_t)nsets * n * splits;  // [2][n] combined L per set
+  float* sInv = sL + 2 * n;                     // [2][n]
+  float* sW = sInv + 2 * n;                     // [n][6]: merge weights pre (3), full (3)
+  const bool staged = (nsets * nd + (size_t)n * RS + (size_t)nsets * n * splits + 10 * (size_t)n) * 4 <=
+                      (size_t)sbuf_bytes;
+  unsigned int* arrive = args.counters + unit;
+  unsigned int* depart = args.counters + (size_t)args.d.b * args.d.hkv * args.plan.n_row_tiles + unit;
+  fence_proxy_async_smem();
+  named_barrier_sync(bar_id, NT);  // this CTA's partials and in-block rows are written
+  bool ok = true;
+  unsigned int dep = 0;
+  if (tid == 0) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(arrive) : "memory");
+    ok = wait_count_bounded(arrive, (unsigned)splits, args.err, DEV_ERR_WAIT_PEERS);
+    dep = atomicAdd(depart, 1u);  // result checked at the end
+    if (ok && staged && n > 0) {
+      fence_proxy_async_global();
+      const uint32_t row_bytes = (uint32_t)n * RS * 4;
+      mbar_arrive_expect_tx(mbar, row_bytes * (uint32_t)(nsets * splits + 1));
+      for (int st = 0; st < nsets; ++st)
+        for (int sp = 0; sp < splits; ++sp)
+          bulk_load(sA + st * nd + (size_t)sp * n * RS, part[st] + ((size_t)sp * RT + r0) * RS, row_bytes, mbar);
+      bulk_load(sIn, pin + (size_t)r0 * RS, row_bytes, mbar);
+    }
+  }
+  ok = named_barrier_and(bar_id, NT, ok);
+  if (ok && n > 0) {
+    if (staged) ok = mbar_wait_bounded(mbar, 0u, args.err, DEV_ERR_WAIT_COMBINE);
+    ok = named_barrier_and(bar_id, NT, ok);
+  }
+  if (ok && n > 0) {
+    auto ld1 = [&](int st, int sp, int rr) -> float {
+      return staged ? sA[st * nd + ((size_t)sp * n + rr) * RS + D]
+                    : __ldcg(part[st] + ((size_t)sp * RT + r0 + rr) * RS + D);
+    };
+    auto ld4 = [&](int st, int sp, int rr, int d4) -> float4 {
+      return staged ? reinterpret_cast<const float4*>(sA + st * nd + ((size_t)sp * n + rr) * RS)[d4]
+                    : __ldcg(reinterpret_cast<const float4*>(part[st] + ((size_t)sp * RT + r0 + rr) * RS) + d4);
+    };
+    auto in1 = [&](int rr) -> float {
+      return staged ? sIn[(size_t)rr * RS + D] : __ldcg(pin + (size_t)(r0 + rr) * RS + D);
+    };
+    auto in4 = [&](int rr, int d4) -> float4 {
+      return staged ? reinterpret_cast<const float4*>(sIn + (size_t)rr * RS)[d4]
+                    : __ldcg(reinterpret_cast<const float4*>(pin + (size_t)(r0 + rr) * RS) + d4);
+    };
+    const int warp = tid >> 5, lane = tid & 31;
+    // split weights, one warp per (set, row)
+    for (int pr = warp; pr < nsets * n; pr += NW) {
+      const int st = pr / n, rr = pr - st * n;
+      float M = -CUDART_INF_F;
+      for (int sp = lane; sp < splits; sp += 32) M = fmaxf(M, ld1(st, sp, rr));
+      M = warp_max(M);
+      float den = 0.f;
+      for (int sp = lane; sp < splits; sp += 32) {
+        const float e = M == -CUDART_INF_F ? 0.f : expf(ld1(st, sp, rr) - M);
+        sE[((size_t)st * n + rr) * splits + sp] = e;
+        den += e;
+      }
+      den = warp_sum(den);
+      if (lane == 0) {
+        sL[st * n + rr] = den > 0.f ? M + logf(den) : -CUDART_INF_F;
+        sInv[st * n + rr] = den > 0.f ? 1.f / den : 0.f;
+      }
+    }
+    named_barrier_sync(bar_id, NT);
+    // per row: pre = merge(sel, res), full = merge(pre, in)
+    for (int rr = tid; rr < n; rr += NT) {
+      const size_t grow = grow0 + r0 + rr;
+      const float ls = sL[rr];
+      const float lr = recompute ? sL[n + rr] : __ldcg(args.l_res + grow);
+      const MergeRow wp = merge_row(ls, lr);
+      const MergeRow wf = merge_row(wp.l, in1(rr));
+      float* w = sW + (size_t)rr * 6;
+      w[0] = wp.w1;
+      w[1] = wp.w2;
+      w[2] = wp.rden;
+      w[3] = wf.w1;
+      w[4] = wf.w2;
+      w[5] = wf.rden;
+      if (recompute) args.l_res[grow] = lr;
+      if (args.l_sel) args.l_sel[grow] = ls;
+      if (args.step.l_full) args.step.l_full[grow] = wf.l;
+    }
+    named_barrier_sync(bar_id, NT);
+    for (int idx = tid; idx < n * D4; idx += NT) {
+      const int rr = idx / D4, d4 = idx - rr * D4;
+      const size_t off = (grow0 + r0 + rr) * D + (size_t)d4 * 4;
+      float4 acc[2];
+#pragma unroll
+      for (int st = 0; st < 2; ++st) {
+        acc[st] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (st >= nsets) continue;
+        const float* er = sE + ((size_t)st * n + rr) * splits;
+        for (int sp = 0; sp < splits; ++sp) {
+          const float e = er[sp];
+          const float4 x = ld4(st, sp, rr, d4);
+          acc[st].x = fmaf(e, x.x, acc[st].x);
+          acc[st].y = fmaf(e, x.y, acc[st].y);
+          acc[st].z = fmaf(e, x.z, acc[st].z);
+          acc[st].w = fmaf(e, x.w, acc[st].w);
+        }
+        const float sc = sInv[st * n + rr];
+        acc[st] = make_float4(acc[st].x * sc, acc[st].y * sc, acc[st].z * sc, acc[st].w * sc);
+      }
+      const float4 as = acc[0];
+      const float4 ar = recompute ? acc[1] : __ldcg(reinterpret_cast<const float4*>(args.a_res + off));
+      if (recompute) *reinterpret_cast<float4*>(args.a_res + off) = ar;
+      if (args.a_sel) *reinterpret_cast<float4*>(args.a_sel + off) = as;
+      const float* w = sW + (size_t)rr * 6;
+      MergeRow wp, wf;
+      wp.w1 = w[0];
+      wp.w2 = w[1];
+      wp.rden = w[2];
+      wf.w1 = w[3];
+      wf.w2 = w[4];
+      wf.rden = w[5];
+      const float4 ai = in4(rr, d4);
+      const float4 pre = make_float4(merge_val(wp, as.x, ar.x), merge_val(wp, as.y, ar.y), merge_val(wp, as.z, ar.z),
+                                     merge_val(wp, as.w, ar.w));
+      store4(args.step.a_full, off,
+             make_float4(merge_val(wf, pre.x, ai.x), merge_val(wf, pre.y, ai.y), merge_val(wf, pre.z, ai.z),
+                         merge_val(wf, pre.w, ai.w)),
+             1);
+    }
+  }
+  if (tid == 0 && dep == (unsigned)splits - 1u) {  // every split has seen the full count
+    *arrive = 0u;
+    *depart = 0u;
+  }
+}
+
+
+
 template <int D, int WARPS_M, int WARPS_N, int STAGES>
 __global__ void __launch_bounds__(SCfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
     sparse_pass_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmK4, const __grid_constant__ CUtensorMap tmV4,
                        const SparseArgs args) {
   using C = SCfg<D, WARPS_M, WARPS_N, STAGES>;
   constexpr int NCW = C::kConsumerWarps;
@@ -507,9 +764,9 @@ __global__ void __launch_bounds__(SCfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1
   __shared__ __align__(8) uint64_t empty_bar[STAGES];
   __shared__ __align__(8) uint64_t comb_bar;
   __shared__ int s_pages[STAGES][kTilePages];
+  __shared__ uint32_t s_bits[kBitsWords];
   __shared__ int s_flags[RT];
   __shared__ int s_red[32];
-  __shared__ int s_last;
   __shared__ int s_M;
   __shared__ int s_recompute;
   __shared__ int s_union_total;
@@ -566,20 +823,47 @@ __global__ void __launch_bounds__(SCfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1
 
   if (warp == C::kProducerWarp) {
     // ---------------- producer: page loads into the ring ----------------
+    const uint32_t* ub = args.union_bits + (size_t)bg * args.words;
+    int wcur = 0, seen = 0;  // reuse: the word holding this split's first union page, pages before it
+    if (!recompute && ntiles > 0) {
+      // The whole warp locates the (t_begin * 4)-th union page: popcounts of 32 words
+      // at a time, an inclusive warp scan, and the first word whose running count
+      // passes the target.
+      const int target = t_begin * kTilePages;
+      int base = 0;
+      bool found = false;
+      for (int w0 = 0; w0 < args.words && !found; w0 += 32) {
+        const int c = (w0 + lane < args.words) ? __popc(__ldg(ub + w0 + lane)) : 0;
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int t = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += t;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, base + incl > target);
+        if (hit) {
+          const int L = __ffs(hit) - 1;
+          wcur = w0 + L;
+          seen = base + __shfl_sync(0xffffffffu, incl - c, L);
+          found = true;
+        } else {
+          base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+      }
+      if (!found) {
+        wcur = args.words;
+        seen = base;
+      }
+    }
     if (lane == 0 && ntiles > 0) {
       prefetch_tmap(&tmK);
       prefetch_tmap(&tmV);
-      const uint32_t* ub = args.union_bits + (size_t)bg * args.words;
+      prefetch_tmap(&tmK4);
+      prefetch_tmap(&tmV4);
       int cur = t_begin * kTilePages;  // index among the pages of the work list
-      int wcur = 0, wbits = 0, seen = 0;  // union enumeration cursor
+      int wbits = 0;                   // union enumeration cursor (word wcur)
       if (!recompute) {
-        // position the cursor on the cur-th union page
-        for (wcur = 0; wcur < args.words; ++wcur) {
-          const int c = __popc(ub[wcur]);
-          if (seen + c > cur) break;
-          seen += c;
-        }
-        wbits = wcur < args.words ? (int)ub[wcur] : 0;
+        wbits = wcur < args.words ? (int)__ldg(ub + wcur) : 0;
         for (int skip = cur - seen; skip > 0; --skip) wbits &= wbits - 1;
       }
       int issued = 0;
@@ -596,7 +880,7 @@ __global__ void __launch_bounds__(SCfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1
             if (recompute) {
               page = cur;
             } else {
-              while (wbits == 0 && wcur + 1 < args.words) wbits = (int)ub[++wcur];
+              while (wbits == 0 && wcur + 1 < args.words) wbits = (int)__ldg(ub + (++wcur));
               page = wcur * 32 + (__ffs(wbits) - 1);
               wbits &= wbits - 1;
             }
@@ -612,14 +896,26 @@ __global__ void __launch_bounds__(SCfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1
         (void)nvalid;
         mbar_arrive_expect_tx(&full_bar[s], (uint32_t)kTilePages * 2u * C::kPageBytes);
         uint8_t* st = smem + s * C::kStageBytes;
+        bool run = pg[0] >= 0;  // four consecutive pages: one 64-row box per half
 #pragma unroll
-        for (int j = 0; j < kTilePages; ++j) {
-          const int row = (pg[j] >= 0 ? pg[j] : args.P) * kPage;
+        for (int j = 1; j < kTilePages; ++j) run = run && pg[j] == pg[0] + j;
+        if (run) {
 #pragma unroll
           for (int h = 0; h < D / 64; ++h) {
-            tma_load_3d(st + j * C::kPageBytes + h * (kPage * 128), &tmK, &full_bar[s], h * 64, row, bg);
-            tma_load_3d(st + C::kTileBytes + j * C::kPageBytes + h * (kPage * 128), &tmV, &full_bar[s], h * 64, row,
-                        bg);
+            tma_load_3d(st + h * (kTilePages * kPage * 128), &tmK4, &full_bar[s], h * 64, pg[0] * kPage, bg);
+            tma_load_3d(st + C::kTileBytes + h * (kTilePages * kPage * 128), &tmV4, &full_bar[s], h * 64,
+                        pg[0] * kPage, bg);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < kTilePages; ++j) {
+            const int row = (pg[j] >= 0 ? pg[j] : args.P) * kPage;
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h) {
+              const int off = h * (kTilePages * kPage * 128) + j * (kPage * 128);
+              tma_load_3d(st + off, &tmK, &full_bar[s], h * 64, row, bg);
+              tma_load_3d(st + C::kTileBytes + off, &tmV, &full_bar[s], h * 64, row, bg);
+            }
           }
         }
         ++issued;
@@ -656,59 +952,79 @@ __global__ void __launch_bounds__(SCfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1
         qf[kk][3] = v1 ? *reinterpret_cast<const uint32_t*>(qb + (size_t)r1 * D + col + 8) : 0u;
       }
     }
-    const uint32_t* bits0 = args.sel_bits + (grow0 + min(r0, rows_valid - 1)) * (size_t)args.words;
-    const uint32_t* bits1 = args.sel_bits + (grow0 + min(r1, rows_valid - 1)) * (size_t)args.words;
+    // The tile rows' selection bitmaps, in shared memory when they fit.
+    const bool bits_smem = RT * args.words <= kBitsWords;
+    if (bits_smem) {
+      for (int i = tid; i < RT * args.words; i += NCW * 32) {
+        const int r = i / args.words, wd = i - r * args.words;
+        s_bits[i] = __ldg(args.sel_bits + (grow0 + min(r, rows_valid - 1)) * (size_t)args.words + wd);
+      }
+      named_barrier_sync(kBarConsumers, NCW * 32);
+    }
+    auto row_sel = [&](int r, int page) -> bool {
+      const int rr = min(r, rows_valid - 1);
+      const uint32_t w = bits_smem ? s_bits[rr * args.words + (page >> 5)]
+                                   : __ldg(args.sel_bits + (grow0 + rr) * (size_t)args.words + (page >> 5));
+      return (w >> (page & 31)) & 1u;
+    };
     Acc<D> As, Ar;
     As.init();
     Ar.init();
     const float sl2 = d.scale * 1.4426950408889634f;
-    bool ok = true;
-    for (int i = 0; i < ntiles && ok; ++i) {
-      const int s = i % STAGES;
-      if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(i / STAGES) & 1u, args.err, DEV_ERR_WAIT_FULL)) {
-        ok = false;
-        break;
-      }
-      const uint32_t sK = smem_u32(smem + s * C::kStageBytes);
-      const uint32_t sV = sK + C::kTileBytes;
-      float sc[KW / 8][4];
+    // The tile loop, compiled twice: reuse steps keep only the selected set's state
+    // live, recompute steps both sets.
+    auto tile_loop = [&](auto dual_tag) {
+      constexpr bool kDual = decltype(dual_tag)::value;
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(i / STAGES) & 1u, args.err, DEV_ERR_WAIT_FULL)) break;
+        const uint32_t sK = smem_u32(smem + s * C::kStageBytes);
+        const uint32_t sV = sK + C::kTileBytes;
+        float sc[KW / 8][4];
 #pragma unroll
-      for (int n = 0; n < KW / 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+        for (int n = 0; n < KW / 8; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D / 16; ++kk) {
 #pragma unroll
-        for (int n = 0; n < KW / 8; n += 2) {
-          const int key = wn * KW + n * 8 + (lane & 7) + ((lane >> 4) << 3);
-          const int dd = kk * 16 + ((lane >> 3) & 1) * 8;
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(sK + pswz(key, dd, D), b0, b1, b2, b3);
-          mma_bf16_16816(sc[n], qf[kk], b0, b1);
-          mma_bf16_16816(sc[n + 1], qf[kk], b2, b3);
+          for (int n = 0; n < KW / 8; n += 2) {
+            const int key = wn * KW + n * 8 + (lane & 7) + ((lane >> 4) << 3);
+            const int dd = kk * 16 + ((lane >> 3) & 1) * 8;
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(sK + pswz(key, dd, D), b0, b1, b2, b3);
+            mma_bf16_16816(sc[n], qf[kk], b0, b1);
+            mma_bf16_16816(sc[n + 1], qf[kk], b2, b3);
+          }
         }
-      }
-      // Route each score to the selected or the residual set of its row.
-      float ss[KW / 8][4], sr[KW / 8][4];
+        // Route each score to the selected or the residual set of its row.
+        bool sm[KW / 8][4];
 #pragma unroll
-      for (int n = 0; n < KW / 8; ++n) {
-        const int colb = wn * KW + n * 8;
-        const int page = s_pages[s][colb >> 4];
-        const bool sel0 = page >= 0 && sel_bit(bits0, page);
-        const bool sel1 = page >= 0 && sel_bit(bits1, page);
+        for (int n = 0; n < KW / 8; ++n) {
+          const int colb = wn * KW + n * 8;
+          const int page = s_pages[s][colb >> 4];
+          const bool sel0 = page >= 0 && row_sel(r0, page);
+          const bool sel1 = page >= 0 && row_sel(r1, page);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const long long key = (long long)page * kPage + (colb & 15) + 2 * c + (j & 1);
-          const bool valid = page >= 0 && key < d.N;
-          const bool sel = j < 2 ? sel0 : sel1;
-          const float v = sc[n][j] * sl2;
-          ss[n][j] = (valid && sel) ? v : -CUDART_INF_F;
-          sr[n][j] = (valid && !sel) ? v : -CUDART_INF_F;
+          for (int j = 0; j < 4; ++j) {
+            const long long key = (long long)page * kPage + (colb & 15) + 2 * c + (j & 1);
+            const bool valid = page >= 0 && key < d.N;
+            const bool sel = j < 2 ? sel0 : sel1;
+            sm[n][j] = sel;
+            // reuse steps: the selected set only; recompute: every valid key in one of the two
+            sc[n][j] = (valid && (sel || kDual)) ? sc[n][j] * sl2 : -CUDART_INF_F;
+          }
         }
+        if constexpr (kDual)
+          softmax_pv_dual<D, KW>(As, Ar, sc, sm, sV, wn, lane);
+        else
+          softmax_pv<D, KW>(As, sc, sV, wn, lane);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[s]);
       }
-      softmax_pv<D, KW>(As, ss, sV, wn, lane);
-      if (recompute) softmax_pv<D, KW>(Ar, sr, sV, wn, lane);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[s]);
-    }
+    };
+    if (recompute)
+      tile_loop(std::true_type{});
+    else
+      tile_loop(std::false_type{});
     As.l0 += __shfl_xor_sync(0xffffffffu, As.l0, 1);
     As.l0 += __shfl_xor_sync(0xffffffffu, As.l0, 2);
     As.l1 += __shfl_xor_sync(0xffffffffu, As.l1, 1);
@@ -728,79 +1044,27 @@ __global__ void __launch_bounds__(SCfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1
       write_partial<D, WARPS_M, WARPS_N>(scr_r, args.part_res + (unit * plan.splits + split) * RT * rs, tid);
   }
 
-  named_barrier_sync(kBarFinish, C::kFinishThreads);
-  if (tid == 0) {
-    __threadfence();
-    const unsigned prev = atomicAdd(args.counters + unit, 1u);
-    __threadfence();
-    s_last = (prev == (unsigned)plan.splits - 1u);
-  }
-  named_barrier_sync(kBarFinish, C::kFinishThreads);
-  if (!s_last) return;
-
-  // ---------------- finisher: consumers + aux ----------------
-  constexpr int NT = C::kFinishThreads;
-  constexpr int D4 = D / 4;
-  constexpr int IT = (RT * D4 + NT - 1) / NT;
+  // ---- consumers + aux: once every split has arrived, combine this CTA's rows ----
   const int ftid = warp < NCW ? tid : NCW * 32 + lane;
-  const int in_bytes = (RT * (D + 4) * 4 + 127) / 128 * 128;
-  float* s_in = reinterpret_cast<float*>(smem);
-  float* s_Ls = reinterpret_cast<float*>(smem + in_bytes);  // per row: L_sel, L_res, w_sel, w_res, w_pre, w_in
-  float* s_Lr = s_Ls + RT;
-  float* s_w = s_Lr + RT;
-  const int hdr = in_bytes + ((6 * RT * 4) + 127) / 128 * 128;
-  uint32_t phase = 0;
-  float4 Asel[IT], Ares[IT];
-  combine_regs<D, RT, NT>(args.part_sel + unit * plan.splits * RT * rs, plan.splits, args.inblock + unit * RT * rs,
-                          s_in, smem + hdr, C::kRingBytes - hdr, &comb_bar, &phase, args.err, ftid, kBarFinish, Asel,
-                          s_Ls);
-  if (recompute)
-    combine_regs<D, RT, NT>(args.part_res + unit * plan.splits * RT * rs, plan.splits, nullptr, nullptr,
-                            smem + hdr, C::kRingBytes - hdr, &comb_bar, &phase, args.err, ftid, kBarFinish, Ares,
-                            s_Lr);
-  // per-row weights: pre = merge(sel, res); full = merge(pre, in)
-  for (int r = ftid; r < rows_valid; r += NT) {
-    const size_t grow = grow0 + r;
-    const float lr = recompute ? s_Lr[r] : __ldcg(args.l_res + grow);
-    float ws, wr, lpre, wp, wi, lf;
-    merge_weights(s_Ls[r], lr, ws, wr, lpre);
-    merge_weights(lpre, s_in[(size_t)r * rs + D], wp, wi, lf);
-    s_w[4 * r + 0] = ws;
-    s_w[4 * r + 1] = wr;
-    s_w[4 * r + 2] = wp;
-    s_w[4 * r + 3] = wi;
-    if (recompute) args.l_res[grow] = s_Lr[r];
-    if (args.l_sel) args.l_sel[grow] = s_Ls[r];
-    if (args.step.l_full) args.step.l_full[grow] = lf;
+  {
+    int r0, r1;
+    split_rows(rows_valid, plan.splits, split, r0, r1);
+    sparse_coop_rows<D, C::kFinishThreads>(args, unit, RT, r0, r1, grow0, recompute, smem, C::kRingBytes, &comb_bar,
+                                           ftid, kBarFinish);
   }
-  named_barrier_sync(kBarFinish, NT);
-#pragma unroll
-  for (int k = 0; k < IT; ++k) {
-    const int idx = ftid + k * NT;
-    if (idx >= RT * D4) continue;
-    const int r = idx / D4, d4 = idx - r * D4;
-    if (r >= rows_valid) continue;
-    const size_t off = (grow0 + r) * D + (size_t)d4 * 4;
-    const float4 ar = recompute ? Ares[k] : __ldcg(reinterpret_cast<const float4*>(args.a_res + off));
-    if (recompute) *reinterpret_cast<float4*>(args.a_res + off) = ar;
-    if (args.a_sel) *reinterpret_cast<float4*>(args.a_sel + off) = Asel[k];
-    const float4 pre = wsum4(s_w[4 * r + 0], Asel[k], s_w[4 * r + 1], ar);
-    const float4 ai = *reinterpret_cast<const float4*>(s_in + (size_t)r * rs + d4 * 4);
-    store4(args.step.a_full, off, wsum4(s_w[4 * r + 2], pre, s_w[4 * r + 3], ai), 1);
-  }
-  if (args.gate.enabled) {
-    for (int r = ftid; r < rows_valid; r += NT) {
+  if (args.gate.enabled && split == 0) {
+    for (int r = ftid; r < rows_valid; r += C::kFinishThreads) {
       const int gr = row0 + r;
       if ((r == 0 || gr % d.B == 0) && args.step.dec_reuse)
         args.step.dec_reuse[(size_t)b * d.hq + kvh * d.G + gr / d.B] = recompute ? 0 : 1;
     }
     if (ftid == 0 && kvh == 0 && rt == 0 && args.step.dec_M) args.step.dec_M[b] = s_M;
   }
-  if (tid == 0) args.counters[unit] = 0u;
 }
 
 template <int D, int WM, int WN, int STAGES>
-cudaError_t launch_sparse_cfg(const SparseArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s) {
+cudaError_t launch_sparse_cfg(const SparseArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                              const CUtensorMap& tk4, const CUtensorMap& tv4, cudaStream_t s) {
   using C = SCfg<D, WM, WN, STAGES>;
   auto kern = sparse_pass_kernel<D, WM, WN, STAGES>;
   static bool attr_set[64] = {};
@@ -811,9 +1075,17 @@ cudaError_t launch_sparse_cfg(const SparseArgs& a, const CUtensorMap& tk, const 
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  dim3 grid(a.plan.splits, a.plan.n_row_tiles, a.d.b * a.d.hkv);
-  kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(tk, tv, a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.plan.splits, a.plan.n_row_tiles, a.d.b * a.d.hkv);
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // the split CTAs of a tile wait for one another
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.plan.splits > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, tk, tv, tk4, tv4, a);
 }
 
 }  // namespace
@@ -857,14 +1129,15 @@ cudaError_t launch_sparse_select(const SparseArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_sparse_pass(const SparseArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s) {
+cudaError_t launch_sparse_pass(const SparseArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                               const CUtensorMap& tk4, const CUtensorMap& tv4, cudaStream_t s) {
   const int D = a.d.D, rt = a.plan.row_tile;
   if (D == 128) {
-    if (rt == 16) return launch_sparse_cfg<128, 1, 4, 4>(a, tk, tv, s);
-    if (rt == 32) return launch_sparse_cfg<128, 2, 2, 4>(a, tk, tv, s);
+    if (rt == 16) return launch_sparse_cfg<128, 1, 4, 6>(a, tk, tv, tk4, tv4, s);
+    if (rt == 32) return launch_sparse_cfg<128, 2, 2, 6>(a, tk, tv, tk4, tv4, s);
   } else if (D == 64) {
-    if (rt == 16) return launch_sparse_cfg<64, 1, 4, 6>(a, tk, tv, s);
-    if (rt == 32) return launch_sparse_cfg<64, 2, 2, 6>(a, tk, tv, s);
+    if (rt == 16) return launch_sparse_cfg<64, 1, 4, 6>(a, tk, tv, tk4, tv4, s);
+    if (rt == 32) return launch_sparse_cfg<64, 2, 2, 6>(a, tk, tv, tk4, tv4, s);
   }
   return cudaErrorInvalidValue;
 }
