@@ -102,57 +102,91 @@ constexpr int kEstRowLanes = 2; // threads per page, each taking every other chu
 constexpr int kEstRows = 8;     // rows per chunk
 constexpr int kEstThreads = kEstPages * kEstRowLanes;
 
+// Page estimates of pages [p_lo, p_hi) of KV group bg for all R rows of the group,
+// by threads [0, NT); the group's q rows are in `sq` as float64 ([R rounded up to
+// 16][D]).  Two threads per page, 8 rows each per chunk; per row a float64 DFMA
+// chain in ascending d (each product exact), so the estimate is bit-identical to
+// the ordered sum.  The bounds of the next 8 channels are loaded while the current
+// 8 are consumed.
+template <int D, int NT>
+__device__ void estimate_pages(const SparseArgs& a, int bg, int p_lo, int p_hi, const double* sq, int tid) {
+  const Dims& d = a.d;
+  const int R = d.R;
+  const int b = bg / d.hkv, kvh = bg - b * d.hkv;
+  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B;
+  const int npg = p_hi - p_lo;
+  for (int it = tid; it < npg * kEstRowLanes; it += NT) {
+    const int p = p_lo + it % npg, rlane = it / npg;
+    const bf16* mn = a.kmin + (size_t)bg * D * a.Pcap + p;
+    const bf16* mx = a.kmax + (size_t)bg * D * a.Pcap + p;
+    for (int r0 = rlane * kEstRows; r0 < R; r0 += kEstRows * kEstRowLanes) {
+      double acc[kEstRows];
+#pragma unroll
+      for (int j = 0; j < kEstRows; ++j) acc[j] = 0.0;
+      // Two register buffers (A, B) of 8 channels' bounds, ping-pong: the loads of
+      // the next 8 channels are in flight while the current 8 are consumed.
+      float an[8], ax[8], bn[8], bx[8];
+      auto load8 = [&](float (&n8)[8], float (&x8)[8], int c0) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          n8[t] = __bfloat162float(__ldg(mn + (size_t)(c0 + t) * a.Pcap));
+          x8[t] = __bfloat162float(__ldg(mx + (size_t)(c0 + t) * a.Pcap));
+        }
+      };
+      auto use8 = [&](const float (&n8)[8], const float (&x8)[8], int c0) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+          const double kmn = (double)n8[t], kmx = (double)x8[t];
+          const double* qc = sq + (size_t)r0 * D + c0 + t;
+#pragma unroll
+          for (int j = 0; j < kEstRows; ++j) {
+            const double qv = qc[(size_t)j * D];
+            acc[j] = fma(qv, qv >= 0.0 ? kmx : kmn, acc[j]);  // exact product, one rounding
+          }
+        }
+      };
+      static_assert(D % 16 == 0, "channels in pairs of 8");
+      load8(an, ax, 0);
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 16) {
+        load8(bn, bx, c0 + 8);
+        use8(an, ax, c0);
+        if (c0 + 16 < D) load8(an, ax, c0 + 16);
+        use8(bn, bx, c0 + 8);
+      }
+#pragma unroll
+      for (int j = 0; j < kEstRows; ++j)
+        if (r0 + j < R) a.est[(grow0 + r0 + j) * (size_t)a.P + p] = acc[j];
+    }
+  }
+}
+
+// The q rows of KV group bg as float64 in shared memory (rows past R are zero).
+template <int D, int NT>
+__device__ void load_group_q(const SparseArgs& a, int bg, double* sq, int tid) {
+  const Dims& d = a.d;
+  const int R = d.R, Rp = (R + 15) / 16 * 16;
+  const int b = bg / d.hkv, kvh = bg - b * d.hkv;
+  const bf16* qg = static_cast<const bf16*>(a.q) + (size_t)(b * d.hq + kvh * d.G) * d.B * D;
+  for (int i = tid; i < Rp * D; i += NT) sq[i] = i < R * D ? (double)__bfloat162float(qg[i]) : 0.0;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kEstThreads) page_estimate_kernel(const SparseArgs a) {
   extern __shared__ double sq[];  // [R rounded up to 16][D] float64 copies of the group's q rows
   __shared__ int s_red[32];
   const Dims& d = a.d;
-  const int bg = blockIdx.y, b = bg / d.hkv, kvh = bg - b * d.hkv;
+  const int bg = blockIdx.y, b = bg / d.hkv;
   if (!sparse_recompute(a.gate, b, d.B, s_red)) return;
-  const int R = d.R, Rp = (R + 15) / 16 * 16;
-  const int p0 = blockIdx.x * kEstPages, p = p0 + (threadIdx.x % kEstPages);
-  const int rlane = threadIdx.x / kEstPages;
-  // The union of the group is rebuilt by topk_kernel: clear this chunk's words.
+  const int p0 = blockIdx.x * kEstPages;
+  // The union of the group is rebuilt by the top-k: clear this chunk's words.
   if (threadIdx.x < kEstPages / 32) {
     const int w = p0 / 32 + threadIdx.x;
     if (w < a.words) a.union_bits[(size_t)bg * a.words + w] = 0u;
   }
-  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B;
-  const bf16* qg = static_cast<const bf16*>(a.q) + grow0 * D;
-  for (int i = threadIdx.x; i < Rp * D; i += kEstThreads)
-    sq[i] = i < R * D ? (double)__bfloat162float(qg[i]) : 0.0;
+  load_group_q<D, kEstThreads>(a, bg, sq, threadIdx.x);
   __syncthreads();
-  if (p >= a.P) return;
-  const bf16* mn = a.kmin + (size_t)bg * D * a.Pcap + p;
-  const bf16* mx = a.kmax + (size_t)bg * D * a.Pcap + p;
-  for (int r0 = rlane * kEstRows; r0 < R; r0 += kEstRows * kEstRowLanes) {
-    double acc[kEstRows];
-#pragma unroll
-    for (int j = 0; j < kEstRows; ++j) acc[j] = 0.0;
-    for (int d0 = 0; d0 < D; d0 += 8) {
-      // Loads of 8 channels' bounds first (memory-level parallelism), then the
-      // DFMA chains in ascending d.
-      float kn[8], kx[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        kn[t] = __bfloat162float(__ldg(mn + (size_t)(d0 + t) * a.Pcap));
-        kx[t] = __bfloat162float(__ldg(mx + (size_t)(d0 + t) * a.Pcap));
-      }
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        const double kmn = (double)kn[t], kmx = (double)kx[t];
-        const double* qc = sq + (size_t)r0 * D + d0 + t;
-#pragma unroll
-        for (int j = 0; j < kEstRows; ++j) {
-          const double qv = qc[(size_t)j * D];
-          acc[j] = fma(qv, qv >= 0.0 ? kmx : kmn, acc[j]);  // exact product, one rounding
-        }
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kEstRows; ++j)
-      if (r0 + j < R) a.est[(grow0 + r0 + j) * (size_t)a.P + p] = acc[j];
-  }
+  estimate_pages<D, kEstThreads>(a, bg, p0, min(a.P, p0 + kEstPages), sq, threadIdx.x);
 }
 
 // ------------------------------------------------------------------ top-k pages
