@@ -404,6 +404,28 @@ def device_arm(args, rank, world):
     torch.cuda.synchronize()
     trans_us = statistics.median(a.elapsed_time(b) for a, b in trans) * 1e3
 
+    # Per-head similarity estimate (gamma workloads): fb_head_similarity over the
+    # block's queries and a reference block, as the estimated gate would run it.
+    sim_us = sim_gbs = None
+    if w.gamma is not None:
+        qa = torch.randn((w.batch, w.h_q, w.block, w.head_dim), device=dev).to(w.torch_dtype)
+        qb = torch.randn_like(qa)
+        sim_out = torch.zeros((w.batch, w.h_q), device=dev)
+        ssh = fb.make_shape(w.batch, w.h_q, w.h_kv, w.head_dim, w.block, w.n_prefix, w.dtype)
+        nb = fb.fb_similarity_workspace_bytes(ssh)
+        sws = torch.zeros(((nb + 15) // 16 * 16,), device=dev, dtype=torch.uint8)
+        ev = []
+        for i in range(20):
+            flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fb.fb_head_similarity(ssh, qa, qb, sim_out, sws)
+            e1.record()
+            ev.append((e0, e1))
+        torch.cuda.synchronize()
+        sim_us = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+        sim_gbs = 2 * qa.numel() * qa.element_size() / (sim_us * 1e-6) / 1e9
+
     e2e = e2e_arm(fb, dw, K, Wm) if (args.e2e and dw.sparse_layer is None) else None
     res = dict(
         metric=METRIC, value=value, unit="steps/s", n_gpus=world, steps=K, warmup=Wm,
@@ -435,6 +457,7 @@ def device_arm(args, rank, world):
                        reuse_step_alg_bytes=alg_reuse,
                        launch_floor_us=floor_us,
                        block_transition_us=trans_us,
+                       sim_estimator_us=sim_us, sim_estimator_gbs=sim_gbs,
                        dense_recompute_step_us=(statistics.mean(dense_ms) * 1e3) if dense_ms else None,
                        dense_steps_per_s=(1e3 / statistics.mean(dense_ms)) if dense_ms else None,
                        wall_s=wall),

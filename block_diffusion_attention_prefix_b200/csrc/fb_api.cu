@@ -629,6 +629,35 @@ extern "C" int fb_page_minmax(const fb_shape* shape, const void* k_cache, int pa
   return cuda_status(launch_page_minmax(a, (cudaStream_t)stream));
 }
 
+extern "C" size_t fb_similarity_workspace_bytes(const fb_shape* shape) {
+  Dims d;
+  if (resolve(shape, &d) != FB_OK) return 0;
+  return similarity_bytes(d);
+}
+
+extern "C" int fb_head_similarity(const fb_shape* shape, const void* q, const void* q_ref, float* sim, void* ws,
+                                  size_t ws_bytes, fb_stream_t stream) {
+  Dims d;
+  FB_TRY(resolve(shape, &d));
+  FB_TRY(check_ptr(q));
+  FB_TRY(check_ptr(q_ref));
+  if (!sim) return FB_ERR_NULL;
+  if (!ws) return FB_ERR_WORKSPACE;
+  if (!aligned16(ws)) return FB_ERR_ALIGN;
+  if (ws_bytes < similarity_bytes(d)) return FB_ERR_WORKSPACE;
+  return cuda_status(launch_similarity(d, q, q_ref, sim, ws, (cudaStream_t)stream));
+}
+
+extern "C" int fb_refresh_reference(const fb_shape* shape, const void* q, void* q_ref, const uint8_t* dec_reuse,
+                                    fb_stream_t stream) {
+  Dims d;
+  FB_TRY(resolve(shape, &d));
+  FB_TRY(check_ptr(q));
+  FB_TRY(check_ptr(q_ref));
+  if (!dec_reuse) return FB_ERR_NULL;
+  return cuda_status(launch_refresh(d, q, q_ref, dec_reuse, (cudaStream_t)stream));
+}
+
 extern "C" int fb_append_block(const fb_shape* shape, void* k_cache, void* v_cache, const void* k_blk,
                                const void* v_blk, int page_size, void* kmin, void* kmax, fb_stream_t stream) {
   Dims d;

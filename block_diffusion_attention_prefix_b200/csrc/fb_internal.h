@@ -160,6 +160,11 @@ cudaError_t launch_gate_eval(const Dims& d, const GateParams& g, int32_t* dec_M,
                              cudaStream_t s);
 cudaError_t launch_merge(const Dims& d, const float* a1, const float* l1, const float* a2,
                          const float* l2, void* a_full, float* l_full, cudaStream_t s);
+// Per-head similarity estimate (similarity.cu): workspace bytes, sim = cosine of
+// Q and the reference queries; refresh of the reference for recomputed heads.
+size_t similarity_bytes(const Dims& d);
+cudaError_t launch_similarity(const Dims& d, const void* q, const void* q_ref, float* sim, void* ws, cudaStream_t s);
+cudaError_t launch_refresh(const Dims& d, const void* q, void* q_ref, const uint8_t* dec_reuse, cudaStream_t s);
 // Block transition: copy the block's K/V ([b, H_kv, B, D]) into cache rows [N, N + B).
 cudaError_t launch_append_block(const Dims& d, void* k_cache, void* v_cache, const void* k_blk, const void* v_blk,
                                 cudaStream_t s);

@@ -17,7 +17,8 @@ __all__ = [
     "FBError", "Shape", "Gate", "load", "lib_path", "make_shape", "make_gate", "FB_F32", "FB_BF16",
     "fb_version", "fb_status_string", "fb_device_error", "fb_workspace_bytes", "fb_workspace_init",
     "fb_gate_eval", "fb_prefix_attn", "fb_prefix_attn_noalloc", "fb_block_attn", "fb_merge", "fb_block_merge", "fb_step",
-    "fb_page_minmax", "fb_append_block", "fb_sparse_workspace_bytes", "fb_sparse_select", "fb_sparse_step", "Sparse",
+    "fb_page_minmax", "fb_append_block", "fb_similarity_workspace_bytes", "fb_head_similarity",
+    "fb_refresh_reference", "fb_sparse_workspace_bytes", "fb_sparse_select", "fb_sparse_step", "Sparse",
     "SparseResidualLayer", "CachedAttentionLayer", "EXPORTED",
 ]
 
@@ -82,6 +83,9 @@ EXPORTED = {
     "fb_prefix_attn_noalloc": (_i, [_PS, _vp, _vp, _vp, _PG, _vp, _vp, _vp]),
     "fb_page_minmax": (_i, [_PS, _vp, _i, _vp, _vp, _vp]),
     "fb_append_block": (_i, [_PS, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
+    "fb_similarity_workspace_bytes": (_sz, [_PS]),
+    "fb_head_similarity": (_i, [_PS, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "fb_refresh_reference": (_i, [_PS, _vp, _vp, _vp, _vp]),
     "fb_sparse_workspace_bytes": (_sz, [_PS, _i]),
     "fb_sparse_select": (_i, [_PS, _vp, _PG, _PSP, _vp, _sz, _vp]),
     "fb_sparse_step": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _PG, _PSP, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -227,6 +231,20 @@ def fb_append_block(shape, k_cache, v_cache, k_blk, v_blk, page_size=16, kmin=No
                                                      _stream()))
 
 
+def fb_similarity_workspace_bytes(shape) -> int:
+    return int(load().fb_similarity_workspace_bytes(ctypes.byref(shape)))
+
+
+def fb_head_similarity(shape, q, q_ref, sim, ws):
+    _check("fb_head_similarity", load().fb_head_similarity(ctypes.byref(shape), _ptr(q), _ptr(q_ref), _ptr(sim),
+                                                           _ptr(ws), ws.numel() * ws.element_size(), _stream()))
+
+
+def fb_refresh_reference(shape, q, q_ref, dec_reuse):
+    _check("fb_refresh_reference", load().fb_refresh_reference(ctypes.byref(shape), _ptr(q), _ptr(q_ref),
+                                                               _ptr(dec_reuse), _stream()))
+
+
 def fb_sparse_workspace_bytes(shape, page_size=16) -> int:
     return int(load().fb_sparse_workspace_bytes(ctypes.byref(shape), int(page_size)))
 
@@ -341,6 +359,21 @@ class CachedAttentionLayer:
         g = make_gate(mask, first_step, tau, head_sim, gamma)
         fb_step(self.shape, q, self.k_cache, self.v_cache, k_blk, v_blk, g, self.a_out, self.l_out,
                 self.a_full, self.l_full, self.dec_M, self.dec_reuse, self.ws)
+        return self.a_full
+
+    def step_estimated(self, q, k_blk, v_blk, mask, first_step, tau, gamma):
+        """A step whose per-head gamma gate uses the on-device similarity estimate:
+        sim = cosine(q, the queries each head's cache was computed with); afterwards
+        the recomputed heads' reference queries become q."""
+        if not hasattr(self, "q_ref"):
+            self.q_ref = torch.zeros_like(q)
+            self.sim = torch.zeros((self.shape.batch, self.shape.h_q), device=q.device, dtype=torch.float32)
+            n = fb_similarity_workspace_bytes(self.shape)
+            self.sim_ws = torch.zeros(((n + 15) // 16 * 16,), device=q.device, dtype=torch.uint8)
+        if not first_step:
+            fb_head_similarity(self.shape, q, self.q_ref, self.sim, self.sim_ws)
+        self.step(q, k_blk, v_blk, mask, first_step, tau, self.sim, gamma)
+        fb_refresh_reference(self.shape, q, self.q_ref, self.dec_reuse)
         return self.a_full
 
     def finish_block(self, k_blk, v_blk):

@@ -198,6 +198,28 @@ typedef struct fb_sparse {
 int fb_page_minmax(const fb_shape* shape, const void* k_cache, int page_size, void* kmin, void* kmax,
                    fb_stream_t stream);
 
+/* Per-head similarity estimate for the gamma gate.  FlashBlock technical summary
+ * (gist.science 2602.05305), "Adaptive reuse strategies": in the video setting only
+ * heads whose estimated cross-step similarity is above gamma reuse their cache; the
+ * pages give no estimator.  This one: sim[b, h] = cosine between the head's block
+ * queries q [b, H_q, B, D] and the reference queries q_ref (same layout and dtype:
+ * the queries the head's cache was last computed with), i.e.
+ * <Q, R> / sqrt(<Q, Q> <R, R>) in float64 rounded to float32 (0 when a norm is 0).
+ * The sums run in one fixed order -- per row ascending d, rows in chunks of 256 as a
+ * pairwise tree, chunk totals in ascending order -- so the result, and the gate
+ * decision sim > gamma taken on it, is reproducible bit for bit.  sim [b, H_q]
+ * float32 device memory, then usable as fb_gate.head_sim.  Workspace: at least
+ * fb_similarity_workspace_bytes(shape) bytes, zeroed once (fb_workspace_init); its
+ * counters return to zero after each call.  Asynchronous on `stream`. */
+size_t fb_similarity_workspace_bytes(const fb_shape* shape);
+int fb_head_similarity(const fb_shape* shape, const void* q, const void* q_ref, float* sim, void* ws,
+                       size_t ws_bytes, fb_stream_t stream);
+
+/* After a step: heads that recomputed (dec_reuse[b, h] == 0, as written by fb_step)
+ * copy their block queries q into q_ref; heads that reused keep their reference. */
+int fb_refresh_reference(const fb_shape* shape, const void* q, void* q_ref, const uint8_t* dec_reuse,
+                         fb_stream_t stream);
+
 /* Block transition (after the last denoising step of a block): the block's tokens
  * join the prefix.  FlashBlock technical summary (gist.science 2602.05305),
  * "1. Problem definition": attention splits into the current block J_in and the

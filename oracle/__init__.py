@@ -23,6 +23,7 @@ Modules:
 * :mod:`oracle.flashblock` -- the tau / gamma gates and the stateful cached step.
 * :mod:`oracle.sparse`     -- page bounds, top-k page selection and the residual split.
 * :mod:`oracle.transition` -- the block transition: a finished block joins the prefix.
+* :mod:`oracle.similarity` -- the per-head similarity estimate behind the gamma gate.
 
 Pins: every function here is pinned by ``tests/test_oracle_*.py`` against
 library routines (torch float64 SDPA, logsumexp, full sorts), closed forms and

@@ -11,11 +11,13 @@ import oracle.attention as OA
 import oracle.flashblock as OF
 import oracle.sparse as OS
 import oracle.transition as OT
+import oracle.similarity as OSim
 
 from tests import test_oracle_attention as TA
 from tests import test_oracle_flashblock as TF
 from tests import test_oracle_sparse as TS
 from tests import test_oracle_transition as TT
+from tests import test_oracle_similarity as TSim
 
 _orig_attend = OA.attend
 _orig_merge = OA.merge
@@ -101,6 +103,30 @@ def _append_block_first(k_cache, v_cache, k_blk, v_blk):
     return _orig_append(k_blk, v_blk, k_cache, v_cache)
 
 
+_orig_ordered_sum = OSim._ordered_sum
+
+
+def _sum_sequential(row_terms):
+    # rows added one after another instead of the pairwise tree
+    total = 0.0
+    for x in np.asarray(row_terms, np.float64):
+        total = total + x
+    return float(total)
+
+
+def _sim_no_sqrt(q, q_ref):
+    q = np.asarray(q, np.float64)
+    r = np.asarray(q_ref, np.float64)
+    out = np.zeros(q.shape[:2], np.float32)
+    for bi in range(q.shape[0]):
+        for h in range(q.shape[1]):
+            a = _orig_ordered_sum(OSim._row_dots(q[bi, h], r[bi, h]))
+            n = _orig_ordered_sum(OSim._row_dots(q[bi, h], q[bi, h])) * _orig_ordered_sum(
+                OSim._row_dots(r[bi, h], r[bi, h]))
+            out[bi, h] = np.float32(a / n) if n > 0 else np.float32(0.0)
+    return out
+
+
 PINS_ATTN = [
     lambda: TA.test_attend_matches_torch_sdpa_and_logsumexp(3, 7, 16, 0.25),
     lambda: TA.test_golden_attention_cases(),
@@ -116,6 +142,10 @@ PINS_TRANSITION = [lambda: TT.test_incremental_page_bounds_equal_recomputed(17, 
                    lambda: TT.test_appended_prefix_is_old_prefix_then_block(37, 5),
                    lambda: TT.test_generation_first_steps_are_dense_over_all_earlier_blocks()]
 
+PINS_SIM = [lambda: TSim.test_matches_library_cosine(300),
+            lambda: TSim.test_closed_forms(),
+            lambda: TSim.test_pairwise_tree_order_inside_a_chunk()]
+
 MUTANTS = [
     ("merge: denominator drops w_in", [(OA, "merge"), (OF, "merge"), (OS, "merge")], _merge_den_drop, PINS_ATTN),
     ("merge: L drops ln(w1+w2)", [(OA, "merge"), (OF, "merge"), (OS, "merge")], _merge_L_drop, PINS_ATTN),
@@ -130,6 +160,8 @@ MUTANTS = [
     ("transition: partial page left stale", [(OT, "update_page_minmax")], _update_skips_partial_page,
      PINS_TRANSITION),
     ("transition: block before the prefix", [(OT, "append_block")], _append_block_first, PINS_TRANSITION),
+    ("similarity: rows summed in sequence", [(OSim, "_ordered_sum")], _sum_sequential, PINS_SIM),
+    ("similarity: norm without the square root", [(OSim, "head_similarity")], _sim_no_sqrt, PINS_SIM),
 ]
 
 
@@ -148,5 +180,5 @@ def test_pins_catch_planted_mistake(monkeypatch, name, targets, mutant, pins):
 
 
 def test_pins_pass_on_unmutated_oracle():
-    for pin in PINS_ATTN + PINS_GATE + PINS_SPARSE + PINS_TRANSITION:
+    for pin in PINS_ATTN + PINS_GATE + PINS_SPARSE + PINS_TRANSITION + PINS_SIM:
         pin()
