@@ -629,6 +629,41 @@ extern "C" int fb_page_minmax(const fb_shape* shape, const void* k_cache, int pa
   return cuda_status(launch_page_minmax(a, (cudaStream_t)stream));
 }
 
+extern "C" int fb_losa_step(const fb_shape* shape, const void* q, const void* q_prev, const void* k_cache,
+                            const void* v_cache, const void* k_blk, const void* v_blk, float delta,
+                            const fb_sparse* sp, void* a_full, float* l_full, float* mse, uint8_t* dec_active,
+                            void* ws, size_t ws_bytes, fb_stream_t stream) {
+  Dims d;
+  GateParams gp;
+  FB_TRY(sparse_check(shape, nullptr, sp, &d, &gp));
+  FB_TRY(check_ptr(q));
+  FB_TRY(check_ptr(q_prev));
+  FB_TRY(check_ptr(k_cache));
+  FB_TRY(check_ptr(v_cache));
+  FB_TRY(check_ptr(k_blk));
+  FB_TRY(check_ptr(v_blk));
+  if (!a_full || !dec_active) return FB_ERR_NULL;
+  if (!(delta == delta)) return FB_ERR_ARG;  // NaN threshold
+  SparseArgs a;
+  FB_TRY(sparse_args(d, gp, sp, q, ws, ws_bytes, &a));
+  a.active = dec_active;
+  a.step.enabled = 1;
+  a.step.k_blk = k_blk;
+  a.step.v_blk = v_blk;
+  a.step.a_full = a_full;
+  a.step.l_full = l_full;
+  a.step.dec_M = nullptr;
+  a.step.dec_reuse = nullptr;
+  CUtensorMap tk, tv, tk4, tv4;
+  FB_TRY(encode_kv_map(&tk, k_cache, d.D, d.N, d.row_stride, d.head_stride, d.b * d.hkv, kSparsePage));
+  FB_TRY(encode_kv_map(&tv, v_cache, d.D, d.N, d.row_stride, d.head_stride, d.b * d.hkv, kSparsePage));
+  FB_TRY(encode_kv_map(&tk4, k_cache, d.D, d.N, d.row_stride, d.head_stride, d.b * d.hkv, 4 * kSparsePage));
+  FB_TRY(encode_kv_map(&tv4, v_cache, d.D, d.N, d.row_stride, d.head_stride, d.b * d.hkv, 4 * kSparsePage));
+  FB_TRY(cuda_status(launch_token_mse(d, q, q_prev, delta, mse, dec_active, (cudaStream_t)stream)));
+  FB_TRY(cuda_status(launch_sparse_select(a, (cudaStream_t)stream)));
+  return cuda_status(launch_sparse_pass(a, tk, tv, tk4, tv4, (cudaStream_t)stream));
+}
+
 extern "C" size_t fb_similarity_workspace_bytes(const fb_shape* shape) {
   Dims d;
   if (resolve(shape, &d) != FB_OK) return 0;

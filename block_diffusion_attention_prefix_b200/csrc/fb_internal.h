@@ -114,6 +114,7 @@ struct SparseArgs {
   uint32_t* sel_bits;     // [b*H_q*B][words]
   uint32_t* union_bits;   // [b*H_kv][words]
   GateParams gate;        // tau only
+  const uint8_t* active;  // LoSA mode: token activity [b, B] (NULL otherwise)
   float* a_res;           // residual cache [b, H_q, B, D] / [b, H_q, B]
   float* l_res;
   float* a_sel;           // optional
@@ -127,6 +128,9 @@ struct SparseArgs {
 };
 int sparse_supported(int D, int row_tile);
 cudaError_t launch_page_minmax(const SparseArgs& a, cudaStream_t s);
+// LoSA: per-token locality score (float32 [b, B], nullable) and activity (score > delta).
+cudaError_t launch_token_mse(const Dims& d, const void* q, const void* q_prev, float delta, float* mse,
+                             uint8_t* active, cudaStream_t s);
 cudaError_t launch_sparse_select(const SparseArgs& a, cudaStream_t s);
 // tk / tv: 16-row boxes (one page); tk4 / tv4: 64-row boxes (four consecutive pages).
 cudaError_t launch_sparse_pass(const SparseArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,

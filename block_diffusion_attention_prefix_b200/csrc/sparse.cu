@@ -56,6 +56,36 @@ __device__ __forceinline__ bool sparse_recompute(const GateParams& g, int b, int
   return !tau_reuse(g, M);
 }
 
+// ------------------------------------------------------------------ LoSA locality score
+
+// One CTA per (token i, batch element b), one thread per query head: the head's
+// sum over d of (q - q_prev)^2 in float64, ascending d, each term a rounded product
+// then a rounded sum (no fused multiply-add: the products are not exact); thread 0
+// adds the heads in ascending order and divides by H_q * D.  Reading L1 of the LoSA
+// page ("2. Methodology": MSE between the queries of steps t and t - 1).
+__global__ void token_mse_kernel(const Dims d, const bf16* q, const bf16* qp, float delta, float* mse,
+                                 uint8_t* active) {
+  extern __shared__ double s_head[];
+  const int i = blockIdx.x, b = blockIdx.y;
+  for (int h = threadIdx.x; h < d.hq; h += blockDim.x) {
+    const size_t off = (((size_t)b * d.hq + h) * d.B + i) * d.D;
+    double acc = 0.0;
+    for (int k = 0; k < d.D; ++k) {
+      const double diff = __dsub_rn((double)__bfloat162float(q[off + k]), (double)__bfloat162float(qp[off + k]));
+      acc = __dadd_rn(acc, __dmul_rn(diff, diff));
+    }
+    s_head[h] = acc;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double tot = 0.0;
+    for (int h = 0; h < d.hq; ++h) tot = __dadd_rn(tot, s_head[h]);
+    const float m = (float)__ddiv_rn(tot, (double)d.hq * d.D);
+    if (mse) mse[(size_t)b * d.B + i] = m;
+    active[(size_t)b * d.B + i] = m > delta ? 1 : 0;
+  }
+}
+
 // ------------------------------------------------------------------ page bounds
 
 template <int D>
@@ -250,6 +280,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
   const int h = (row / d.B) % d.hq;
   const int kvh = h / d.G;
   if (!sparse_recompute(a.gate, b, d.B, s_tmp)) return;
+  if (a.active && !a.active[(size_t)b * d.B + row % d.B]) return;  // LoSA: stable tokens keep their cache
   const int P = a.P, tid = threadIdx.x;
   if (a.k_sel <= 0 || P <= 0) return;
   const int per = (P + kTopkThreads - 1) / kTopkThreads;
@@ -715,9 +746,24 @@ __device__ void sparse_coop_rows(const SparseArgs& args, size_t unit, int RT, in
     }
     named_barrier_sync(bar_id, NT);
     // per row: pre = merge(sel, res), full = merge(pre, in)
+    const bool losa = args.active != nullptr;
     for (int rr = tid; rr < n; rr += NT) {
       const size_t grow = grow0 + r0 + rr;
       const float ls = sL[rr];
+      if (losa) {  // active rows: the fresh sparse result is the new cache; stable rows read it
+        const bool act = args.active[(size_t)(grow / ((size_t)args.d.hq * args.d.B)) * args.d.B + grow % args.d.B] != 0;
+        const float lc = act ? ls : __ldcg(args.l_res + grow);
+        const MergeRow wf = merge_row(lc, in1(rr));
+        float* w = sW + (size_t)rr * 6;
+        w[0] = act ? 1.f : 0.f;
+        w[3] = wf.w1;
+        w[4] = wf.w2;
+        w[5] = wf.rden;
+        if (act) args.l_res[grow] = ls;
+        if (args.l_sel) args.l_sel[grow] = ls;
+        if (args.step.l_full) args.step.l_full[grow] = wf.l;
+        continue;
+      }
       const float lr = recompute ? sL[n + rr] : __ldcg(args.l_res + grow);
       const MergeRow wp = merge_row(ls, lr);
       const MergeRow wf = merge_row(wp.l, in1(rr));
@@ -754,6 +800,23 @@ __device__ void sparse_coop_rows(const SparseArgs& args, size_t unit, int RT, in
         acc[st] = make_float4(acc[st].x * sc, acc[st].y * sc, acc[st].z * sc, acc[st].w * sc);
       }
       const float4 as = acc[0];
+      if (losa) {
+        const float* w = sW + (size_t)rr * 6;
+        const bool act = w[0] != 0.f;
+        const float4 ac = act ? as : __ldcg(reinterpret_cast<const float4*>(args.a_res + off));
+        if (act) *reinterpret_cast<float4*>(args.a_res + off) = as;
+        if (args.a_sel) *reinterpret_cast<float4*>(args.a_sel + off) = as;
+        MergeRow wf;
+        wf.w1 = w[3];
+        wf.w2 = w[4];
+        wf.rden = w[5];
+        const float4 ai = in4(rr, d4);
+        store4(args.step.a_full, off,
+               make_float4(merge_val(wf, ac.x, ai.x), merge_val(wf, ac.y, ai.y), merge_val(wf, ac.z, ai.z),
+                           merge_val(wf, ac.w, ai.w)),
+               1);
+        continue;
+      }
       const float4 ar = recompute ? acc[1] : __ldcg(reinterpret_cast<const float4*>(args.a_res + off));
       if (recompute) *reinterpret_cast<float4*>(args.a_res + off) = ar;
       if (args.a_sel) *reinterpret_cast<float4*>(args.a_sel + off) = as;
@@ -824,6 +887,7 @@ __global__ void __launch_bounds__(SCfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1
       M = block_updated_count(args.gate.mask + (size_t)b * d.B, d.B, s_red);
       rec = !tau_reuse(args.gate, M);
     }
+    if (args.active) rec = false;  // LoSA: stream the active rows' union pages, no residual
     if (tid == 0) {
       s_M = M;
       s_recompute = rec ? 1 : 0;
@@ -973,6 +1037,13 @@ __global__ void __launch_bounds__(SCfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1
     const int wm = warp / WARPS_N, wn = warp - (warp / WARPS_N) * WARPS_N;
     const int c = lane & 3;
     const int r0 = wm * 16 + (lane >> 2), r1 = r0 + 8;
+    // LoSA: rows of stable tokens take no key (their scores are all masked)
+    auto row_active = [&](int r) -> bool {
+      if (!args.active) return true;
+      const size_t grow = grow0 + min(r, rows_valid - 1);
+      return args.active[(size_t)b * d.B + grow % d.B] != 0;
+    };
+    const bool act0 = row_active(r0), act1 = row_active(r1);
     uint32_t qf[D / 16][4];
     {
       const bf16* qb = q + grow0 * D;
@@ -1035,8 +1106,8 @@ __global__ void __launch_bounds__(SCfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1
         for (int n = 0; n < KW / 8; ++n) {
           const int colb = wn * KW + n * 8;
           const int page = s_pages[s][colb >> 4];
-          const bool sel0 = page >= 0 && row_sel(r0, page);
-          const bool sel1 = page >= 0 && row_sel(r1, page);
+          const bool sel0 = page >= 0 && act0 && row_sel(r0, page);
+          const bool sel1 = page >= 0 && act1 && row_sel(r1, page);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const long long key = (long long)page * kPage + (colb & 15) + 2 * c + (j & 1);
@@ -1086,7 +1157,7 @@ __global__ void __launch_bounds__(SCfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1
     sparse_coop_rows<D, C::kFinishThreads>(args, unit, RT, r0, r1, grow0, recompute, smem, C::kRingBytes, &comb_bar,
                                            ftid, kBarFinish);
   }
-  if (args.gate.enabled && split == 0) {
+  if (args.gate.enabled && !args.active && split == 0) {
     for (int r = ftid; r < rows_valid; r += C::kFinishThreads) {
       const int gr = row0 + r;
       if ((r == 0 || gr % d.B == 0) && args.step.dec_reuse)
@@ -1125,6 +1196,14 @@ cudaError_t launch_sparse_cfg(const SparseArgs& a, const CUtensorMap& tk, const 
 }  // namespace
 
 int sparse_supported(int D, int row_tile) { return (D == 64 || D == 128) && (row_tile == 16 || row_tile == 32); }
+
+cudaError_t launch_token_mse(const Dims& d, const void* q, const void* q_prev, float delta, float* mse,
+                             uint8_t* active, cudaStream_t s) {
+  const int threads = d.hq < 32 ? 32 : (d.hq > 256 ? 256 : (d.hq + 31) / 32 * 32);
+  token_mse_kernel<<<dim3(d.B, d.b), threads, (size_t)d.hq * sizeof(double), s>>>(
+      d, static_cast<const bf16*>(q), static_cast<const bf16*>(q_prev), delta, mse, active);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_page_minmax(const SparseArgs& a, cudaStream_t s) {
   if (a.P <= a.p_first) return cudaSuccess;

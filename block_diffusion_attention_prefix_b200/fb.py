@@ -18,7 +18,7 @@ __all__ = [
     "fb_version", "fb_status_string", "fb_device_error", "fb_workspace_bytes", "fb_workspace_init",
     "fb_gate_eval", "fb_prefix_attn", "fb_prefix_attn_noalloc", "fb_block_attn", "fb_merge", "fb_block_merge", "fb_step",
     "fb_page_minmax", "fb_append_block", "fb_similarity_workspace_bytes", "fb_head_similarity",
-    "fb_refresh_reference", "fb_sparse_workspace_bytes", "fb_sparse_select", "fb_sparse_step", "Sparse",
+    "fb_refresh_reference", "fb_losa_step", "LosaLayer", "fb_sparse_workspace_bytes", "fb_sparse_select", "fb_sparse_step", "Sparse",
     "SparseResidualLayer", "CachedAttentionLayer", "EXPORTED",
 ]
 
@@ -86,6 +86,8 @@ EXPORTED = {
     "fb_similarity_workspace_bytes": (_sz, [_PS]),
     "fb_head_similarity": (_i, [_PS, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fb_refresh_reference": (_i, [_PS, _vp, _vp, _vp, _vp]),
+    "fb_losa_step": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_float, _PSP, _vp, _vp, _vp, _vp, _vp, _sz,
+                          _vp]),
     "fb_sparse_workspace_bytes": (_sz, [_PS, _i]),
     "fb_sparse_select": (_i, [_PS, _vp, _PG, _PSP, _vp, _sz, _vp]),
     "fb_sparse_step": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _PG, _PSP, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -245,6 +247,15 @@ def fb_refresh_reference(shape, q, q_ref, dec_reuse):
                                                                _ptr(dec_reuse), _stream()))
 
 
+def fb_losa_step(shape, q, q_prev, k_cache, v_cache, k_blk, v_blk, delta, sparse, a_full, l_full, mse, dec_active,
+                 ws):
+    _check("fb_losa_step", load().fb_losa_step(ctypes.byref(shape), _ptr(q), _ptr(q_prev), _ptr(k_cache),
+                                               _ptr(v_cache), _ptr(k_blk), _ptr(v_blk), float(delta),
+                                               ctypes.byref(sparse), _ptr(a_full), _ptr(l_full), _ptr(mse),
+                                               _ptr(dec_active), _ptr(ws), ws.numel() * ws.element_size(),
+                                               _stream()))
+
+
 def fb_sparse_workspace_bytes(shape, page_size=16) -> int:
     return int(load().fb_sparse_workspace_bytes(ctypes.byref(shape), int(page_size)))
 
@@ -386,3 +397,32 @@ class CachedAttentionLayer:
         nbytes = fb_workspace_bytes(self.shape)
         if nbytes > self.ws.numel():
             self.ws = torch.zeros(((nbytes + 15) // 16 * 16,), device=self.ws.device, dtype=torch.uint8)
+
+
+class LosaLayer(SparseResidualLayer):
+    """One layer in LoSA mode: the first step of a block runs fb_step densely into the
+    prefix cache (held in the sparse state's a_res / l_res); later steps run
+    fb_losa_step with the previous step's queries."""
+
+    def __init__(self, batch, h_q, h_kv, head_dim, block, k_cache, v_cache, n_select, delta, page_size=16,
+                 scale=0.0, keep_sel=False):
+        super().__init__(batch, h_q, h_kv, head_dim, block, k_cache, v_cache, n_select, page_size, scale, keep_sel)
+        dev = k_cache.device
+        self.delta = float(delta)
+        self.mse = torch.zeros((batch, block), device=dev, dtype=torch.float32)
+        self.active = torch.zeros((batch, block), device=dev, dtype=torch.uint8)
+        nb = fb_workspace_bytes(self.shape)
+        self.dense_ws = torch.zeros(((nb + 15) // 16 * 16,), device=dev, dtype=torch.uint8)
+        self.q_prev = None
+
+    def step(self, q, k_blk, v_blk, mask, first_step, tau=0):
+        if first_step:
+            g = make_gate(mask, True, 1)
+            fb_step(self.shape, q, self.k_cache, self.v_cache, k_blk, v_blk, g, self.a_res, self.l_res,
+                    self.a_full, self.l_full, self.dec_M, self.dec_reuse, self.dense_ws)
+            self.active.fill_(1)
+        else:
+            fb_losa_step(self.shape, q, self.q_prev, self.k_cache, self.v_cache, k_blk, v_blk, self.delta,
+                         self.sparse, self.a_full, self.l_full, self.mse, self.active, self.ws)
+        self.q_prev = q.clone()
+        return self.a_full

@@ -198,6 +198,28 @@ typedef struct fb_sparse {
 int fb_page_minmax(const fb_shape* shape, const void* k_cache, int page_size, void* kmin, void* kmax,
                    fb_stream_t stream);
 
+/* LoSA-style step (after a block's first step, which runs fb_step densely with
+ * sp->a_res / sp->l_res as its cache A_out / L_out).  "LoSA: Locality Aware Sparse
+ * Attention for Block-Wise Diffusion Language Models" (gist.science 2604.12056),
+ * "2. Methodology": tokens whose queries moved (active) get sparse attention over
+ * the prefix, stable tokens reuse the prefix attention of the previous step, and
+ * the KV pages loaded are the union over the active tokens only.
+ *   1. score[b, i] = mean over heads and channels of (q - q_prev)^2 (float64, fixed
+ *      order: per head ascending d, heads ascending; float32 result) -> `mse`
+ *      (nullable); dec_active[b, i] = score > delta;
+ *   2. every row (head) of an active token: page estimates and top-k as in
+ *      fb_sparse_select (sel_idx / sel_bits rows of stable tokens are not written);
+ *      union_bits = union over the active rows of each KV group;
+ *   3. one pass over the union pages: active rows get (A, L) over their selected
+ *      pages, which overwrites their cache row in sp->a_res / sp->l_res; stable rows
+ *      keep theirs; A_full = merge(cache row, in-block row) for every row.
+ * q, q_prev [b, H_q, B, D] bf16; the other arguments as in fb_sparse_step (gate
+ * none: the score decides).  Workspace: fb_sparse_workspace_bytes. */
+int fb_losa_step(const fb_shape* shape, const void* q, const void* q_prev, const void* k_cache,
+                 const void* v_cache, const void* k_blk, const void* v_blk, float delta, const fb_sparse* sp,
+                 void* a_full, float* l_full, float* mse, uint8_t* dec_active, void* ws, size_t ws_bytes,
+                 fb_stream_t stream);
+
 /* Per-head similarity estimate for the gamma gate.  FlashBlock technical summary
  * (gist.science 2602.05305), "Adaptive reuse strategies": in the video setting only
  * heads whose estimated cross-step similarity is above gamma reuse their cache; the

@@ -24,6 +24,7 @@ Modules:
 * :mod:`oracle.sparse`     -- page bounds, top-k page selection and the residual split.
 * :mod:`oracle.transition` -- the block transition: a finished block joins the prefix.
 * :mod:`oracle.similarity` -- the per-head similarity estimate behind the gamma gate.
+* :mod:`oracle.losa`       -- LoSA-style per-token reuse: active tokens sparse, stable tokens cached.
 
 Pins: every function here is pinned by ``tests/test_oracle_*.py`` against
 library routines (torch float64 SDPA, logsumexp, full sorts), closed forms and

@@ -12,12 +12,14 @@ import oracle.flashblock as OF
 import oracle.sparse as OS
 import oracle.transition as OT
 import oracle.similarity as OSim
+import oracle.losa as OL
 
 from tests import test_oracle_attention as TA
 from tests import test_oracle_flashblock as TF
 from tests import test_oracle_sparse as TS
 from tests import test_oracle_transition as TT
 from tests import test_oracle_similarity as TSim
+from tests import test_oracle_losa as TL
 
 _orig_attend = OA.attend
 _orig_merge = OA.merge
@@ -127,6 +129,22 @@ def _sim_no_sqrt(q, q_ref):
     return out
 
 
+_orig_token_mse = OL.token_mse
+_orig_union = OL.union_bitmap
+
+
+def _mse_no_mean(q, q_prev):
+    # the squared differences summed but not divided by H_q * D
+    return (_orig_token_mse(q, q_prev).astype(np.float64) * (np.asarray(q).shape[1] * np.asarray(q).shape[3])
+            ).astype(np.float32)
+
+
+def _union_with_stable_rows(sel_rows, n_pages_):
+    # stable rows' -1 entries folded in as page 0 (the union taken over every row)
+    s = np.asarray(sel_rows)
+    return _orig_union(np.concatenate([s, np.zeros(1, np.int64)]), n_pages_)
+
+
 PINS_ATTN = [
     lambda: TA.test_attend_matches_torch_sdpa_and_logsumexp(3, 7, 16, 0.25),
     lambda: TA.test_golden_attention_cases(),
@@ -146,6 +164,9 @@ PINS_SIM = [lambda: TSim.test_matches_library_cosine(300),
             lambda: TSim.test_closed_forms(),
             lambda: TSim.test_pairwise_tree_order_inside_a_chunk()]
 
+PINS_LOSA = [lambda: TL.test_token_mse_matches_library_mean(),
+             lambda: TL.test_union_is_over_active_rows_only()]
+
 MUTANTS = [
     ("merge: denominator drops w_in", [(OA, "merge"), (OF, "merge"), (OS, "merge")], _merge_den_drop, PINS_ATTN),
     ("merge: L drops ln(w1+w2)", [(OA, "merge"), (OF, "merge"), (OS, "merge")], _merge_L_drop, PINS_ATTN),
@@ -162,6 +183,8 @@ MUTANTS = [
     ("transition: block before the prefix", [(OT, "append_block")], _append_block_first, PINS_TRANSITION),
     ("similarity: rows summed in sequence", [(OSim, "_ordered_sum")], _sum_sequential, PINS_SIM),
     ("similarity: norm without the square root", [(OSim, "head_similarity")], _sim_no_sqrt, PINS_SIM),
+    ("LoSA: score summed, not averaged", [(OL, "token_mse")], _mse_no_mean, PINS_LOSA),
+    ("LoSA: union over every row", [(OL, "union_bitmap")], _union_with_stable_rows, PINS_LOSA),
 ]
 
 
@@ -180,5 +203,5 @@ def test_pins_catch_planted_mistake(monkeypatch, name, targets, mutant, pins):
 
 
 def test_pins_pass_on_unmutated_oracle():
-    for pin in PINS_ATTN + PINS_GATE + PINS_SPARSE + PINS_TRANSITION + PINS_SIM:
+    for pin in PINS_ATTN + PINS_GATE + PINS_SPARSE + PINS_TRANSITION + PINS_SIM + PINS_LOSA:
         pin()
