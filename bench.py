@@ -203,10 +203,15 @@ class DeviceWorkload:
         self.a_full = torch.zeros((w.batch, w.h_q, w.block, w.head_dim), device=dev, dtype=w.torch_dtype)
         self.l_full = torch.zeros((w.batch, w.h_q, w.block), **f32)
         self.sparse_layer = None
+        self.losa = w.losa_delta is not None
         if w.page_size:
             n_sel = sparse_n_select(w)
-            self.sparse_layer = fb.SparseResidualLayer(w.batch, w.h_q, w.h_kv, w.head_dim, w.block, self.k, self.v,
-                                                       n_sel, w.page_size)
+            if self.losa:
+                self.sparse_layer = fb.LosaLayer(w.batch, w.h_q, w.h_kv, w.head_dim, w.block, self.k, self.v,
+                                                 n_sel, w.losa_delta, w.page_size)
+            else:
+                self.sparse_layer = fb.SparseResidualLayer(w.batch, w.h_q, w.h_kv, w.head_dim, w.block, self.k,
+                                                           self.v, n_sel, w.page_size)
             self.ws = self.sparse_layer.ws
         else:
             n = fb.fb_workspace_bytes(self.shape)
@@ -222,6 +227,8 @@ class DeviceWorkload:
         return 1 if self.w.block <= 64 else 3
 
     def entry(self, lib):
+        if self.losa:  # the marshalled arguments start with the entry point of that step
+            return lambda fn, *a: fn(*a)
         return lib.fb_sparse_step if self.sparse_layer is not None else lib.fb_step
 
     def step_args(self, i: int, dec_M, dec_reuse, tau_override=None):
@@ -232,6 +239,23 @@ class DeviceWorkload:
         g = fb.make_gate(s["mask"], s["first"], tau, s["sim"], self.w.gamma or 0.0)
         vp = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
         stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+        if self.losa:
+            lay, lib = self.sparse_layer, fb.load()
+            pos = i % len(self.sched)
+            if s["first"]:  # dense first step into the LoSA cache
+                g = fb.make_gate(s["mask"], True, 1)
+                args = (lib.fb_step, ctypes.byref(self.shape), vp(s["q"]), vp(self.k), vp(self.v), vp(s["k_blk"]),
+                        vp(s["v_blk"]), ctypes.byref(g), vp(lay.a_res), vp(lay.l_res), vp(self.a_full),
+                        vp(self.l_full), vp(dec_M), vp(dec_reuse), vp(lay.dense_ws), lay.dense_ws.numel(), stream)
+                return args, g
+            # tau_override=0 asks for the no-reuse reference: every token active (plain sparse attention)
+            delta = float("-inf") if tau_override == 0 else self.w.losa_delta
+            prev = self.sched[pos - 1]["q"]
+            args = (lib.fb_losa_step, ctypes.byref(self.shape), vp(s["q"]), vp(prev), vp(self.k), vp(self.v),
+                    vp(s["k_blk"]), vp(s["v_blk"]), ctypes.c_float(delta), ctypes.byref(lay.sparse),
+                    vp(self.a_full), vp(self.l_full), vp(lay.mse), vp(lay.active), vp(self.ws), self.ws.numel(),
+                    stream)
+            return args, g
         if self.sparse_layer is not None:
             sl = self.sparse_layer
             args = (ctypes.byref(self.shape), vp(s["q"]), vp(self.k), vp(self.v), vp(s["k_blk"]), vp(s["v_blk"]),
@@ -341,6 +365,40 @@ def device_arm(args, rank, world):
     alg, alg_reuse = dw.algorithmic_bytes()
     rec_ms = [step_ms[i] for i in recompute_steps]
     achieved = (alg * len(rec_ms)) / (sum(rec_ms) / 1e3) / 1e9 if rec_ms else None
+    losa = None
+    if dw.losa:
+        # Dense first steps vs LoSA steps; the roofline is taken over the LoSA steps with
+        # each schedule position's own bytes (its active rows' union pages), counted in an
+        # untimed replay of the schedule (positions are deterministic).
+        firsts = [dw.sched[(start + i) % npos]["first"] for i in range(K)]
+        recompute_steps = [i for i in range(K) if firsts[i]]
+        reuse_steps = [i for i in range(K) if not firsts[i]]
+        lay = dw.sparse_layer
+        q_b = w.batch * w.h_q * w.block * w.head_dim * w.elem_bytes
+        kvb = 2 * w.batch * w.h_kv * w.block * w.head_dim * w.elem_bytes
+        cache = w.batch * w.h_q * w.block * (w.head_dim + 1) * 4
+        out = w.batch * w.h_q * w.block * (w.head_dim * w.elem_bytes + 4)
+        page_kv = 2 * 16 * w.head_dim * w.elem_bytes
+        pos_bytes, pos_union, pos_active = {}, {}, {}
+        for pos in range(npos):
+            st = step_fn(*warm[pos][0])
+            assert st == 0, fb.fb_status_string(st)
+            if not dw.sched[pos]["first"]:
+                torch.cuda.synchronize()
+                u = lay.union_bits.cpu().numpy().astype("uint32")
+                pages = sum(bin(int(x)).count("1") for x in u.reshape(-1))
+                pos_union[pos] = pages / (u.shape[0] * u.shape[1] * lay.n_pages)
+                pos_active[pos] = float(lay.active.float().mean())
+                pos_bytes[pos] = pages * page_kv + 2 * q_b + kvb + cache + out
+        l_ms = [step_ms[i] for i in reuse_steps]
+        l_bytes = [pos_bytes[(start + i) % npos] for i in reuse_steps]
+        achieved = sum(l_bytes) / (sum(l_ms) / 1e3) / 1e9 if l_ms else None
+        alg = int(sum(l_bytes) / len(l_bytes)) if l_bytes else 0
+        rec_ms = l_ms
+        losa = dict(delta=w.losa_delta, active_token_fraction=statistics.mean(pos_active.values()),
+                    union_density_active_rows=statistics.mean(pos_union.values()),
+                    losa_step_us=_mean_us(step_ms, reuse_steps), dense_first_step_us=_mean_us(step_ms,
+                                                                                             recompute_steps))
     traffic = ncu_traffic(args.workload)
     tensor = None
     if w.block > 64:
@@ -437,7 +495,9 @@ def device_arm(args, rank, world):
                     l2="flushed between timed steps, outside the step events: 256 MiB write then 256 MiB read "
                        "(the read evicts the write's dirty lines)",
                     parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
-        roofline=dict(bound="hbm", kernel=("sparse step (page estimate + top-k + sparse_pass_kernel), recompute steps"
+        roofline=dict(bound="hbm", kernel=("LoSA step (token score + page estimate + top-k + sparse_pass_kernel), "
+                                           "LoSA steps" if dw.losa else
+                                           "sparse step (page estimate + top-k + sparse_pass_kernel), recompute steps"
                                            if dw.sparse_layer is not None else
                                            (("pass_tc_kernel" if w.group * w.block > 16 and w.head_dim == 128
                                              else "pass_bf16_kernel") if w.dtype == "bf16" else "pass_f32_kernel")
@@ -461,8 +521,10 @@ def device_arm(args, rank, world):
                        dense_recompute_step_us=(statistics.mean(dense_ms) * 1e3) if dense_ms else None,
                        dense_steps_per_s=(1e3 / statistics.mean(dense_ms)) if dense_ms else None,
                        wall_s=wall),
-        gpu_launches=dw.launches_per_step() * K,
-        sparse=None if dw.sparse_layer is None else dict(
+        gpu_launches=(sum(1 if dw.sched[(start + i) % npos]["first"] else 4 for i in range(K)) if dw.losa
+                      else dw.launches_per_step() * K),
+        losa=losa,
+        sparse=None if (dw.sparse_layer is None or dw.losa) else dict(
             n_select=dw.sparse_layer.sparse.n_select, pages=dw.sparse_layer.n_pages, union_density=dw.union_density(),
             reuse_step_gbs=(alg_reuse * len(reuse_steps)) / (sum(step_ms[i] for i in reuse_steps) / 1e3) / 1e9
             if reuse_steps else None),
@@ -559,7 +621,17 @@ def oracle_steps(w: W.Workload, seed: int, budget_s: float, max_steps: int, kv_g
     kk = k[:, :hk].double().numpy()
     vv = v[:, :hk].double().numpy()
     del k, v
-    if w.page_size:
+    if w.losa_delta is not None:
+        from oracle import losa as OL
+        lo = OL.LosaAttention(kk, vv, hq, 1 / math.sqrt(w.head_dim), w.page_size, w.density)
+        prev = {}
+
+        def losa_step(q, kb, vb, mask, first, tau, sim, gamma):
+            r = lo.step(q, prev.get("q"), kb, vb, first, w.losa_delta)
+            prev["q"] = q
+            return r
+        st = type("LosaStep", (), {"step": staticmethod(losa_step)})()
+    elif w.page_size:
         sp = OS.SparseResidualAttention(kk, vv, hq, 1 / math.sqrt(w.head_dim), w.page_size, w.density)
         st = type("SparseStep", (), {"step": staticmethod(
             lambda q, kb, vb, mask, first, tau, sim, gamma: sp.step(q, kb, vb, mask, first, tau))})()

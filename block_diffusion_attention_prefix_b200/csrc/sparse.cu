@@ -139,9 +139,10 @@ constexpr int kEstThreads = kEstPages * kEstRowLanes;
 // the ordered sum.  The bounds of the next 8 channels are loaded while the current
 // 8 are consumed.
 template <int D, int NT>
-__device__ void estimate_pages(const SparseArgs& a, int bg, int p_lo, int p_hi, const double* sq, int tid) {
+__device__ void estimate_pages(const SparseArgs& a, int bg, int p_lo, int p_hi, const double* sq, int tid,
+                               const int* rows, int nrows) {
   const Dims& d = a.d;
-  const int R = d.R;
+  const int R = nrows;  // rows[0 .. nrows) are the group rows to estimate
   const int b = bg / d.hkv, kvh = bg - b * d.hkv;
   const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B;
   const int npg = p_hi - p_lo;
@@ -167,10 +168,9 @@ __device__ void estimate_pages(const SparseArgs& a, int bg, int p_lo, int p_hi, 
 #pragma unroll
         for (int t = 0; t < 8; ++t) {
           const double kmn = (double)n8[t], kmx = (double)x8[t];
-          const double* qc = sq + (size_t)r0 * D + c0 + t;
 #pragma unroll
           for (int j = 0; j < kEstRows; ++j) {
-            const double qv = qc[(size_t)j * D];
+            const double qv = sq[(size_t)rows[min(r0 + j, R - 1)] * D + c0 + t];
             acc[j] = fma(qv, qv >= 0.0 ? kmx : kmn, acc[j]);  // exact product, one rounding
           }
         }
@@ -186,7 +186,7 @@ __device__ void estimate_pages(const SparseArgs& a, int bg, int p_lo, int p_hi, 
       }
 #pragma unroll
       for (int j = 0; j < kEstRows; ++j)
-        if (r0 + j < R) a.est[(grow0 + r0 + j) * (size_t)a.P + p] = acc[j];
+        if (r0 + j < R) a.est[(grow0 + rows[r0 + j]) * (size_t)a.P + p] = acc[j];
     }
   }
 }
@@ -214,9 +214,19 @@ __global__ void __launch_bounds__(kEstThreads) page_estimate_kernel(const Sparse
     const int w = p0 / 32 + threadIdx.x;
     if (w < a.words) a.union_bits[(size_t)bg * a.words + w] = 0u;
   }
+  // The group rows to estimate: all, or (LoSA) the rows of active tokens.
+  __shared__ int s_rows[1024];
+  __shared__ int s_nrows;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int r = 0; r < d.R && r < 1024; ++r)
+      if (!a.active || a.active[(size_t)b * d.B + r % d.B]) s_rows[n++] = r;
+    s_nrows = n;
+  }
   load_group_q<D, kEstThreads>(a, bg, sq, threadIdx.x);
   __syncthreads();
-  estimate_pages<D, kEstThreads>(a, bg, p0, min(a.P, p0 + kEstPages), sq, threadIdx.x);
+  if (s_nrows > 0)
+    estimate_pages<D, kEstThreads>(a, bg, p0, min(a.P, p0 + kEstPages), sq, threadIdx.x, s_rows, s_nrows);
 }
 
 // ------------------------------------------------------------------ top-k pages

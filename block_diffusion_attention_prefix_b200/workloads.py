@@ -54,6 +54,7 @@ class Workload:
     kv_head_scale: bool        # per-KV-head scale c_g ~ U(0.5, 2), times 0.5
     page_size: int = 0         # sparse workloads only
     density: float = 0.0       # sparse workloads only
+    losa_delta: Optional[float] = None  # LoSA workloads: activity threshold on the locality score
     description: str = ""
 
     @property
@@ -107,6 +108,10 @@ WORKLOADS = {
     "sparse64k": _dlm("sparse64k", 65536, 4, 16, page_size=16, density=0.2,
                       description="sparse+residual bf16: dLM-8B-like shapes, N=65536, 16-token pages, "
                                   "density 0.2, B=4, 16 steps, tau=2"),
+    "losa64k": _dlm("losa64k", 65536, 4, 16, page_size=16, density=0.2, losa_delta=0.01,
+                    description="LoSA-style bf16: sparse64k shapes; after a dense first step, tokens whose "
+                                "queries moved (score > 0.01) get sparse attention over their top 20% pages, "
+                                "stable tokens reuse; union over active tokens only"),
 }
 
 
