@@ -19,6 +19,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+from typing import Optional
 import json
 import math
 import os
@@ -48,18 +49,27 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash() -> str:
+# Sources each profiled kernel is built from (its own translation unit and the headers
+# it includes): a committed DRAM-traffic figure stays valid while these are unchanged.
+KERNEL_SOURCES = {
+    "pass_bf16_kernel": ["prefix_bf16.cu", "fb_device.cuh", "fb_ptx.cuh", "fb_internal.h"],
+    "pass_tc_kernel": ["flash_tc.cu", "fb_device.cuh", "fb_ptx.cuh", "fb_internal.h"],
+}
+
+
+def kernel_source_hash(kernel: Optional[str] = None) -> str:
+    """sha256 (16 hex) of one kernel's sources, or of every CUDA source when None."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_diffusion_attention_prefix_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    files = KERNEL_SOURCES[kernel] if kernel else sorted(f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh", ".h")))
+    for f in files:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(workload: str):
-    """DRAM bytes per launch of the prefix kernel from the committed ncu summary,
-    or None when the summary is absent or was taken on other kernel sources."""
+    """DRAM bytes per launch of the profiled kernel from the committed ncu summary,
+    or None when the summary is absent or was taken on other sources of that kernel."""
     path = os.path.join(ROOT, "profiles", f"prefix_pass_{workload}.md")
     if not os.path.exists(path):
         return None
@@ -68,7 +78,8 @@ def ncu_traffic(workload: str):
         if ":" in line and line.strip().startswith("- "):
             k, v = line.strip()[2:].split(":", 1)
             vals[k.strip()] = v.strip().strip("`")
-    if vals.get("kernel_source_sha") != kernel_source_hash():
+    kernel = vals.get("kernel")
+    if kernel not in KERNEL_SOURCES or vals.get("kernel_source_sha") != kernel_source_hash(kernel):
         return None
     try:
         return float(vals["dram_bytes_per_launch"])

@@ -79,15 +79,18 @@ __global__ void merge_kernel(const Dims d, const float* a1, const float* l1, con
   }
 }
 
-// Block transition: one CTA per (b, KV head) copies the block's B rows of K and V
-// into cache rows [N, N + B) (16-byte vectors; rows of the cache may be padded).
+// Block transition: CTA (chunk, b * H_kv) copies rows [64 chunk, 64 chunk + 64) of the
+// block's K and V into cache rows N + those (16-byte vectors; cache rows may be padded).
+constexpr int kAppendRows = 64;
 __global__ void append_block_kernel(const Dims d, uint8_t* k_cache, uint8_t* v_cache, const uint8_t* k_blk,
                                     const uint8_t* v_blk, int elem_bytes) {
-  const int bg = blockIdx.x;
+  const int bg = blockIdx.y;
+  const int row0 = blockIdx.x * kAppendRows;
+  const int rows = min(kAppendRows, d.B - row0);
   const int vec_per_row = d.D * elem_bytes / 16;
-  const size_t n = (size_t)d.B * vec_per_row;
-  const size_t src0 = (size_t)bg * d.B * d.D * elem_bytes;
-  const size_t dst0 = ((size_t)bg * d.head_stride + (size_t)d.N * d.row_stride) * elem_bytes;
+  const size_t n = (size_t)rows * vec_per_row;
+  const size_t src0 = ((size_t)bg * d.B + row0) * d.D * elem_bytes;
+  const size_t dst0 = ((size_t)bg * d.head_stride + (size_t)(d.N + row0) * d.row_stride) * elem_bytes;
   for (size_t i = threadIdx.x; i < 2 * n; i += blockDim.x) {
     const bool isv = i >= n;
     const size_t j = isv ? i - n : i;
@@ -124,7 +127,8 @@ cudaError_t launch_gate_eval(const Dims& d, const GateParams& g, int32_t* dec_M,
 
 cudaError_t launch_append_block(const Dims& d, void* k_cache, void* v_cache, const void* k_blk, const void* v_blk,
                                 cudaStream_t s) {
-  append_block_kernel<<<d.b * d.hkv, 256, 0, s>>>(d, static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache),
+  const dim3 grid((d.B + kAppendRows - 1) / kAppendRows, d.b * d.hkv);
+  append_block_kernel<<<grid, 256, 0, s>>>(d, static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache),
                                                    static_cast<const uint8_t*>(k_blk),
                                                    static_cast<const uint8_t*>(v_blk), d.dtype == 1 ? 2 : 4);
   return cudaGetLastError();

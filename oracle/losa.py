@@ -53,7 +53,8 @@ def token_mse(q: np.ndarray, q_prev: np.ndarray) -> np.ndarray:
     total = np.zeros((b, B))
     for h in range(hq):                     # heads in ascending order
         total = total + head_sums[:, h]
-    return (total / (hq * D)).astype(np.float32)
+    with np.errstate(over="ignore"):  # scores beyond the float32 range round to inf, as a float32 cast does
+        return (total / (hq * D)).astype(np.float32)
 
 
 @dataclasses.dataclass
