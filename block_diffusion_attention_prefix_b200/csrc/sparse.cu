@@ -69,10 +69,27 @@ __global__ void token_mse_kernel(const Dims d, const bf16* q, const bf16* qp, fl
   const int i = blockIdx.x, b = blockIdx.y;
   for (int h = threadIdx.x; h < d.hq; h += blockDim.x) {
     const size_t off = (((size_t)b * d.hq + h) * d.B + i) * d.D;
+    const uint4* qv = reinterpret_cast<const uint4*>(q + off);
+    const uint4* pv = reinterpret_cast<const uint4*>(qp + off);
     double acc = 0.0;
-    for (int k = 0; k < d.D; ++k) {
-      const double diff = __dsub_rn((double)__bfloat162float(q[off + k]), (double)__bfloat162float(qp[off + k]));
-      acc = __dadd_rn(acc, __dmul_rn(diff, diff));
+    for (int c0 = 0; c0 < d.D / 8; c0 += 8) {  // 64 channels' loads in flight, then their terms in order
+      uint4 xa[8], xb[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        xa[c] = c0 + c < d.D / 8 ? __ldg(qv + c0 + c) : make_uint4(0, 0, 0, 0);
+        xb[c] = c0 + c < d.D / 8 ? __ldg(pv + c0 + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        if (c0 + c >= d.D / 8) break;
+        const bf16* ea = reinterpret_cast<const bf16*>(&xa[c]);
+        const bf16* eb = reinterpret_cast<const bf16*>(&xb[c]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const double diff = __dsub_rn((double)__bfloat162float(ea[e]), (double)__bfloat162float(eb[e]));
+          acc = __dadd_rn(acc, __dmul_rn(diff, diff));
+        }
+      }
     }
     s_head[h] = acc;
   }
