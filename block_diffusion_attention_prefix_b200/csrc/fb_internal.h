@@ -51,7 +51,7 @@ struct SplitPlan {
   size_t total() const { return counter_bytes + partial_bytes + inblock_bytes; }
 };
 
-// What the last-arriving CTA of a (b, kv head, row tile) does with the combined rows.
+// What the split combine of a (b, kv head, row tile) does with the combined rows.
 struct Epilogue {
   int mode;               // 0: write (A, L) fp32 to a_dst / l_dst; 1: merge with (a_prev, l_prev)
   float* a_dst;           // mode 0, [b, H_q, B, D]

@@ -15,7 +15,7 @@ namespace fb {
 enum : uint32_t {
   DEV_ERR_WAIT_FULL = 1,   // consumer gave up waiting for a TMA tile
   DEV_ERR_WAIT_EMPTY = 2,  // producer gave up waiting for a free stage
-  DEV_ERR_WAIT_COMBINE = 3, // last CTA gave up waiting for its partials copy
+  DEV_ERR_WAIT_COMBINE = 3, // the split combine gave up waiting for its bulk copy of the partials
   DEV_ERR_WAIT_PEERS = 4,   // a split CTA gave up waiting for the other splits of its tile
 };
 

@@ -442,8 +442,9 @@ struct SCfg {
   static constexpr int kRingBytes = STAGES * kStageBytes;
   static constexpr int kSmemBytes = (kRingBytes > kScratchBytes ? kRingBytes : kScratchBytes) + 1024;
   static_assert(KW % 16 == 0, "whole k16 steps per warp");
-  static_assert(kRingBytes >= 2 * kRowTile * (D + 4) * 4 + 1024 + ((150 * kRowTile * 4 + 127) / 128) * 128,
-                "finisher space");
+  // The split combine stages rows x (2 splits + 1) partial rows (rows <= ceil(RT / splits)):
+  // at most 2 (2 RT + 149) + RT rows for up to 148 splits (it reads the workspace otherwise).
+  static_assert(kRingBytes >= 3 * kRowTile * (D + 4) * 4, "combine staging");
 };
 
 // Byte offset of (key in tile, d) for a tile of 4 pages (64 keys) stored as D/64

@@ -9,7 +9,7 @@ Shapes follow the FlashBlock technical summary (gist.science paper 2602.05305,
 "1. Problem definition" and "2. Methodology / Core mechanism"): a block of B
 query tokens per step, a prefix KV cache of N tokens that the block attends to
 (J_out) and the block's own B keys (J_in).  The pages give no input laws; the
-recipes below are this library's readings and are restated in the design doc:
+recipes below are this library's readings:
 
 * Q ~ N(0, 1).  Prefix and in-block K/V ~ N(0, 1) * 0.5 * c_g with a per-KV-head
   scale c_g ~ U(0.5, 2) (dLM, long-context, video and sparse workloads); the

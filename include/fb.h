@@ -104,8 +104,12 @@ int fb_version(void);
 const char* fb_status_string(int status);
 
 /* Reads and clears the device error word of the current device: 0 if no kernel
- * hit a wait bound since the last call, else a nonzero code.  Synchronises the
- * current device. */
+ * hit a wait bound since the last call, else a nonzero code: 1 a tile load did not
+ * arrive, 2 the producer found no free stage, 3 the bulk copy of split partials did
+ * not arrive, 4 the split CTAs of a tile (or the grid) did not all arrive.  Each wait
+ * gives up after 2 s.  Synchronises the current device.  After a nonzero code the
+ * outputs of the failed calls are undefined and workspaces should be re-initialised
+ * (fb_workspace_init). */
 int fb_device_error(int32_t* code);
 
 /* Workspace (device bytes) needed by fb_prefix_attn / fb_step / fb_block_merge for
@@ -115,12 +119,14 @@ int fb_device_error(int32_t* code);
 size_t fb_workspace_bytes(const fb_shape* shape);
 int fb_workspace_init(void* ws, size_t ws_bytes, fb_stream_t stream);
 
-/* Gate only (a1-a3): writes dec_M [b] and dec_reuse [b, H_q]. */
+/* Gate only (the updated-token count, the tau gate and the per-head gamma gate):
+ * writes dec_M [b] and dec_reuse [b, H_q]. */
 int fb_gate_eval(const fb_shape* shape, const fb_gate* gate, int32_t* dec_M, uint8_t* dec_reuse,
                  fb_stream_t stream);
 
-/* Out-of-block attention (a4, a5, a8): (A_out, L_out) of every query row over the
- * whole prefix J_out, computed split-KV and reduced in log space.  With gate ==
+/* Out-of-block attention (split-KV pass, split combine, cache write): (A_out, L_out)
+ * of every query row over the whole prefix J_out, computed split-KV and reduced in
+ * log space.  With gate ==
  * NULL every row is recomputed; otherwise only rows of heads whose decision is
  * "recompute" are written, and rows of reusing heads are left bit-for-bit
  * untouched (the decision is taken on the device; no host synchronisation).
@@ -129,19 +135,19 @@ int fb_prefix_attn(const fb_shape* shape, const void* q, const void* k_cache, co
                    const fb_gate* gate, float* a_out, float* l_out, void* ws, size_t ws_bytes,
                    fb_stream_t stream);
 
-/* In-block attention (a6): (A_in, L_in) of every query row over the B block keys,
+/* In-block attention: (A_in, L_in) of every query row over the B block keys,
  * bidirectional (no mask).  ws may be NULL when block <= 64; larger blocks need
  * fb_workspace_bytes(shape) bytes. */
 int fb_block_attn(const fb_shape* shape, const void* q, const void* k_blk, const void* v_blk,
                   float* a_in, float* l_in, void* ws, size_t ws_bytes, fb_stream_t stream);
 
-/* Log-space merge (a7), elementwise over [b, H_q, B] rows:
+/* Log-space merge, elementwise over [b, H_q, B] rows:
  * A_full = merge((a1, l1), (a2, l2)) in the shape's dtype; l_full (nullable) gets
  * m + ln(e^{l1-m} + e^{l2-m}).  Two empty inputs give (0, -inf). */
 int fb_merge(const fb_shape* shape, const float* a1, const float* l1, const float* a2,
              const float* l2, void* a_full, float* l_full, fb_stream_t stream);
 
-/* Second half of a step (a1-a3, a6, a7): evaluates the gate, records dec_M /
+/* Second half of a step (gate, in-block attention, merge): evaluates the gate, records dec_M /
  * dec_reuse (nullable), computes (A_in, L_in) and merges it with the cache
  * (a_out, l_out) as it is in memory, writing A_full and L_full (nullable).
  * gate may be NULL (then no decision is recorded).  ws as for fb_block_attn. */

@@ -17,7 +17,7 @@ Follows the FlashBlock technical summary (gist.science, paper 2602.05305):
   - per-head selection (video): only heads whose estimated similarity is above
     gamma reuse the cache.
 
-Readings where the pages are silent (listed in the design doc):
+Readings where the pages are silent:
   R3  tau: strict ``M < tau`` reuses; ``M >= tau`` recomputes.
   R4  gamma: strict ``sim > gamma`` reuses (compared in float32, as given).
   R5  tau is one decision per batch element; gamma one per (batch, head).

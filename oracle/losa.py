@@ -15,7 +15,7 @@ Models" (gist.science, paper 2604.12056):
 The prefix result is then combined with the block's own keys by the FlashBlock
 merge (FlashBlock technical summary, "Core mechanism"), as in the cached step.
 
-Readings where the pages are silent (listed in the design doc):
+Readings where the pages are silent:
   L1  the locality score of token i is the mean over all query heads and channels
       of (q_t - q_{t-1})^2, in float64 in a fixed order (per head ascending d, each
       term rounded as a product then a sum; heads in ascending order), divided by

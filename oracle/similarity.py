@@ -8,7 +8,7 @@ each head, how similar the current denoising step is to the cached one, and only
 heads whose estimated similarity is above gamma reuse their cache.  The pages do
 not give the estimator.
 
-Readings (listed in DESIGN.md):
+Readings where the pages are silent:
   S1  the similarity of head h is the cosine between its block queries now (Q_h,
       B x D, flattened) and the queries its cached A_out was computed with (its
       queries at its last recompute): a cached row is stale exactly as far as its

@@ -9,7 +9,7 @@ to the tokens outside it (J_out), which are the earlier blocks.  When a block's
 last denoising step is done, its tokens are part of what every later block
 attends to as J_out: the prefix grows by one block.
 
-Readings where the pages are silent (listed in the design doc):
+Readings where the pages are silent:
   T1  the keys and values a finished block contributes are its in-block K/V as of
       its last denoising step; they are appended after the prefix, in block order.
   T2  the cached (A_out, L_out) of the finished block is not carried over: the next
