@@ -62,7 +62,7 @@ typedef enum fb_status {
   FB_ERR_DTYPE = -4,       /* dtype not supported for this call */
   FB_ERR_WORKSPACE = -5,   /* workspace missing or smaller than fb_workspace_bytes() */
   FB_ERR_CUDA = -6,        /* a CUDA runtime/driver call failed */
-  FB_ERR_UNSUPPORTED = -7, /* valid request this build does not implement */
+  FB_ERR_UNSUPPORTED = -7, /* valid request the library does not implement */
   FB_ERR_ARG = -8          /* other invalid argument (e.g. page size, k) */
 } fb_status;
 
