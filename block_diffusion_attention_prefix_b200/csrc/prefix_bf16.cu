@@ -111,6 +111,31 @@ __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
   }
+  if (args.step.enabled && warp == C::kAuxWarp) {
+    // Whatever the gate decides, this CTA computes its share of the in-block rows:
+    // pull their q rows, the group's block keys and values and the cached rows into
+    // L1 while the gate reads the mask.
+    int r0, r1;
+    split_rows(rows_valid, plan.splits, split, r0, r1);
+    const int lines_row = D * (int)sizeof(bf16) / 128;  // 128-byte lines per bf16 row
+    const int nq = (r1 - r0) * lines_row;
+    const int nkv = d.B * lines_row;  // per tensor
+    const int nc = (r1 - r0) * (D * 4 / 128);
+    const bf16* kb = k_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
+    const bf16* vb = v_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
+    for (int i = lane; i < nq + 2 * nkv + nc; i += 32) {
+      const void* p;
+      if (i < nq)
+        p = q + (grow0 + r0) * D + (size_t)i * (128 / sizeof(bf16));
+      else if (i < nq + nkv)
+        p = kb + (size_t)(i - nq) * (128 / sizeof(bf16));
+      else if (i < nq + 2 * nkv)
+        p = vb + (size_t)(i - nq - nkv) * (128 / sizeof(bf16));
+      else
+        p = args.ep.a_dst + (grow0 + r0) * D + (size_t)(i - nq - 2 * nkv) * 32;
+      prefetch_l1(p);
+    }
+  }
 
   if (!gate_row_flags(args.gate, d, b, kvh, row0, rows_valid, RT, s_flags, s_red, &s_M)) {
     // Every row of this tile reuses its cache: no K/V is read.  In a fused step the
