@@ -460,7 +460,7 @@ def device_arm(args, rank, world):
     tsh = fb.make_shape(w.batch, w.h_q, w.h_kv, w.head_dim, w.block, n0, w.dtype, kv_head_stride=cap * w.head_dim)
     kmn = kmx = None
     if dw.sparse_layer is not None:
-        kmn = torch.zeros((w.batch, w.h_kv, w.head_dim, (cap + 15) // 16), device=dev, dtype=w.torch_dtype)
+        kmn = torch.zeros((w.batch, w.h_kv, w.head_dim, fb.fb_page_cap(tsh)), device=dev, dtype=w.torch_dtype)
         kmx = torch.zeros_like(kmn)
     trans = []
     for i in range(32):

@@ -607,6 +607,14 @@ int sparse_args(const Dims& d, const GateParams& gp, const fb_sparse* sp, const 
 }  // namespace
 }  // namespace fb
 
+extern "C" int fb_page_cap(const fb_shape* shape, int page_size) {
+  Dims d;
+  FB_TRY(resolve(shape, &d));
+  if (page_size != kSparsePage) return FB_ERR_ARG;
+  if (d.N < 1) return FB_ERR_UNSUPPORTED;
+  return page_capacity(d);
+}
+
 extern "C" int fb_page_minmax(const fb_shape* shape, const void* k_cache, int page_size, void* kmin, void* kmax,
                               fb_stream_t stream) {
   Dims d;

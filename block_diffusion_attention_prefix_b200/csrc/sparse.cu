@@ -299,8 +299,8 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
   extern __shared__ uint32_t s_bits[];  // [words] row bitmap
   __shared__ unsigned hist[256];
   __shared__ int s_tmp[32];
-  __shared__ unsigned long long s_prefix;
-  __shared__ int s_kk;
+  __shared__ unsigned long long s_prefix, s_key;
+  __shared__ int s_kk, s_unique;
   const Dims& d = a.d;
   const int row = blockIdx.x;
   const int b = row / (d.hq * d.B);
@@ -320,12 +320,15 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
 #define FB_KEY(t) (REG > 0 ? kc.k[(t)] : desc_key(est[pb + (t)]))
 #define FB_FOR_MINE(t) _Pragma("unroll") for (int t = 0; t < (REG > 0 ? REG : 1); ++t) if (REG > 0 ? (t < n) : false)
 
-  // Radix select (8 passes of 8 bits, most significant first) of the k-th smallest key.
+  // Radix select (up to 8 passes of 8 bits, most significant first) of the k-th
+  // smallest key; it stops early once the chosen bin holds a single key, which is
+  // then the k-th smallest itself.
   unsigned long long prefix = 0, mask = 0;
   int kk = a.k_sel;
   for (int pass = 0; pass < 8; ++pass) {
     const int shift = 56 - 8 * pass;
     if (tid < 256) hist[tid] = 0u;
+    if (tid == 0) s_unique = 0;
     __syncthreads();
     if (REG > 0) {
       FB_FOR_MINE(t) {
@@ -356,24 +359,44 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
       const unsigned long long hit = __ballot_sync(0xffffffffu, excl < (unsigned)kk && (unsigned)kk <= incl);
       const int owner = __ffsll((long long)hit) - 1;
       if (tid == owner) {
-        unsigned run = excl;
+        unsigned run = excl, cnt = 0;
         int bin = 0;
         for (int j = 0; j < 8; ++j) {
           if ((unsigned)kk <= run + c[j]) {
             bin = tid * 8 + j;
+            cnt = c[j];
             break;
           }
           run += c[j];
         }
         s_prefix = prefix | ((unsigned long long)bin << shift);
         s_kk = kk - (int)run;
+        s_unique = cnt == 1u;
       }
     }
     __syncthreads();
     prefix = s_prefix;
     kk = s_kk;
     mask |= 0xFFull << shift;
+    const bool unique = s_unique != 0;
+    if (unique) {  // the one key under this prefix is the k-th smallest (kk == 1)
+      if (REG > 0) {
+        FB_FOR_MINE(t) {
+          const unsigned long long key = FB_KEY(t);
+          if ((key & mask) == prefix) s_key = key;
+        }
+      } else {
+        for (int t = 0; t < n; ++t) {
+          const unsigned long long key = FB_KEY(t);
+          if ((key & mask) == prefix) s_key = key;
+        }
+      }
+    }
     __syncthreads();
+    if (unique) {
+      prefix = s_key;
+      break;
+    }
   }
   const unsigned long long T = prefix;  // the k-th smallest key; take `kk` of the keys equal to it
 

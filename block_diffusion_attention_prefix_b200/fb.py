@@ -81,6 +81,7 @@ EXPORTED = {
     "fb_block_merge": (_i, [_PS, _vp, _vp, _vp, _PG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fb_step": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _PG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fb_prefix_attn_noalloc": (_i, [_PS, _vp, _vp, _vp, _PG, _vp, _vp, _vp]),
+    "fb_page_cap": (_i, [_PS, _i]),
     "fb_page_minmax": (_i, [_PS, _vp, _i, _vp, _vp, _vp]),
     "fb_append_block": (_i, [_PS, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
     "fb_similarity_workspace_bytes": (_sz, [_PS]),
@@ -222,6 +223,14 @@ def fb_prefix_attn_noalloc(shape, q, k_cache, v_cache, gate, a_out, l_out):
         _stream()))
 
 
+def fb_page_cap(shape, page_size=16) -> int:
+    """Page stride of the [b, H_kv, D, page_cap] bounds layout for this shape."""
+    n = int(load().fb_page_cap(ctypes.byref(shape), int(page_size)))
+    if n <= 0:
+        _check("fb_page_cap", n)
+    return n
+
+
 def fb_page_minmax(shape, k_cache, page_size, kmin, kmax):
     _check("fb_page_minmax", load().fb_page_minmax(ctypes.byref(shape), _ptr(k_cache), int(page_size), _ptr(kmin),
                                                    _ptr(kmax), _stream()))
@@ -290,7 +299,7 @@ class SparseResidualLayer:
         self.page_size = page_size
         self.n_pages = (n + page_size - 1) // page_size
         words = (self.n_pages + 31) // 32
-        page_cap = (cap + page_size - 1) // page_size
+        page_cap = fb_page_cap(self.shape, page_size)
         self.kmin = torch.empty((batch, h_kv, head_dim, page_cap), device=dev, dtype=k_cache.dtype)
         self.kmax = torch.empty_like(self.kmin)
         fb_page_minmax(self.shape, k_cache, page_size, self.kmin, self.kmax)

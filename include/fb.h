@@ -185,8 +185,8 @@ typedef struct fb_sparse {
   int32_t page_size;      /* 16 */
   int32_t n_select;       /* pages per query row, 1 .. n_pages */
   const void* kmin;       /* [b, H_kv, D, page_cap] bf16 page minima (fb_page_minmax), pages
-                             [0, n_pages) valid; page_cap = ceil(cap / page_size) with cap the
-                             K cache's row capacity per head (rows r with
+                             [0, n_pages) valid; page_cap (fb_page_cap) = ceil(cap / page_size)
+                             with cap the K cache's row capacity per head (rows r with
                              r * kv_row_stride + head_dim <= kv_head_stride; = n_prefix for a
                              contiguous cache), so the layout survives fb_append_block */
   const void* kmax;       /* same layout, page maxima */
@@ -198,6 +198,11 @@ typedef struct fb_sparse {
   float* a_sel;           /* optional output (fresh part) [b, H_q, B, D] fp32, or NULL */
   float* l_sel;           /* optional output [b, H_q, B], or NULL */
 } fb_sparse;
+
+/* The page stride page_cap of the bounds layout (see fb_sparse.kmin) for this
+ * shape: > 0, or a negative fb_status (bad shape, page_size != 16, n_prefix < 1).
+ * Host only; allocate kmin / kmax as [b, H_kv, D, page_cap] bf16. */
+int fb_page_cap(const fb_shape* shape, int page_size);
 
 /* Channel-wise page bounds of the prefix keys (exact bf16 min / max over each
  * page's real tokens; the last page may be partial). */

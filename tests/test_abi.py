@@ -121,3 +121,16 @@ def test_workspace_bytes_for_valid_and_invalid_shapes(lib):
     assert n > 0 and n % 4 == 0
     big = fb.fb_workspace_bytes(S(n_prefix=800_000, h_q=32, h_kv=8))
     assert big >= n
+
+
+@pytest.mark.parametrize("n,cap,want", [
+    (1, None, 1), (16, None, 1), (17, None, 2), (65536, None, 4096), (65536, 65552, 4097), (1000, 2000, 125),
+])
+def test_page_cap_is_the_pages_of_the_cache_capacity(lib, n, cap, want):
+    kw = dict(n_prefix=n) if cap is None else dict(n_prefix=n, kv_head_stride=cap * 128)
+    assert fb.fb_page_cap(S(**kw)) == want
+
+
+def test_page_cap_rejects_other_page_sizes(lib):
+    assert lib.fb_page_cap(ctypes.byref(S()), 8) == -8      # FB_ERR_ARG
+    assert lib.fb_page_cap(ctypes.byref(S(n_prefix=0)), 16) == -7  # FB_ERR_UNSUPPORTED

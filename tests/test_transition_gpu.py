@@ -65,13 +65,14 @@ def test_append_block_copies_rows(fb, dtype, D, rs, N, B):
 @pytest.mark.parametrize("N,B", [(15, 4), (16, 16), (17, 37), (1000, 16), (2000, 64)])
 def test_append_block_refreshes_touched_page_bounds(fb, N, B):
     b, hkv, D, cap = 1, 2, 128, N + B + 40
-    page_cap = (cap + 15) // 16
     k, v = cache_with_room(b, hkv, N, cap, D, D, torch.bfloat16, N)
     g = torch.Generator().manual_seed(9)
     kb = torch.randn((b, hkv, B, D), generator=g).to(torch.bfloat16)
     vb = torch.randn((b, hkv, B, D), generator=g).to(torch.bfloat16)
     kd, vd = k.cuda(), v.cuda()
     sh = fb.make_shape(b, 4 * hkv, hkv, D, B, N, "bf16", kv_head_stride=cap * D)
+    page_cap = fb.fb_page_cap(sh)
+    assert page_cap == (cap + 15) // 16
     kmin = torch.full((b, hkv, D, page_cap), 5.0, dtype=torch.bfloat16, device="cuda")
     kmax = kmin.clone()
     fb.fb_page_minmax(sh, kd, 16, kmin, kmax)
