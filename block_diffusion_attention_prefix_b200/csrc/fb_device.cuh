@@ -298,6 +298,10 @@ __device__ __forceinline__ float inblock_row(const T* qrow, const T* kb, const T
 // In-block rows [r_begin, r_end) of tile rows (group rows row0 + r) of KV group
 // (b, kvh), one warp per row, executed by warps [0, nwarps) of the CTA.  In mode 1
 // the cache row is loaded before the in-block math so the two latencies overlap.
+// Every mode-1 caller reads a cache that an earlier launch wrote and that no CTA of
+// its own launch writes (a reusing tile leaves its cache rows alone), so the cache
+// is read through the read-only L1 path, where the pass kernels' aux warp has
+// prefetched it while the gate read the mask.
 template <typename T, int D>
 __device__ void inblock_rows(const Dims& d, const T* q, const T* k_blk, const T* v_blk, int b, int kvh,
                              int row0, int r_begin, int r_end, const Epilogue& ep, int warp, int nwarps,
@@ -310,9 +314,9 @@ __device__ void inblock_rows(const Dims& d, const T* q, const T* k_blk, const T*
     const size_t grow = grow0 + r;
     float ap[DC], lp = 0.f;
     if (ep.mode == 1) {
-      lp = __ldcg(ep.l_prev + grow);
+      lp = __ldg(ep.l_prev + grow);
 #pragma unroll
-      for (int t = 0; t < DC; ++t) ap[t] = __ldcg(ep.a_prev + grow * D + lane * DC + t);
+      for (int t = 0; t < DC; ++t) ap[t] = __ldg(ep.a_prev + grow * D + lane * DC + t);
     }
     float a[DC];
     const float L = inblock_row<T, D>(q + grow * D, kb, vb, d.B, d.scale, a, lane);
