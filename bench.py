@@ -192,6 +192,23 @@ class L2Flush:
         torch.sum(self.r, dim=0, out=self.sink)
 
 
+def step_bytes(w: W.Workload, batch: Optional[int] = None):
+    """(recompute, reuse) algorithmic bytes of one dense step: what the fused step
+    kernel must move for `batch` problems (default: the workload's batch).
+
+    Recompute: prefix K and V, Q, the block's K and V, the cache rows written
+    (A_out and L_out, fp32) and the output (A_full in the dtype, L_full fp32).
+    Reuse: the same without the prefix K/V, with the cache read instead of written.
+    """
+    b = w.batch if batch is None else batch
+    q = b * w.h_q * w.block * w.head_dim * w.elem_bytes
+    kvb = 2 * b * w.h_kv * w.block * w.head_dim * w.elem_bytes
+    cache = b * w.h_q * w.block * (w.head_dim + 1) * 4
+    out = b * w.h_q * w.block * (w.head_dim * w.elem_bytes + 4)
+    prefix = w.prefix_bytes() // w.batch * b
+    return prefix + q + kvb + cache + out, q + kvb + cache + out
+
+
 class DeviceWorkload:
     """The workload's inputs resident in HBM and the layer state, stepped through libfb."""
 
@@ -307,18 +324,7 @@ class DeviceWorkload:
                 int(w.prefix_bytes() * dens) + q + kvb + res + out)
 
     def dense_algorithmic_bytes(self):
-        """(recompute, reuse) bytes of one step: what the fused step kernel must move.
-
-        Recompute: prefix K and V, Q, the block's K and V, the cache rows written
-        (A_out and L_out, fp32) and the output (A_full in the dtype, L_full fp32).
-        Reuse: the same without the prefix K/V, with the cache read instead of written.
-        """
-        w = self.w
-        q = w.batch * w.h_q * w.block * w.head_dim * w.elem_bytes
-        kvb = 2 * w.batch * w.h_kv * w.block * w.head_dim * w.elem_bytes
-        cache = w.batch * w.h_q * w.block * (w.head_dim + 1) * 4
-        out = w.batch * w.h_q * w.block * (w.head_dim * w.elem_bytes + 4)
-        return w.prefix_bytes() + q + kvb + cache + out, q + kvb + cache + out
+        return step_bytes(self.w)
 
 
 def batched_reuse(fb, w: W.Workload, flush, reps: int = 20, n_prefix: int = 64,
@@ -333,9 +339,7 @@ def batched_reuse(fb, w: W.Workload, flush, reps: int = 20, n_prefix: int = 64,
     if w.block > 64 or w.page_size or w.losa_delta is not None:
         return None
     dev = torch.device("cuda")
-    eb = w.elem_bytes
-    per = (w.h_q * w.block * w.head_dim * eb + 2 * w.h_kv * w.block * w.head_dim * eb
-           + w.h_q * w.block * (w.head_dim + 1) * 4 + w.h_q * w.block * (w.head_dim * eb + 4))
+    per = step_bytes(w, batch=1)[1]
     P = max(1, min(max_problems, -(-target_bytes // per)))
     g = torch.Generator(device=dev).manual_seed(1234)
     rnd = lambda *sh: torch.randn(sh, device=dev, generator=g).to(w.torch_dtype)  # noqa: E731
