@@ -40,8 +40,10 @@ from .attention import attend, merge
 
 
 def updated_count(mask: np.ndarray) -> np.ndarray:
-    """M^{s+1} per batch element: the number of block tokens marked updated."""
-    return np.asarray(mask, dtype=np.int64).reshape(mask.shape[0], -1).sum(axis=1)
+    """M^{s+1} per batch element: the number of block tokens marked updated (a
+    nonzero mask entry marks a token, whatever its value)."""
+    m = np.asarray(mask)
+    return (m != 0).reshape(m.shape[0], -1).sum(axis=1).astype(np.int64)
 
 
 def tau_reuse(M: np.ndarray, tau: int, first_step: bool) -> np.ndarray:

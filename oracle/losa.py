@@ -57,6 +57,12 @@ def token_mse(q: np.ndarray, q_prev: np.ndarray) -> np.ndarray:
         return (total / (hq * D)).astype(np.float32)
 
 
+def active_tokens(mse: np.ndarray, delta: float) -> np.ndarray:
+    """bool [b, B]: reading L2, a token is active iff its score is above delta
+    (strict, both in float32)."""
+    return np.asarray(mse, np.float32) > np.float32(delta)
+
+
 @dataclasses.dataclass
 class LosaStepResult:
     mse: np.ndarray        # float32 [b, B] (zeros on a first step)
@@ -102,7 +108,7 @@ class LosaAttention:
             if self.a_out is None:
                 raise ValueError("the first step of a block must have first_step=True")
             mse = token_mse(q, q_prev)
-            active = mse > np.float32(delta)
+            active = active_tokens(mse, delta)
             for bi in range(b):
                 rows = np.nonzero(active[bi])[0]
                 if rows.size == 0:

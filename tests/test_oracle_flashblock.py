@@ -152,3 +152,9 @@ def test_gqa_head_mapping():
         np.testing.assert_array_equal(A[0, h], a)
     A2, _ = OF.prefix_attention(q, k[:, ::-1], v[:, ::-1], 0.3)
     assert np.abs(A2[0, 0] - A[0, 0]).max() > 1e-6
+
+
+def test_updated_count_counts_nonzero_entries():
+    # a nonzero mask entry marks an updated token, whatever its value
+    mask = np.array([[0, 2, 255, 0], [1, 1, 0, 0], [0, 0, 0, 0]], dtype=np.uint8)
+    np.testing.assert_array_equal(OF.updated_count(mask), [2, 2, 0])

@@ -88,3 +88,16 @@ def test_union_is_over_active_rows_only():
             assert np.all(rows[:, ~r.active[0]] == -1)
         some_stable |= bool((~r.active).any()) and bool(r.active.any())
     assert some_stable, "want steps with both active and stable tokens"
+
+
+def test_delta_zero_keeps_unmoved_tokens_stable():
+    # tokens not updated keep their queries bit for bit, so their score is exactly 0;
+    # with delta = 0 the strict comparison keeps them stable and only moved tokens
+    # are active
+    k, v, out = _run(W_SMALL, 5, 0.0, 0.2, steps=6)
+    mixed = 0
+    for s, r in out[1:]:
+        moved = s.mask.numpy()[0].astype(bool)
+        np.testing.assert_array_equal(r.active[0], moved)
+        mixed += bool(moved.any()) and bool((~moved).any())
+    assert mixed > 0

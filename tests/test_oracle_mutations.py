@@ -4,6 +4,10 @@ Each mutant replaces one oracle function with a subtly wrong copy (a dropped ter
 a wrong sign, a transposed operand, a non-strict comparison, a wrong tie-break);
 the test passes only if at least one pin then fails.
 """
+import dataclasses
+import math
+from fractions import Fraction
+
 import numpy as np
 import pytest
 
@@ -145,16 +149,80 @@ def _union_with_stable_rows(sel_rows, n_pages_):
     return _orig_union(np.concatenate([s, np.zeros(1, np.int64)]), n_pages_)
 
 
+def _n_selected_floor(n_prefix, page, density):
+    # k rounded down instead of up
+    P = OS.n_pages(n_prefix, page)
+    return min(P, max(1 if P else 0, math.floor(Fraction(str(density)) * P)))
+
+
+def _page_minmax_zero_padded(k, page):
+    # the partial last page padded with zero rows that enter its bounds
+    N, D = k.shape
+    P = -(-N // page)
+    pad = np.zeros((P * page, D))
+    pad[:N] = k
+    blk = pad.reshape(P, page, D)
+    return blk.min(axis=1), blk.max(axis=1)
+
+
+_orig_key_mask = OS.key_mask_from_pages
+
+
+def _key_mask_complement(sel_rows, n_prefix, page):
+    # selected and residual key sets swapped
+    return ~_orig_key_mask(sel_rows, n_prefix, page)
+
+
+def _updated_count_complement(mask):
+    # counts the tokens that were not updated
+    m = np.asarray(mask)
+    return (m == 0).reshape(m.shape[0], -1).sum(axis=1).astype(np.int64)
+
+
+_orig_step = OF.CachedBlockAttention.step
+
+
+def _step_refreshes_cache(self, q, k_blk, v_blk, mask, first_step, tau, sim=None, gamma=0.0):
+    # every step recomputes the cache (a reuse step refreshes it with the new queries)
+    if self.a_out is None:
+        return _orig_step(self, q, k_blk, v_blk, mask, first_step, tau, sim, gamma)
+    r = _orig_step(self, q, k_blk, v_blk, mask, True, tau, sim, gamma)
+    M, reuse = OF.decisions(np.asarray(mask), first_step, tau, sim, gamma, np.asarray(q).shape[1])
+    return dataclasses.replace(r, M=M, reuse=reuse)
+
+
+def _active_ge(mse, delta):
+    # a token whose score equals delta counted as active
+    return np.asarray(mse, np.float32) >= np.float32(delta)
+
+
+_orig_refresh = OSim.refresh_reference
+
+
+def _refresh_reusing_heads(q, q_ref, reuse):
+    # the reusing heads take the new queries instead of the recomputing ones
+    return _orig_refresh(q, q_ref, ~np.asarray(reuse, bool))
+
+
 PINS_ATTN = [
     lambda: TA.test_attend_matches_torch_sdpa_and_logsumexp(3, 7, 16, 0.25),
     lambda: TA.test_golden_attention_cases(),
     lambda: TA.test_golden_merge_cases(),
     lambda: TA.test_merge_of_partition_equals_dense_over_union(0),
 ]
-PINS_GATE = [lambda: TF.test_golden_gate_cases()]
+PINS_GATE = [lambda: TF.test_golden_gate_cases(),
+             lambda: TF.test_updated_count_and_decision_per_step(),
+             lambda: TF.test_updated_count_counts_nonzero_entries()]
+PINS_STEP = [lambda: TF.test_tau_above_block_reuses_after_first_step(),
+             lambda: TF.test_reuse_rows_with_unchanged_query_equal_dense()]
 PINS_SPARSE = [lambda: TS.test_page_estimate_bounds_every_score_in_page(),
                lambda: TS.test_select_pages_matches_full_lexsort(0),
-               lambda: TS.test_select_ties_prefer_lower_page()]
+               lambda: TS.test_select_ties_prefer_lower_page(),
+               lambda: TS.test_n_selected(),
+               lambda: TS.test_page_minmax_partial_last_page(),
+               lambda: TS.test_page_minmax_partial_page_ignores_missing_rows(),
+               lambda: TS.test_density_one_leaves_empty_residual_and_equals_dense(),
+               lambda: TS.test_selected_part_is_attention_over_selected_pages()]
 
 PINS_TRANSITION = [lambda: TT.test_incremental_page_bounds_equal_recomputed(17, 4),
                    lambda: TT.test_appended_prefix_is_old_prefix_then_block(37, 5),
@@ -162,10 +230,12 @@ PINS_TRANSITION = [lambda: TT.test_incremental_page_bounds_equal_recomputed(17, 
 
 PINS_SIM = [lambda: TSim.test_matches_library_cosine(300),
             lambda: TSim.test_closed_forms(),
-            lambda: TSim.test_pairwise_tree_order_inside_a_chunk()]
+            lambda: TSim.test_pairwise_tree_order_inside_a_chunk(),
+            lambda: TSim.test_refresh_reference_takes_recomputing_heads()]
 
 PINS_LOSA = [lambda: TL.test_token_mse_matches_library_mean(),
-             lambda: TL.test_union_is_over_active_rows_only()]
+             lambda: TL.test_union_is_over_active_rows_only(),
+             lambda: TL.test_delta_zero_keeps_unmoved_tokens_stable()]
 
 MUTANTS = [
     ("merge: denominator drops w_in", [(OA, "merge"), (OF, "merge"), (OS, "merge")], _merge_den_drop, PINS_ATTN),
@@ -185,6 +255,17 @@ MUTANTS = [
     ("similarity: norm without the square root", [(OSim, "head_similarity")], _sim_no_sqrt, PINS_SIM),
     ("LoSA: score summed, not averaged", [(OL, "token_mse")], _mse_no_mean, PINS_LOSA),
     ("LoSA: union over every row", [(OL, "union_bitmap")], _union_with_stable_rows, PINS_LOSA),
+    ("LoSA: score equal to delta counted active", [(OL, "active_tokens")], _active_ge, PINS_LOSA),
+    ("top-k size: floor instead of ceil", [(OS, "n_selected"), (OL, "n_selected")], _n_selected_floor, PINS_SPARSE),
+    ("page bounds: partial page padded with zeros", [(OS, "page_minmax"), (OL, "page_minmax")],
+     _page_minmax_zero_padded, PINS_SPARSE),
+    ("sparse: selected and residual keys swapped", [(OS, "key_mask_from_pages"), (OL, "key_mask_from_pages")],
+     _key_mask_complement, PINS_SPARSE),
+    ("M: counts the tokens not updated", [(OF, "updated_count")], _updated_count_complement, PINS_GATE),
+    ("cached step: reuse refreshes the cache", [(OF.CachedBlockAttention, "step")], _step_refreshes_cache,
+     PINS_STEP),
+    ("similarity: reusing heads refresh their reference", [(OSim, "refresh_reference")], _refresh_reusing_heads,
+     PINS_SIM),
 ]
 
 
@@ -203,5 +284,5 @@ def test_pins_catch_planted_mistake(monkeypatch, name, targets, mutant, pins):
 
 
 def test_pins_pass_on_unmutated_oracle():
-    for pin in PINS_ATTN + PINS_GATE + PINS_SPARSE + PINS_TRANSITION + PINS_SIM + PINS_LOSA:
+    for pin in PINS_ATTN + PINS_GATE + PINS_STEP + PINS_SPARSE + PINS_TRANSITION + PINS_SIM + PINS_LOSA:
         pin()

@@ -144,3 +144,15 @@ def test_selected_part_is_attention_over_selected_pages():
             a, l = OA.attend(q[0, h, 1:2], f64(k)[0, g][keep[1]], f64(v)[0, g][keep[1]], W.default_scale(16))
             np.testing.assert_allclose(r.a_sel[0, h, 1], a[0], rtol=0, atol=1e-12)
         break
+
+
+def test_page_minmax_partial_page_ignores_missing_rows():
+    # the last page holds 5 real rows; rows past the prefix must not enter its bounds
+    rng = np.random.default_rng(4)
+    pos = 1.0 + np.abs(rng.standard_normal((37, 6)))
+    kmin, kmax = OS.page_minmax(pos, 16)
+    np.testing.assert_array_equal(kmin[2], pos[32:].min(0))
+    assert (kmin >= 1.0).all()
+    kmin, kmax = OS.page_minmax(-pos, 16)
+    np.testing.assert_array_equal(kmax[2], (-pos)[32:].max(0))
+    assert (kmax <= -1.0).all()
