@@ -771,11 +771,25 @@ def oracle_steps(w: W.Workload, seed: int, budget_s: float, max_steps: int, kv_g
     return n, el, w.h_kv / hk
 
 
-def cpu_baseline(w, seed, budget_s=12.0):
+def cpu_baseline(w, seed, budget_s=12.0, one_thread_budget_s=4.0):
+    """The float64 oracle on the host cores (all BLAS threads), plus the same sample
+    with the BLAS pools held to one thread (`one_thread`)."""
     n, el, scale = oracle_steps(w, seed, budget_s, 10 ** 6, kv_groups=1)
-    return dict(value=n / (el * scale), unit="steps/s", cores=blas_threads(), kind="oracle",
-                sample=f"{n} steps of the seeded schedule through the float64 oracle, 1 of {w.h_kv} KV-head "
-                       f"groups ({w.group} query heads) at full prefix length; time x{scale:g} = whole layer")
+    out = dict(value=n / (el * scale), unit="steps/s", cores=blas_threads(), kind="oracle",
+               sample=f"{n} steps of the seeded schedule through the float64 oracle, 1 of {w.h_kv} KV-head "
+                      f"groups ({w.group} query heads) at full prefix length; time x{scale:g} = whole layer")
+    one = None
+    if one_thread_budget_s > 0:
+        try:
+            from threadpoolctl import threadpool_limits
+        except ImportError:
+            threadpool_limits = None
+        if threadpool_limits is not None:
+            with threadpool_limits(limits=1):
+                n1, el1, scale1 = oracle_steps(w, seed, one_thread_budget_s, 10 ** 6, kv_groups=1)
+            one = dict(value=n1 / (el1 * scale1), unit="steps/s", cores=1, sample=f"{n1} steps, same sample")
+    out["one_thread"] = one
+    return out
 
 
 def reference_arm(args):

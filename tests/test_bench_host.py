@@ -39,3 +39,11 @@ def test_committed_traffic_is_near_the_algorithmic_bytes(name):
         pytest.skip("profile taken on other sources")
     alg = bench.step_bytes(W.get(name))[0]
     assert 1.0 <= t / alg < 1.05
+
+
+def test_cpu_baseline_reports_all_cores_and_one_thread():
+    r = bench.cpu_baseline(W.get("tiny_f32"), 0, budget_s=0.3, one_thread_budget_s=0.3)
+    assert r["kind"] == "oracle" and r["unit"] == "steps/s" and r["value"] > 0 and r["cores"] >= 1
+    assert "KV-head" in r["sample"]
+    one = r["one_thread"]
+    assert one is not None and one["cores"] == 1 and one["value"] > 0
