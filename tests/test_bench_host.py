@@ -47,3 +47,11 @@ def test_cpu_baseline_reports_all_cores_and_one_thread():
     assert "KV-head" in r["sample"]
     one = r["one_thread"]
     assert one is not None and one["cores"] == 1 and one["value"] > 0
+
+
+def test_tensor_roofline_uses_the_burst_peak():
+    r = bench.tensor_roofline(706.0)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["peak"] > 0 and r["frac"] == pytest.approx(706.0 / r["peak"])
+    assert r["frac_of_sustained"] >= r["frac"]        # the sustained figure is the lower one
+    assert "burst" in r["peak_source"]
