@@ -35,7 +35,6 @@ from __future__ import annotations
 import dataclasses
 import math
 from fractions import Fraction
-from typing import Optional
 
 import numpy as np
 

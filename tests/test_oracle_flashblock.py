@@ -4,7 +4,6 @@ import json
 import os
 
 import numpy as np
-import pytest
 
 from block_diffusion_attention_prefix_b200 import workloads as W
 from oracle import attention as OA

@@ -9,7 +9,6 @@ own selections (subset of the union over all rows)."""
 import math
 
 import numpy as np
-import pytest
 
 from block_diffusion_attention_prefix_b200 import workloads as W
 from oracle import flashblock as OF

@@ -12,7 +12,6 @@ import pytest
 import torch
 
 from block_diffusion_attention_prefix_b200 import workloads as W
-from oracle import attention as OA
 from oracle import flashblock as OF
 from oracle import sparse as OS
 
