@@ -134,3 +134,14 @@ def test_page_cap_is_the_pages_of_the_cache_capacity(lib, n, cap, want):
 def test_page_cap_rejects_other_page_sizes(lib):
     assert lib.fb_page_cap(ctypes.byref(S()), 8) == -8      # FB_ERR_ARG
     assert lib.fb_page_cap(ctypes.byref(S(n_prefix=0)), 16) == -7  # FB_ERR_UNSUPPORTED
+
+
+def test_sparse_and_similarity_workspace_queries(lib):
+    sh = S(h_q=32, h_kv=8, n_prefix=65536)
+    n = fb.fb_sparse_workspace_bytes(sh, 16)
+    assert (1 << 20) < n < (64 << 20)                      # partials, in-block slot, f64 estimates
+    assert fb.fb_sparse_workspace_bytes(S(h_q=32, h_kv=8, n_prefix=2 * 65536), 16) > n   # estimates grow with N
+    assert fb.fb_sparse_workspace_bytes(sh, 8) == 0         # page size 16 only
+    assert fb.fb_sparse_workspace_bytes(S(dtype=9), 16) == 0
+    assert fb.fb_similarity_workspace_bytes(S(h_q=12, h_kv=12, block=4680)) > 0
+    assert fb.fb_similarity_workspace_bytes(S(batch=0)) == 0
