@@ -168,3 +168,26 @@ def test_attend_masked_rows():
         np.testing.assert_array_equal(A[r], a[0])
         np.testing.assert_array_equal(L[r], l[0])
     assert np.all(A[2] == 0) and np.isneginf(L[2])
+
+
+def test_key_order_does_not_matter():
+    # permuting the keys together with their values leaves (A, L) unchanged
+    rng = np.random.default_rng(11)
+    q, k, v = rand_qkv(rng, 5, 41, 16)
+    perm = rng.permutation(41)
+    A, L = OA.attend(q, k, v, 0.25)
+    Ap, Lp = OA.attend(q, k[perm], v[perm], 0.25)
+    np.testing.assert_allclose(Ap, A, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(Lp, L, rtol=0, atol=1e-12)
+
+
+def test_common_score_shift_moves_L_only():
+    # adding u to every key adds scale * q.u to every score of the row: the weights,
+    # hence A, are unchanged and L moves by exactly that amount
+    rng = np.random.default_rng(12)
+    q, k, v = rand_qkv(rng, 4, 29, 8)
+    u = rng.standard_normal(8)
+    A, L = OA.attend(q, k, v, 0.5)
+    As, Ls = OA.attend(q, k + u, v, 0.5)
+    np.testing.assert_allclose(As, A, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(Ls, L + 0.5 * (q @ u), rtol=0, atol=1e-12)

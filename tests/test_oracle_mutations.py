@@ -65,6 +65,12 @@ def _attend_L_no_max(q, k, v, scale):
     return A, np.log(np.exp(s - s.max(1, keepdims=True)).sum(1))
 
 
+def _attend_values_rolled(q, k, v, scale):
+    # each key paired with the next key's value
+    v = np.asarray(v)
+    return _orig_attend(q, k, np.roll(v, 1, axis=0) if v.shape[0] > 1 else v, scale)
+
+
 def _tau_le(M, tau, first_step):
     return np.zeros(M.shape, bool) if first_step else M <= tau
 
@@ -206,6 +212,8 @@ def _refresh_reusing_heads(q, q_ref, reuse):
 
 PINS_ATTN = [
     lambda: TA.test_attend_matches_torch_sdpa_and_logsumexp(3, 7, 16, 0.25),
+    lambda: TA.test_key_order_does_not_matter(),
+    lambda: TA.test_common_score_shift_moves_L_only(),
     lambda: TA.test_golden_attention_cases(),
     lambda: TA.test_golden_merge_cases(),
     lambda: TA.test_merge_of_partition_equals_dense_over_union(0),
@@ -243,6 +251,8 @@ MUTANTS = [
     ("merge: exponent sign flipped", [(OA, "merge"), (OF, "merge"), (OS, "merge")], _merge_sign, PINS_ATTN),
     ("attend: softmax scale dropped", [(OA, "attend"), (OF, "attend"), (OS, "attend")], _attend_no_scale, PINS_ATTN),
     ("attend: K used in place of V", [(OA, "attend"), (OF, "attend"), (OS, "attend")], _attend_kv_swapped, PINS_ATTN),
+    ("attend: values paired with the wrong keys", [(OA, "attend"), (OF, "attend"), (OS, "attend")],
+     _attend_values_rolled, PINS_ATTN),
     ("attend: L drops the max term", [(OA, "attend"), (OF, "attend"), (OS, "attend")], _attend_L_no_max, PINS_ATTN),
     ("tau gate: <= instead of <", [(OF, "tau_reuse")], _tau_le, PINS_GATE),
     ("gamma gate: >= instead of >", [(OF, "gamma_reuse")], _gamma_ge, PINS_GATE),
