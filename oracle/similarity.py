@@ -13,14 +13,13 @@ Readings where the pages are silent:
       B x D, flattened) and the queries its cached A_out was computed with (its
       queries at its last recompute): a cached row is stale exactly as far as its
       query has moved.
-  S2  the sums run in one fixed order, so that every implementation produces the
+  S2  the sums run in one plain order, so that every implementation produces the
       same bits and the gate decision (sim > gamma, in float32) is reproducible:
-      each row's products are summed in ascending d (float64; the products of
-      float32 or bfloat16 inputs are exact in float64); the rows are taken in
-      chunks of 256 consecutive rows, and the 256 row sums of a chunk (rows past B
-      count as zero) are added as a pairwise tree (neighbours first); the chunk
-      totals are added in ascending chunk order.  Three such sums are formed:
-      <Q, R>, <Q, Q>, <R, R>.
+      each row's products are summed in ascending d, starting from 0 (float64;
+      the products of float32 or bfloat16 inputs are exact in float64, so every
+      term costs one rounding), which gives the row's dot product; the row dot
+      products are then added one after another in ascending row order, starting
+      from 0.  Three such sums are formed: <Q, R>, <Q, Q>, <R, R>.
   S3  sim = <Q, R> / sqrt(<Q, Q> <R, R>) in float64, then rounded to float32; a
       zero norm gives sim = 0 (no evidence of similarity: recompute).
   S4  after a step, the reference queries of the heads that recomputed become
@@ -30,20 +29,13 @@ from __future__ import annotations
 
 import numpy as np
 
-CHUNK = 256
-
 
 def _ordered_sum(row_terms: np.ndarray) -> float:
-    """Sum of per-row values [B] in the order of reading S2 (chunks of 256 rows,
-    pairwise tree inside a chunk, chunks in ascending order)."""
-    B = row_terms.shape[0]
+    """Sum of the per-row values [B] in the order of reading S2: one after another,
+    in ascending row order, starting from 0."""
     total = 0.0
-    for c0 in range(0, B, CHUNK):
-        x = np.zeros(CHUNK)
-        x[:min(CHUNK, B - c0)] = row_terms[c0:c0 + CHUNK]
-        while x.shape[0] > 1:
-            x = x[0::2] + x[1::2]
-        total = total + x[0]
+    for x in np.asarray(row_terms, np.float64).tolist():
+        total = total + x
     return float(total)
 
 

@@ -118,12 +118,20 @@ def _append_block_first(k_cache, v_cache, k_blk, v_blk):
 _orig_ordered_sum = OSim._ordered_sum
 
 
-def _sum_sequential(row_terms):
-    # rows added one after another instead of the pairwise tree
-    total = 0.0
-    for x in np.asarray(row_terms, np.float64):
-        total = total + x
-    return float(total)
+def _sum_pairwise(row_terms):
+    # rows added as a pairwise tree (neighbours first) instead of one after another
+    x = list(np.asarray(row_terms, np.float64))
+    while len(x) > 1:
+        x = [x[i] + x[i + 1] if i + 1 < len(x) else x[i] for i in range(0, len(x), 2)]
+    return float(x[0]) if x else 0.0
+
+
+_orig_row_dots = OSim._row_dots
+
+
+def _row_dots_descending(a, b):
+    # channels added from the last to the first
+    return _orig_row_dots(np.asarray(a)[:, ::-1], np.asarray(b)[:, ::-1])
 
 
 def _sim_no_sqrt(q, q_ref):
@@ -238,7 +246,9 @@ PINS_TRANSITION = [lambda: TT.test_incremental_page_bounds_equal_recomputed(17, 
 
 PINS_SIM = [lambda: TSim.test_matches_library_cosine(300),
             lambda: TSim.test_closed_forms(),
-            lambda: TSim.test_pairwise_tree_order_inside_a_chunk(),
+            lambda: TSim.test_rows_added_in_ascending_order(),
+            lambda: TSim.test_channels_added_in_ascending_order(),
+            lambda: TSim.test_sum_error_within_the_sequential_bound(),
             lambda: TSim.test_refresh_reference_takes_recomputing_heads()]
 
 PINS_LOSA = [lambda: TL.test_token_mse_matches_library_mean(),
@@ -261,7 +271,8 @@ MUTANTS = [
     ("transition: partial page left stale", [(OT, "update_page_minmax")], _update_skips_partial_page,
      PINS_TRANSITION),
     ("transition: block before the prefix", [(OT, "append_block")], _append_block_first, PINS_TRANSITION),
-    ("similarity: rows summed in sequence", [(OSim, "_ordered_sum")], _sum_sequential, PINS_SIM),
+    ("similarity: rows summed as a pairwise tree", [(OSim, "_ordered_sum")], _sum_pairwise, PINS_SIM),
+    ("similarity: channels summed in descending order", [(OSim, "_row_dots")], _row_dots_descending, PINS_SIM),
     ("similarity: norm without the square root", [(OSim, "head_similarity")], _sim_no_sqrt, PINS_SIM),
     ("LoSA: score summed, not averaged", [(OL, "token_mse")], _mse_no_mean, PINS_LOSA),
     ("LoSA: union over every row", [(OL, "union_bitmap")], _union_with_stable_rows, PINS_LOSA),

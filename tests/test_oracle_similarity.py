@@ -1,8 +1,9 @@
 """Pins of oracle.similarity (CPU only): the per-head similarity estimate.
 
 Pinned by the library (torch float64 cosine similarity of the flattened blocks),
-exact summation (math.fsum), and closed forms (identical, negated, scaled and
-orthogonal blocks; a zero block)."""
+exact summation (math.fsum) within the error bound of recursive summation,
+hand-derived values that only the stated summation order gives, and closed forms
+(identical, negated, scaled and orthogonal blocks; a zero block)."""
 import math
 
 import numpy as np
@@ -48,14 +49,32 @@ def test_closed_forms():
     assert np.all(OSim.head_similarity(q, np.zeros_like(q)) == 0.0)
 
 
-def test_pairwise_tree_order_inside_a_chunk():
-    # 4 rows: ((a + b) + (c + d)), not ((a + b) + c) + d -- the two differ here
-    rows = np.zeros(300)
-    rows[:4] = [1.0, 1e-16, -1.0, 1e-16]
-    tree = (1.0 + 1e-16) + (-1.0 + 1e-16)
-    seq = ((1.0 + 1e-16) + -1.0) + 1e-16
-    assert tree != seq
-    assert OSim._ordered_sum(rows) == tree
+def test_rows_added_in_ascending_order():
+    # one channel, four rows whose products are 1, 1e-16, -1, 1e-16.  Added one
+    # after another from 0: 1 + 1e-16 rounds to 1, minus 1 gives 0, plus 1e-16
+    # gives 1e-16.  (The exact sum is 2e-16; a pairwise tree gives 2^-53, the
+    # reverse order 2^-52.)  <Q,Q> = 2 and <R,R> = 4 exactly, so
+    # sim = 1e-16 / sqrt(8) rounded to float32.
+    q = np.array([1.0, 1e-16, -1.0, 1e-16]).reshape(1, 1, 4, 1)
+    r = np.ones_like(q)
+    assert OSim.head_similarity(q, r)[0, 0] == np.float32(1e-16 / math.sqrt(8.0))
+
+
+def test_channels_added_in_ascending_order():
+    # the same four products along d of one row: ascending d gives 1e-16 again
+    q = np.array([1.0, 1e-16, -1.0, 1e-16]).reshape(1, 1, 1, 4)
+    r = np.ones_like(q)
+    assert OSim.head_similarity(q, r)[0, 0] == np.float32(1e-16 / math.sqrt(8.0))
+
+
+def test_sum_error_within_the_sequential_bound():
+    # recursive summation of n terms: |error| <= (n - 1) u sum|x_i| (u = 2^-53),
+    # against the exact sum (math.fsum is correctly rounded)
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal(5000) * np.exp(rng.uniform(-20, 20, 5000))
+    exact = math.fsum(x.tolist())
+    bound = (len(x) - 1) * 2.0 ** -53 * np.abs(x).sum()
+    assert abs(OSim._ordered_sum(x) - exact) <= bound
 
 
 def test_refresh_reference_takes_recomputing_heads():
