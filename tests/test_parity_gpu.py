@@ -4,8 +4,9 @@ Integer outputs (M^{s+1}, reuse decisions) must match bit for bit.  Floating
 outputs must be within max-abs 1e-5 for fp32 workloads and 2e-2 for bf16
 workloads (fp32 accumulation), the tolerances the FlashBlock build targets.
 Sizes span several key tiles (64 keys for bf16, 32 for fp32), several splits
-and ragged tails; the full-size workloads are checked on every row where the
-oracle is fast enough and on sampled rows otherwise.
+and ragged tails.  The dLM-like workloads run at full size on every row here;
+the long-context and video workloads at full size are in
+test_parity_fullsize_gpu.py.
 """
 import math
 
@@ -286,63 +287,6 @@ def test_step_is_deterministic(fb):
         outs.append((layer.a_full.clone(), layer.a_out.clone(), layer.l_out.clone()))
     for x, y in zip(*outs):
         assert torch.equal(x, y)
-
-
-# --------------------------------------------------------------------------- full-size, sampled rows
-
-
-def sampled_prefix_check(fb, w, seed, heads, rows):
-    """Recompute step of workload w at full size; check (A_out, L_out) on sampled rows."""
-    k, v = W.prefix_kv(w, seed)
-    s = next(iter(W.block_schedule(w, seed, 1)))
-    sh = fb.make_shape(w.batch, w.h_q, w.h_kv, w.head_dim, w.block, w.n_prefix, w.dtype)
-    a, l = alloc_pass_outputs(w.batch, w.h_q, w.block, w.head_dim)
-    ws = workspace(fb, sh)
-    gate = fb.make_gate(s.mask.cuda(), True, w.tau)
-    fb.fb_prefix_attn(sh, s.q.cuda(), k.cuda(), v.cuda(), gate, a, l, ws)
-    torch.cuda.synchronize()
-    assert fb.fb_device_error() == 0
-    q = f64(s.q)
-    for h in heads:
-        g = h // w.group
-        kh, vh = f64(k[0, g]), f64(v[0, g])
-        A, L = OA.attend(q[0, h, rows], kh, vh, 1 / math.sqrt(w.head_dim))
-        close(f64(a[0, h, rows]), A, 2e-2, f"A_out h={h}")
-        close(f64(l[0, h, rows]), L, 2e-2, f"L_out h={h}")
-
-
-@pytest.mark.parametrize("name", ["long_100k", "long_800k"])
-def test_long_context_full_size_sampled(fb, name):
-    sampled_prefix_check(fb, W.get(name), seed=2, heads=[0, 13, 31], rows=[0, 3])
-
-
-def test_video_gamma_full_size_sampled(fb):
-    """Video workload at full size: 12 heads, 4680 block queries over a 31200-token
-    prefix and the 4680 block keys; the gamma gate picks the heads that reuse."""
-    w = W.get("video")
-    k, v = W.prefix_kv(w, 4)
-    kd, vd = k.cuda(), v.cuda()
-    layer = fb.CachedAttentionLayer(1, w.h_q, w.h_kv, w.head_dim, w.block, kd, vd)
-    rows = np.array([0, 1, 1559, 2345, 4679])
-    scale = 1 / math.sqrt(w.head_dim)
-    cache = {}
-    for s in W.block_schedule(w, 4):
-        layer.step(s.q.cuda(), s.k_blk.cuda(), s.v_blk.cuda(), s.mask.cuda(), s.first, w.tau, s.sim.cuda(),
-                   w.gamma)
-        torch.cuda.synchronize()
-        M, reuse = OF.decisions(s.mask.numpy(), s.first, w.tau, s.sim.numpy(), w.gamma, w.h_q)
-        assert np.array_equal(layer.dec_M.cpu().numpy(), M)
-        assert np.array_equal(layer.dec_reuse.cpu().numpy().astype(bool), reuse)
-        q = f64(s.q)
-        for h in range(w.h_q):
-            if not reuse[0, h]:
-                cache[h] = OA.attend(q[0, h, rows], f64(k[0, h]), f64(v[0, h]), scale)
-            ai, li = OA.attend(q[0, h, rows], f64(s.k_blk[0, h]), f64(s.v_blk[0, h]), scale)
-            A, L = OA.merge(cache[h][0], cache[h][1], ai, li)
-            close(f64(layer.a_full[0, h, rows]), A, 2e-2, f"step {s.index} head {h} A_full")
-            close(f64(layer.l_full[0, h, rows]), L, 2e-2, f"step {s.index} head {h} L_full")
-            close(f64(layer.a_out[0, h, rows]), cache[h][0], 2e-2, f"step {s.index} head {h} A_out")
-    assert fb.fb_device_error() == 0
 
 
 # --------------------------------------------------------------------------- fused step
