@@ -229,10 +229,10 @@ def step_bytes(w: W.Workload, batch: Optional[int] = None):
 class DeviceWorkload:
     """The workload's inputs resident in HBM and the layer state, stepped through libfb."""
 
-    def __init__(self, fb, w: W.Workload, seed: int):
+    def __init__(self, fb, w: W.Workload, seed: int, kv=None):
         self.fb, self.w = fb, w
         dev = torch.device("cuda")
-        k, v = W.prefix_kv(w, seed)
+        k, v = W.prefix_kv(w, seed) if kv is None else kv
         self.k, self.v = k.to(dev), v.to(dev)
         del k, v
         self.sched = []
@@ -400,11 +400,14 @@ def batched_reuse(fb, w: W.Workload, flush, reps: int = 20, n_prefix: int = 64,
     return out
 
 
-def device_arm(args, rank, world):
+def device_arm(args, rank, world, w: Optional[W.Workload] = None, kv=None, extras: bool = True):
+    """One workload through libfb on this rank's GPU.  `kv`: the prefix K/V already
+    drawn on the host (else drawn here); `extras`: also measure the batched reuse
+    view (independent of the prefix length)."""
     from block_diffusion_attention_prefix_b200 import fb
     fb.load()
-    w = W.get(args.workload)
-    dw = DeviceWorkload(fb, w, seed=replica_seed(args.seed, rank))
+    w = W.get(args.workload) if w is None else w
+    dw = DeviceWorkload(fb, w, seed=replica_seed(args.seed, rank), kv=kv)
     K, Wm = args.steps, args.warmup
     dev = torch.device("cuda")
     flush = L2Flush(dev)
@@ -489,7 +492,7 @@ def device_arm(args, rank, world):
                     union_density_active_rows=statistics.mean(pos_union.values()),
                     losa_step_us=_mean_us(step_ms, reuse_steps), dense_first_step_us=_mean_us(step_ms,
                                                                                              recompute_steps))
-    traffic = ncu_traffic(args.workload)
+    traffic = ncu_traffic(w.name)
     tensor = None
     if w.block > 64:
         # Large blocks (video): the passes are dense contractions.  FLOPs of a step =
@@ -571,7 +574,16 @@ def device_arm(args, rank, world):
         sim_us = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
         sim_gbs = 2 * qa.numel() * qa.element_size() / (sim_us * 1e-6) / 1e9
 
-    reuse_batched = batched_reuse(fb, w, flush)
+    reuse_batched = batched_reuse(fb, w, flush) if extras else None
+    reuse_ms = [step_ms[i] for i in reuse_steps]
+    roofline_reuse = None
+    if reuse_ms and not dw.losa:
+        gbs = alg_reuse * len(reuse_ms) / (sum(reuse_ms) / 1e3) / 1e9
+        roofline_reuse = dict(bound="launch", achieved=gbs, peak=hbm, unit="GB/s", frac=gbs / hbm,
+                              alg_bytes_per_launch=alg_reuse, launches=len(reuse_ms),
+                              avg_launch_us=sum(reuse_ms) / len(reuse_ms) * 1e3, launch_floor_us=floor_us,
+                              note="a single reuse step reads no prefix K/V (Q, block K/V, cache, output only): "
+                                   "launch bound; breakdown.reuse_batched is its HBM-bound view")
     e2e = e2e_arm(fb, dw, K, Wm) if (args.e2e and dw.sparse_layer is None) else None
     res = dict(
         metric=METRIC, value=value, unit="steps/s", n_gpus=world, steps=K, warmup=Wm,
@@ -603,6 +615,7 @@ def device_arm(args, rank, world):
                        recompute_step_us=_mean_us(step_ms, recompute_steps),
                        reuse_step_us=_mean_us(step_ms, reuse_steps),
                        reuse_step_alg_bytes=alg_reuse,
+                       roofline_reuse=roofline_reuse,
                        reuse_batched=reuse_batched,
                        launch_floor_us=floor_us,
                        block_transition_us=trans_us,
@@ -726,7 +739,12 @@ def e2e_arm(fb, dw, K, Wm):
         one(Wm + i)
     torch.cuda.synchronize()  # every step's result is on the host
     el = time.perf_counter() - t0
+    kv_bytes = w.prefix_bytes()
     return dict(value=K / el, unit="steps/s", h2d_bytes_per_step=in_bytes, d2h_bytes_per_step=out_bytes,
+                l2=f"not flushed between steps (wall clock of back-to-back steps); the prefix K/V hold "
+                   f"{kv_bytes / 1e6:.0f} MB against a 126 MB L2" + (", so recompute steps stream them from HBM"
+                                                                       if kv_bytes > 4 * (126 << 20) else
+                                                                       ", so part of them can stay resident"),
                 note="wall clock per step incl. one pinned H2D copy of the step's packed inputs, fb_step, one "
                      "D2H copy of A_full + decisions; the host runs one step ahead (waits for step i's result "
                      "before reusing its output buffer at step i+2); prefix KV cache resident in HBM")
@@ -744,13 +762,14 @@ def blas_threads() -> int:
         return 1
 
 
-def oracle_steps(w: W.Workload, seed: int, budget_s: float, max_steps: int, kv_groups: int):
+def oracle_steps(w: W.Workload, seed: int, budget_s: float, max_steps: int, kv_groups: int, kv=None):
     """Time the CPU oracle's cached step on the workload, restricted to the first
     `kv_groups` KV-head groups (a bounded sample).  Returns (steps, seconds,
-    scale) where scale converts the sample's time to a whole-layer step."""
+    scale) where scale converts the sample's time to a whole-layer step.  `kv`:
+    the prefix K/V already drawn (else drawn here)."""
     from oracle import flashblock as OF
     from oracle import sparse as OS
-    k, v = W.prefix_kv(w, seed)
+    k, v = W.prefix_kv(w, seed) if kv is None else kv
     hk = min(kv_groups, w.h_kv)
     hq = hk * w.group
     kk = k[:, :hk].double().numpy()
@@ -785,10 +804,10 @@ def oracle_steps(w: W.Workload, seed: int, budget_s: float, max_steps: int, kv_g
     return n, el, w.h_kv / hk
 
 
-def cpu_baseline(w, seed, budget_s=12.0, one_thread_budget_s=4.0):
+def cpu_baseline(w, seed, budget_s=12.0, one_thread_budget_s=4.0, kv=None):
     """The float64 oracle on the host cores (all BLAS threads), plus the same sample
     with the BLAS pools held to one thread (`one_thread`)."""
-    n, el, scale = oracle_steps(w, seed, budget_s, 10 ** 6, kv_groups=1)
+    n, el, scale = oracle_steps(w, seed, budget_s, 10 ** 6, kv_groups=1, kv=kv)
     out = dict(value=n / (el * scale), unit="steps/s", cores=blas_threads(), kind="oracle",
                sample=f"{n} steps of the seeded schedule through the float64 oracle, 1 of {w.h_kv} KV-head "
                       f"groups ({w.group} query heads) at full prefix length; time x{scale:g} = whole layer")
@@ -800,16 +819,17 @@ def cpu_baseline(w, seed, budget_s=12.0, one_thread_budget_s=4.0):
             threadpool_limits = None
         if threadpool_limits is not None:
             with threadpool_limits(limits=1):
-                n1, el1, scale1 = oracle_steps(w, seed, one_thread_budget_s, 10 ** 6, kv_groups=1)
+                n1, el1, scale1 = oracle_steps(w, seed, one_thread_budget_s, 10 ** 6, kv_groups=1, kv=kv)
             one = dict(value=n1 / (el1 * scale1), unit="steps/s", cores=1, sample=f"{n1} steps, same sample")
     out["one_thread"] = one
     return out
 
 
 def reference_arm(args):
-    w = W.get(args.workload)
-    _, _, _ = oracle_steps(w, args.seed, 0.0, max(1, min(args.warmup, 16)), kv_groups=1)
-    n, el, scale = oracle_steps(w, args.seed, 1e9, args.steps, kv_groups=1)
+    w = W.get(SWEEP[-1] if args.workload == "long_sweep" else args.workload)
+    kv = W.prefix_kv(w, args.seed)
+    _, _, _ = oracle_steps(w, args.seed, 0.0, max(1, min(args.warmup, 16)), kv_groups=1, kv=kv)
+    n, el, scale = oracle_steps(w, args.seed, 1e9, args.steps, kv_groups=1, kv=kv)
     value = n / (el * scale)
     return dict(metric=METRIC, value=value, unit="steps/s", n_gpus=args.gpus, steps=n, warmup=args.warmup,
                 ms_per_step=el * scale / n * 1e3, higher_is_better=True, scaling="weak", vs_baseline=None,
@@ -823,23 +843,161 @@ def reference_arm(args):
                 e2e=dict(value=value, unit="steps/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
 
 
+# ----------------------------------------------------------------------------- context-length sweep
+
+# The metric is taken against context length: the long-context workloads at 100k,
+# 200k, 400k and 800k prefix tokens, the top-level figures at the largest; the
+# dLM-8B-like 32k layer rides along as a secondary record.
+SWEEP = ("long_100k", "long_200k", "long_400k", "long_800k")
+SWEEP_SECONDARY = ("dlm8b_b4",)
+
+
+def sweep_entry(r: dict) -> dict:
+    """The per-length summary of one workload's record."""
+    bd, rf = r["breakdown"], r["roofline"]
+    cb = r.get("cpu_baseline")
+    return dict(
+        workload=r["config"]["workload"], n_prefix=r["config"]["n_prefix"], steps_per_s=r["value"],
+        ms_per_step=r["ms_per_step"], steps=r["steps"],
+        roofline=dict(achieved=rf["achieved"], peak=rf["peak"], unit=rf["unit"], frac=rf["frac"],
+                      frac_of_8tbs=rf.get("frac_of_8tbs"), alg_bytes_per_launch=rf["alg_bytes_per_launch"],
+                      launches=rf["launches"], avg_launch_us=rf["avg_launch_us"], traffic=rf.get("traffic")),
+        roofline_reuse=bd.get("roofline_reuse"),
+        recompute_steps=bd["recompute_steps"], reuse_steps=bd["reuse_steps"],
+        recompute_step_us=bd["recompute_step_us"], reuse_step_us=bd["reuse_step_us"],
+        dense_recompute_step_us=bd["dense_recompute_step_us"], dense_steps_per_s=bd["dense_steps_per_s"],
+        e2e_steps_per_s=(r.get("e2e") or {}).get("value"),
+        cpu_baseline=None if cb is None else dict(value=cb["value"], unit=cb["unit"], cores=cb["cores"],
+                                                  sample=cb["sample"]),
+        clocks=r.get("clocks"))
+
+
+def sweep_arm(args, rank, world):
+    """Every sweep length (and the secondary workloads) through device_arm; the
+    top-level record is the largest length's, with one summary per length."""
+    recs = {}
+    for name in SWEEP + SWEEP_SECONDARY:
+        w = W.get(name)
+        kv = W.prefix_kv(w, replica_seed(args.seed, rank))
+        r = device_arm(args, rank, world, w=w, kv=kv, extras=(name == SWEEP[-1]))
+        if rank == 0 and world == 1 and args.cpu_baseline:
+            r["cpu_baseline"] = cpu_baseline(w, args.seed, budget_s=5.0, one_thread_budget_s=2.0, kv=kv)
+        del kv
+        torch.cuda.empty_cache()
+        recs[name] = r
+    res = recs[SWEEP[-1]]
+    res["config"]["sweep"] = list(SWEEP)
+    res["sweep"] = [sweep_entry(recs[n]) for n in SWEEP]
+    res["secondary"] = {n: sweep_entry(recs[n]) for n in SWEEP_SECONDARY}
+    return res
+
+
+# ----------------------------------------------------------------------------- context-parallel arm
+
+
+def context_arm(args, rank, world):
+    """--split context: the workload's prefix cut into `world` key ranges, one per
+    rank (block_diffusion_attention_prefix_b200.context_parallel): every step each
+    rank computes its range's partial, one all-gather exchanges the partials, and
+    every rank merges them and finishes the step.  The whole job is one layer, so
+    this is strong scaling: value = steps of the layer per second, timed as the
+    slowest rank's summed step events."""
+    from block_diffusion_attention_prefix_b200 import fb
+    from block_diffusion_attention_prefix_b200.context_parallel import ContextParallelLayer, shard_range
+    fb.load()
+    w = W.get(SWEEP[-1] if args.workload == "long_sweep" else args.workload)
+    if w.block > 64 or w.page_size or w.losa_delta is not None:
+        raise SystemExit(f"--split context takes the dense small-block workloads, not {w.name}")
+    dev = torch.device("cuda")
+    n0, n1 = shard_range(w.n_prefix, world, rank)
+    # this rank's range of the prefix, drawn on the device (seeded per rank); the
+    # block's inputs are the same on every rank
+    g = torch.Generator(device=dev).manual_seed(args.seed * 1_000_003 + rank)
+    c = (0.5 * (0.5 + 1.5 * torch.rand(w.h_kv, generator=g, device=dev))).view(1, w.h_kv, 1, 1)
+    shape = (w.batch, w.h_kv, n1 - n0, w.head_dim)
+    k = (torch.randn(shape, generator=g, device=dev) * c).to(w.torch_dtype)
+    v = (torch.randn(shape, generator=g, device=dev) * c).to(w.torch_dtype)
+    sched = [dict(q=s.q.to(dev), k_blk=s.k_blk.to(dev), v_blk=s.v_blk.to(dev), mask=s.mask.to(dev), first=s.first)
+             for s in W.block_schedule(w, args.seed)]
+    layer = ContextParallelLayer(fb, w.batch, w.h_q, w.h_kv, w.head_dim, w.block, w.n_prefix, k, v, rank, world)
+    flush = L2Flush(dev)
+    K, Wm, npos = args.steps, args.warmup, len(sched)
+
+    def one(i):
+        s = sched[i % npos]
+        layer.step(s["q"], s["k_blk"], s["v_blk"], s["mask"], s["first"], w.tau)
+
+    for i in range(Wm):
+        flush()
+        one(i)
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    reuse = []
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        for i in range(K):
+            flush()
+            evs[i][0].record()
+            one(Wm + i)
+            evs[i][1].record()
+            reuse.append(layer.dec_reuse.clone())
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    t_max = max_over_ranks(sum(step_ms), world, dev)
+    rec = [i for i in range(K) if not bool(reuse[i].bool().all())]
+    re_ = [i for i in range(K) if bool(reuse[i].bool().all())]
+    hbm, peak_kind = peaks()
+    shard_bytes = 2 * w.batch * w.h_kv * (n1 - n0) * w.head_dim * w.elem_bytes
+    rec_us = _mean_us(step_ms, rec)
+    achieved = shard_bytes / (rec_us * 1e-6) / 1e9 if rec_us else None
+    exch = world * layer.flat * 4
+    return dict(
+        metric=METRIC, value=K / (t_max / 1e3), unit="steps/s", n_gpus=world, steps=K, warmup=Wm,
+        ms_per_step=t_max / K, higher_is_better=True, scaling="strong", vs_baseline=None, dtype=w.dtype,
+        data="synthetic",
+        config=dict(workload=w.name, description=w.description, batch=w.batch, h_q=w.h_q, h_kv=w.h_kv,
+                    head_dim=w.head_dim, block=w.block, n_prefix=w.n_prefix, tau=w.tau, seed=args.seed,
+                    l2="flushed between timed steps, outside the step events",
+                    parallelism=f"context x{world} (prefix key ranges of {n1 - n0} tokens on rank {rank})"),
+        roofline=dict(bound="hbm", kernel="rank's recompute step: prefix pass over its key range + all-gather of "
+                                          "the partials + merge + in-block", achieved=achieved, peak=hbm, unit="GB/s",
+                      frac=achieved / hbm if achieved else None, peak_source=f"{peak_kind} copy bandwidth",
+                      alg_bytes_per_launch=shard_bytes, traffic=None),
+        breakdown=dict(recompute_steps=len(rec), reuse_steps=len(re_), recompute_step_us=rec_us,
+                       reuse_step_us=_mean_us(step_ms, re_), exchange_bytes_per_step=exch,
+                       note="every step runs the all-gather (the gate is evaluated on the device)"),
+        gpu_launches=3 * K, clocks=clocks.summary(), kernel_source_sha=kernel_source_hash())
+
+
 # ----------------------------------------------------------------------------- main
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps per workload (default 200 for the long-context workloads, else 2000)")
     ap.add_argument("--warmup", type=int, default=32)
-    ap.add_argument("--workload", default="dlm8b_b4", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--workload", default="long_sweep", choices=["long_sweep"] + sorted(W.WORKLOADS),
+                    help="long_sweep (default): the context-length sweep 100k/200k/400k/800k, top-level "
+                         "figures at 800k, dlm8b_b4 as a secondary record")
     ap.add_argument("--impl", default="fb", choices=["fb", "reference"])
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--dense-steps", type=int, default=64)
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--no-e2e", dest="e2e", action="store_false")
+    ap.add_argument("--split", default="replicas", choices=["replicas", "context"],
+                    help="replicas (default): one replica of the workload per rank (weak scaling); context: the "
+                         "prefix split over the ranks by key range (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.steps is None:
+        args.steps = 200 if args.workload == "long_sweep" or args.workload.startswith("long_") else 2000
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -855,9 +1013,14 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
-    res = device_arm(args, rank, world)
-    if rank == 0 and world == 1 and args.cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(W.get(args.workload), args.seed)
+    if args.split == "context":
+        res = context_arm(args, rank, world)
+    elif args.workload == "long_sweep":
+        res = sweep_arm(args, rank, world)
+    else:
+        res = device_arm(args, rank, world)
+        if rank == 0 and world == 1 and args.cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(W.get(args.workload), args.seed)
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
