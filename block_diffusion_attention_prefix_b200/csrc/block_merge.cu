@@ -9,6 +9,10 @@
 //    mechanism" merge equation and "Adaptive reuse strategies" gates.)
 //  * gate_kernel: the gate alone (M^{s+1} and the per-head decisions).
 //  * merge_kernel: the merge equation alone, elementwise, 16-byte vectors.
+//  * merge_parts_kernel: the context-parallel combine -- the prefix split into P
+//    key ranges (one per GPU), each range's partial (A, L), and the cache rows of
+//    the heads that recompute set to the merge of all P partials in range order
+//    (the merge equation over a partition of J_out).
 //  * append_block_kernel: the block transition -- once a block's last step is
 //    done its tokens belong to the prefix: their K/V rows are copied to the end
 //    of the prefix cache (the prefix J_out grows by B; FlashBlock technical
@@ -79,6 +83,47 @@ __global__ void merge_kernel(const Dims d, const float* a1, const float* l1, con
   }
 }
 
+// One CTA per (query head, b), a warp per row: the merge of the P partials of each
+// row in range order -- M = max_p L_p, e_p = e^{L_p - M}, den = sum_p e_p (in order),
+// A = (sum_p e_p A_p) / den, L = M + ln den -- written to the cache, for the heads
+// whose gate decision is "recompute" (all heads without a gate).  Rows of reusing
+// heads are left untouched.
+template <int DC>
+__global__ void __launch_bounds__(128) merge_parts_kernel(const Dims d, const GateParams g, const float* a_parts,
+                                                           long long a_stride, const float* l_parts,
+                                                           long long l_stride, int P, float* a_out, float* l_out) {
+  constexpr int D = 32 * DC;
+  __shared__ int s_red[32];
+  const int h = blockIdx.x, b = blockIdx.y;
+  if (g.enabled) {
+    const int M = block_updated_count(g.mask + (size_t)b * d.B, d.B, s_red);
+    if (head_reuse(g, tau_reuse(g, M), b, d.hq, h)) return;  // uniform over the CTA
+  }
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = warp; i < d.B; i += 4) {
+    const size_t grow = ((size_t)b * d.hq + h) * d.B + i;
+    float M = -CUDART_INF_F;
+    for (int p = 0; p < P; ++p) M = fmaxf(M, __ldg(l_parts + p * l_stride + grow));
+    float acc[DC], den = 0.f;
+#pragma unroll
+    for (int t = 0; t < DC; ++t) acc[t] = 0.f;
+    if (M != -CUDART_INF_F) {
+      for (int p = 0; p < P; ++p) {
+        const float e = expf(__ldg(l_parts + p * l_stride + grow) - M);
+        float a[DC];
+        load_vec<DC>(a_parts + p * a_stride + grow * D + lane * DC, a);
+        den += e;
+#pragma unroll
+        for (int t = 0; t < DC; ++t) acc[t] = fmaf(e, a[t], acc[t]);
+      }
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+    for (int t = 0; t < DC; ++t) a_out[grow * D + lane * DC + t] = acc[t] * inv;
+    if (lane == 0) l_out[grow] = den > 0.f ? M + logf(den) : -CUDART_INF_F;
+  }
+}
+
 // Block transition: CTA (chunk, b * H_kv) copies rows [64 chunk, 64 chunk + 64) of the
 // block's K and V into cache rows N + those (16-byte vectors; cache rows may be padded).
 constexpr int kAppendRows = 64;
@@ -131,6 +176,20 @@ cudaError_t launch_append_block(const Dims& d, void* k_cache, void* v_cache, con
   append_block_kernel<<<grid, 256, 0, s>>>(d, static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache),
                                                    static_cast<const uint8_t*>(k_blk),
                                                    static_cast<const uint8_t*>(v_blk), d.dtype == 1 ? 2 : 4);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_merge_parts(const Dims& d, const GateParams& g, const float* a_parts, long long a_stride,
+                               const float* l_parts, long long l_stride, int P, float* a_out, float* l_out,
+                               cudaStream_t s) {
+  const dim3 grid(d.hq, d.b);
+  switch (d.D / 32) {
+    case 1: merge_parts_kernel<1><<<grid, 128, 0, s>>>(d, g, a_parts, a_stride, l_parts, l_stride, P, a_out, l_out); break;
+    case 2: merge_parts_kernel<2><<<grid, 128, 0, s>>>(d, g, a_parts, a_stride, l_parts, l_stride, P, a_out, l_out); break;
+    case 3: merge_parts_kernel<3><<<grid, 128, 0, s>>>(d, g, a_parts, a_stride, l_parts, l_stride, P, a_out, l_out); break;
+    case 4: merge_parts_kernel<4><<<grid, 128, 0, s>>>(d, g, a_parts, a_stride, l_parts, l_stride, P, a_out, l_out); break;
+    default: return cudaErrorInvalidValue;
+  }
   return cudaGetLastError();
 }
 

@@ -8,6 +8,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -204,7 +205,8 @@ int run_pass(const Dims& d0, long long keys, const void* q, const void* k, const
   d.head_stride = head_stride;
   PassArgs a;
   a.d = d;
-  a.plan = plan_split(d.R, d.D, keys, d.b, d.hkv, d.dtype, sms, step != nullptr && step->enabled);
+  const bool fused = step != nullptr && step->enabled;
+  a.plan = plan_split(d.R, d.D, keys, d.b, d.hkv, d.dtype, sms, fused, true, fused);
   if (a.plan.n_row_tiles > 65535) return FB_ERR_SHAPE;
   if (ws_bytes < a.plan.total()) return FB_ERR_WORKSPACE;
   a.q = q;
@@ -222,6 +224,13 @@ int run_pass(const Dims& d0, long long keys, const void* q, const void* k, const
                   ? reinterpret_cast<float*>(static_cast<char*>(ws) + a.plan.counter_bytes + a.plan.partial_bytes)
                   : nullptr;
   a.err = err;
+  if (a.plan.reuse_rows) {
+    // Batched fused step: every reusing row (and the decision record) first, in the
+    // light kernel; the pass then only touches tiles with a row that recomputes.
+    if (!reuse_rows_supported(d.dtype, d.D)) return FB_ERR_UNSUPPORTED;
+    a.step.reuse_done = 1;
+    FB_TRY(cuda_status(launch_reuse_rows(a, stream)));
+  }
   if (a.plan.tc) {
     // Dense contraction (more than 16 query rows per KV head): tcgen05 + TMEM.
     CUtensorMap tq, tk, tv;
@@ -244,15 +253,42 @@ int run_pass(const Dims& d0, long long keys, const void* q, const void* k, const
 size_t pass_bytes(const Dims& d, long long keys, bool with_inblock = false) {
   const int dev = current_device();
   const int sms = dev >= 0 ? device_sms(dev) : 0;
-  return plan_split(d.R, d.D, keys, d.b, d.hkv, d.dtype, sms > 0 ? sms : 148, with_inblock).total();
+  return plan_split(d.R, d.D, keys, d.b, d.hkv, d.dtype, sms > 0 ? sms : 148, with_inblock, true, with_inblock)
+      .total();
 }
 
 }  // namespace
 
 SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int num_sms, bool with_inblock,
-                     bool allow_tc) {
+                     bool allow_tc, bool batch_reuse) {
   SplitPlan p;
   std::memset(&p, 0, sizeof(p));
+  if (batch_reuse && with_inblock) {
+    // Batched fused step: when the units (on the mma.sync / fp32 row tiles) fill two
+    // waves or more, every tile is one split, the reuse-rows kernel writes the
+    // reusing rows, and bf16 runs persistent CTAs that skip tiles whose rows all reuse.
+    const int rt = dtype == FB_BF16 ? (R <= 16 ? 16 : (R <= 32 ? 32 : 64)) : 16;
+    const long long n_rt = (R + rt - 1) / rt;
+    const long long units = (long long)b * hkv * n_rt;
+    const long long wave = (long long)num_sms * (dtype == FB_BF16 ? 1 : 4);
+    if (units >= 2 * wave) {
+      p.row_tile = rt;
+      p.n_row_tiles = (int)n_rt;
+      p.key_tile = dtype == FB_BF16 ? 64 : 32;
+      p.splits = 1;
+      p.tiles_per_split = (int)((N + p.key_tile - 1) / p.key_tile);
+      p.reuse_rows = 1;
+      if (dtype == FB_BF16) {
+        p.persistent = 1;
+        const long long min_grid = (units + kMaxUnitsPerCta - 1) / kMaxUnitsPerCta;
+        p.grid = (int)std::max<long long>(std::min<long long>(units, num_sms), min_grid);
+      }
+      p.counter_bytes = ((size_t)units * 2 * 4 + 255) / 256 * 256;
+      p.partial_bytes = (size_t)units * p.row_tile * (D + 4) * sizeof(float);
+      p.inblock_bytes = (size_t)units * p.row_tile * (D + 4) * sizeof(float);
+      return p;
+    }
+  }
   if (dtype == FB_BF16) {
     // More than 16 packed query rows per KV head make the tiles a real dense
     // contraction: tcgen05 (M = 128, rows past the tile padded); otherwise mma.sync.
@@ -419,6 +455,24 @@ int fb_merge(const fb_shape* shape, const float* a1, const float* l1, const floa
   return cuda_status(launch_merge(d, a1, l1, a2, l2, a_full, l_full, (cudaStream_t)stream));
 }
 
+int fb_merge_partials(const fb_shape* shape, const float* a_parts, int64_t a_part_stride, const float* l_parts,
+                      int64_t l_part_stride, int n_parts, const fb_gate* gate, float* a_out, float* l_out,
+                      fb_stream_t stream) {
+  Dims d;
+  FB_TRY(resolve(shape, &d));
+  FB_TRY(check_ptr(a_parts));
+  FB_TRY(check_ptr(a_out));
+  if (!l_parts || !l_out) return FB_ERR_NULL;
+  if (n_parts < 1) return FB_ERR_ARG;
+  const long long rows = (long long)d.b * d.hq * d.B;
+  if (n_parts > 1 && (a_part_stride < rows * d.D || l_part_stride < rows)) return FB_ERR_SHAPE;
+  if (a_part_stride % 4) return FB_ERR_ALIGN;  // every partial's A starts 16-byte aligned
+  GateParams gp;
+  FB_TRY(gate_params(gate, d, &gp));
+  return cuda_status(launch_merge_parts(d, gp, a_parts, a_part_stride, l_parts, l_part_stride, n_parts, a_out,
+                                        l_out, (cudaStream_t)stream));
+}
+
 int fb_block_merge(const fb_shape* shape, const void* q, const void* k_blk, const void* v_blk,
                    const fb_gate* gate, const float* a_out, const float* l_out, void* a_full, float* l_full,
                    int32_t* dec_M, uint8_t* dec_reuse, void* ws, size_t ws_bytes, fb_stream_t stream) {
@@ -489,6 +543,7 @@ int fb_step(const fb_shape* shape, const void* q, const void* k_cache, const voi
     ep.a_dst = a_out;
     ep.l_dst = l_out;
     StepArgs st;
+    std::memset(&st, 0, sizeof(st));
     st.enabled = 1;
     st.k_blk = k_blk;
     st.v_blk = v_blk;
@@ -797,20 +852,15 @@ namespace fb {
 namespace {
 
 static __device__ __align__(256) unsigned char g_static_scratch[FB_STATIC_SCRATCH_BYTES];
-void* g_static_scratch_ptr[kMaxDevices];
 
-// Device address of g_static_scratch on `dev` (which must be current).  In host
-// code the array's name is only a stand-in, so the address is looked up once per
-// device and cached.
-int static_scratch(int dev, void** out) {
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_static_scratch_ptr[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
-    if (e != cudaSuccess || !p) return FB_ERR_CUDA;
-    g_static_scratch_ptr[dev] = p;
-  }
-  *out = g_static_scratch_ptr[dev];
+// Device address of g_static_scratch on the current device.  In host code the
+// array's name is only a stand-in, so the address is looked up on every call (a
+// host-side query; nothing is cached that a device reset could leave stale).
+int static_scratch(void** out) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+  if (e != cudaSuccess || !p) return FB_ERR_CUDA;
+  *out = p;
   return FB_OK;
 }
 
@@ -838,7 +888,7 @@ extern "C" int fb_prefix_attn_noalloc(const fb_shape* shape, const void* q, cons
   const SplitPlan plan = plan_split(d.R, d.D, d.N, d.b, d.hkv, d.dtype, sms);
   if (plan.total() > (size_t)FB_STATIC_SCRATCH_BYTES) return FB_ERR_WORKSPACE;
   void* ws = nullptr;
-  FB_TRY(static_scratch(dev, &ws));
+  FB_TRY(static_scratch(&ws));
   // The array keeps the previous call's contents: the arrival counters must start at zero.
   if (cudaMemsetAsync(ws, 0, plan.counter_bytes, (cudaStream_t)stream) != cudaSuccess) return FB_ERR_CUDA;
   Epilogue ep;

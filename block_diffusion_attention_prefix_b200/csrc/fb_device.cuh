@@ -295,49 +295,55 @@ __device__ __forceinline__ float inblock_row(const T* qrow, const T* kb, const T
   return m + logf(l);
 }
 
+// One in-block row of a step, by one warp: A_full = merge(cache row, in-block
+// row) (mode 1), or (A_in, L_in) written out (mode 0).  `grow` indexes [b, H_q, B];
+// `kb` / `vb` are the KV group's [B][D] block keys and values.  In mode 1 the cache
+// row is loaded before the in-block math so the two latencies overlap.  Every
+// mode-1 caller reads a cache that an earlier launch wrote and that no CTA of its
+// own launch writes (a reusing row's cache is left alone), so the cache is read
+// through the read-only L1 path.
+template <typename T, int D>
+__device__ __forceinline__ void inblock_merge_row(const Dims& d, const T* q, const T* kb, const T* vb, size_t grow,
+                                                  const Epilogue& ep, int lane) {
+  constexpr int DC = D / 32;
+  float ap[DC], lp = 0.f;
+  if (ep.mode == 1) {
+    lp = __ldg(ep.l_prev + grow);
+#pragma unroll
+    for (int t = 0; t < DC; ++t) ap[t] = __ldg(ep.a_prev + grow * D + lane * DC + t);
+  }
+  float a[DC];
+  const float L = inblock_row<T, D>(q + grow * D, kb, vb, d.B, d.scale, a, lane);
+  const size_t off = grow * D + (size_t)lane * DC;
+  if (ep.mode == 0) {
+#pragma unroll
+    for (int t = 0; t < DC; ++t) ep.a_dst[off + t] = a[t];
+    if (lane == 0) ep.l_dst[grow] = L;
+    return;
+  }
+  const MergeRow w = merge_row(lp, L);
+#pragma unroll
+  for (int t = 0; t < DC; ++t) {
+    const float v = merge_val(w, ap[t], a[t]);
+    if (ep.out_bf16)
+      static_cast<__nv_bfloat16*>(ep.a_full)[off + t] = __float2bfloat16_rn(v);
+    else
+      static_cast<float*>(ep.a_full)[off + t] = v;
+  }
+  if (lane == 0 && ep.l_full) ep.l_full[grow] = w.l;
+}
+
 // In-block rows [r_begin, r_end) of tile rows (group rows row0 + r) of KV group
-// (b, kvh), one warp per row, executed by warps [0, nwarps) of the CTA.  In mode 1
-// the cache row is loaded before the in-block math so the two latencies overlap.
-// Every mode-1 caller reads a cache that an earlier launch wrote and that no CTA of
-// its own launch writes (a reusing tile leaves its cache rows alone), so the cache
-// is read through the read-only L1 path, where the pass kernels' aux warp has
-// prefetched it while the gate read the mask.
+// (b, kvh), one warp per row (inblock_merge_row), executed by warps [0, nwarps) of
+// the CTA.
 template <typename T, int D>
 __device__ void inblock_rows(const Dims& d, const T* q, const T* k_blk, const T* v_blk, int b, int kvh,
                              int row0, int r_begin, int r_end, const Epilogue& ep, int warp, int nwarps,
                              int lane) {
-  constexpr int DC = D / 32;
   const T* kb = k_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
   const T* vb = v_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
   const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B + row0;
-  for (int r = r_begin + warp; r < r_end; r += nwarps) {
-    const size_t grow = grow0 + r;
-    float ap[DC], lp = 0.f;
-    if (ep.mode == 1) {
-      lp = __ldg(ep.l_prev + grow);
-#pragma unroll
-      for (int t = 0; t < DC; ++t) ap[t] = __ldg(ep.a_prev + grow * D + lane * DC + t);
-    }
-    float a[DC];
-    const float L = inblock_row<T, D>(q + grow * D, kb, vb, d.B, d.scale, a, lane);
-    const size_t off = grow * D + (size_t)lane * DC;
-    if (ep.mode == 0) {
-#pragma unroll
-      for (int t = 0; t < DC; ++t) ep.a_dst[off + t] = a[t];
-      if (lane == 0) ep.l_dst[grow] = L;
-      continue;
-    }
-    const MergeRow w = merge_row(lp, L);
-#pragma unroll
-    for (int t = 0; t < DC; ++t) {
-      const float v = merge_val(w, ap[t], a[t]);
-      if (ep.out_bf16)
-        static_cast<__nv_bfloat16*>(ep.a_full)[off + t] = __float2bfloat16_rn(v);
-      else
-        static_cast<float*>(ep.a_full)[off + t] = v;
-    }
-    if (lane == 0 && ep.l_full) ep.l_full[grow] = w.l;
-  }
+  for (int r = r_begin + warp; r < r_end; r += nwarps) inblock_merge_row<T, D>(d, q, kb, vb, grow0 + r, ep, lane);
 }
 
 // In-block rows [r_begin, r_end) of one tile written as (A_in, L_in) into the

@@ -15,6 +15,10 @@ namespace fb {
 // Largest block handled by the fused small-block code (scores on CUDA cores).
 constexpr int kSmallBlockMax = 64;
 
+// Largest number of row tiles a persistent pass CTA walks (its list of tiles that
+// recompute lives in shared memory).
+constexpr int kMaxUnitsPerCta = 1024;
+
 // Gate of one denoising step, as device-readable arguments.  enabled == 0 means
 // "recompute every row" (no gate).  See fb_gate in include/fb.h.
 struct GateParams {
@@ -45,6 +49,9 @@ struct SplitPlan {
   int splits;           // CTAs along the key axis per (b, kv head, row tile)
   int tiles_per_split;  // key tiles per split
   int tc;               // 0: mma.sync / CUDA-core pass; 1: tcgen05 split pass; 2: tcgen05, one CTA per row tile
+  int persistent;       // bf16 mma.sync pass, one split: a grid of `grid` CTAs that each walk their row tiles
+  int grid;             // persistent: CTAs of the launch
+  int reuse_rows;       // batched fused step: the reuse-rows kernel runs first (see plan_split)
   size_t counter_bytes; // arrival then departure counters, one each per (b, kv head, row tile), 256-B padded
   size_t partial_bytes; // [b*hkv][n_row_tiles][splits][row_tile][D + 4] fp32
   size_t inblock_bytes; // fused step only: [b*hkv][n_row_tiles][row_tile][D + 4] fp32 (A_in, L_in)
@@ -76,6 +83,7 @@ struct StepArgs {
   float* l_full;          // nullable
   int32_t* dec_M;         // nullable
   uint8_t* dec_reuse;     // nullable
+  int reuse_done;         // the reuse-rows kernel already wrote the reusing rows and the decisions
 };
 
 // Arguments of a split-KV attention pass (prefix, or in-block for large B).
@@ -136,8 +144,12 @@ cudaError_t launch_sparse_select(const SparseArgs& a, cudaStream_t s);
 cudaError_t launch_sparse_pass(const SparseArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                                const CUtensorMap& tk4, const CUtensorMap& tv4, cudaStream_t s);
 
+// batch_reuse: a fused step (fb_step) may take the batched plan -- when the (b, KV
+// head, row tile) units fill two waves or more, the reuse-rows kernel writes every
+// reusing row first and the pass (one split per tile, persistent CTAs for bf16)
+// walks only the tiles that recompute.
 SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int num_sms,
-                     bool with_inblock = false, bool allow_tc = true);
+                     bool with_inblock = false, bool allow_tc = true, bool batch_reuse = false);
 
 // Launchers (return cudaError_t of the launch).
 cudaError_t launch_pass_f32(const PassArgs& a, cudaStream_t s);
@@ -147,6 +159,12 @@ int bf16_pass_supported(int D, int row_tile);
 // tcgen05 pass (flash_tc.cu): bf16, D = 128, more than 16 query rows per KV head.
 cudaError_t launch_pass_tc(const PassArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            cudaStream_t s);
+
+// Reusing rows of a step for many (b, KV head) groups at once (reuse.cu): the gate,
+// the decisions, and A_full = merge(cache row, in-block row) for every row whose
+// head reuses; one CTA per group, a warp per row.
+cudaError_t launch_reuse_rows(const PassArgs& a, cudaStream_t s);
+int reuse_rows_supported(int dtype, int D);
 
 // Small in-block pass fused with gate and merge (B <= kSmallBlockMax).
 struct SmallBlockArgs {
@@ -162,6 +180,10 @@ struct SmallBlockArgs {
 cudaError_t launch_small_block(const SmallBlockArgs& a, cudaStream_t s);
 cudaError_t launch_gate_eval(const Dims& d, const GateParams& g, int32_t* dec_M, uint8_t* dec_reuse,
                              cudaStream_t s);
+// Context-parallel combine: cache rows of recomputing heads = merge of P partials.
+cudaError_t launch_merge_parts(const Dims& d, const GateParams& g, const float* a_parts, long long a_stride,
+                               const float* l_parts, long long l_stride, int P, float* a_out, float* l_out,
+                               cudaStream_t s);
 cudaError_t launch_merge(const Dims& d, const float* a1, const float* l1, const float* a2,
                          const float* l2, void* a_full, float* l_full, cudaStream_t s);
 // Per-head similarity estimate (similarity.cu): workspace bytes, sim = cosine of

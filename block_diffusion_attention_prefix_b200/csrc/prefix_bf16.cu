@@ -76,29 +76,41 @@ struct Cfg {
 constexpr int kBarConsumers = 1;
 constexpr int kBarFinish = 2;
 
+// Shared state of one CTA of the pass, kept across the work items of a persistent CTA.
+template <int RT>
+struct PassShared {
+  uint64_t full_bar[8];
+  uint64_t empty_bar[8];
+  uint64_t fin_bar;
+  int flags[RT];
+  int red[32];
+  int M;
+};
+
+// One work item of the pass -- split `split` of row tile `rt` of (b, KV head) `bg`
+// -- executed by every thread of the CTA (the producer warp included).  `tile_base`
+// counts the K/V tiles this CTA pushed through its ring before this item, so the
+// ring's mbarrier phases continue from one item to the next.  `init_bars`: the
+// mbarriers are initialised here, once the gate says the item has work (single-item
+// CTAs); persistent CTAs initialise them once up front.  Returns false when a
+// bounded wait of this thread gave up.
 template <int D, int WARPS_M, int WARPS_N, int STAGES>
-__global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
-    pass_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                     const PassArgs args) {
+__device__ __forceinline__ bool pass_unit(const CUtensorMap* tmK, const CUtensorMap* tmV, const PassArgs& args,
+                                          int split, int rt, int bg, uint8_t* smem,
+                                          PassShared<Cfg<D, WARPS_M, WARPS_N, STAGES>::kRowTile>& sh,
+                                          uint32_t& fin_phase, long long tile_base, bool init_bars) {
   using C = Cfg<D, WARPS_M, WARPS_N, STAGES>;
   constexpr int NCW = C::kConsumerWarps;
   constexpr int KW = C::KW;
   constexpr int RT = C::kRowTile;
   using bf16 = __nv_bfloat16;
-
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ __align__(8) uint64_t full_bar[STAGES];
-  __shared__ __align__(8) uint64_t empty_bar[STAGES];
-  __shared__ __align__(8) uint64_t fin_bar;
-  __shared__ int s_flags[RT];
-  __shared__ int s_red[32];
-  __shared__ int s_M;
+  uint64_t* full_bar = sh.full_bar;
+  uint64_t* empty_bar = sh.empty_bar;
+  int* s_flags = sh.flags;
 
   const Dims& d = args.d;
   const SplitPlan& plan = args.plan;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int split = blockIdx.x, rt = blockIdx.y, bg = blockIdx.z;
   const int b = bg / d.hkv, kvh = bg - b * d.hkv;
   const int row0 = rt * RT;
   const int rows_valid = min(RT, d.R - row0);
@@ -107,11 +119,7 @@ __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
   const bf16* q = static_cast<const bf16*>(args.q);
   const bf16* k_blk = static_cast<const bf16*>(args.step.k_blk);
   const bf16* v_blk = static_cast<const bf16*>(args.step.v_blk);
-  if (warp == C::kProducerWarp && lane == 0) {
-    prefetch_tmap(&tmK);
-    prefetch_tmap(&tmV);
-  }
-  if (args.step.enabled && warp == C::kAuxWarp) {
+  if (args.step.enabled && !plan.persistent && warp == C::kAuxWarp) {
     // Whatever the gate decides, this CTA computes its share of the in-block rows:
     // pull their q rows, the group's block keys and values and the cached rows into
     // L1 while the gate reads the mask.
@@ -137,58 +145,68 @@ __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
     }
   }
 
-  if (!gate_row_flags(args.gate, d, b, kvh, row0, rows_valid, RT, s_flags, s_red, &s_M)) {
+  if (!gate_row_flags(args.gate, d, b, kvh, row0, rows_valid, RT, s_flags, sh.red, &sh.M)) {
     // Every row of this tile reuses its cache: no K/V is read.  In a fused step the
     // tile's CTAs still produce the step's output from the cache.
-    if (args.step.enabled) {
+    // (When the reusing rows were handled by the reuse-rows kernel, nothing is left.)
+    if (args.step.enabled && !args.step.reuse_done) {
       int r0, r1;
       split_rows(rows_valid, plan.splits, split, r0, r1);
       inblock_rows<bf16, D>(d, q, k_blk, v_blk, b, kvh, row0, r0, r1, step_epilogue(args), warp, C::kThreads / 32,
                             lane);
       if (split == 0)
-        record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, s_M, args.step.dec_M,
+        record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, sh.M, args.step.dec_M,
                          args.step.dec_reuse, kvh == 0 && rt == 0, tid, C::kThreads);
     }
-    return;
+    return true;
   }
 
   const long long key_begin = (long long)split * plan.tiles_per_split * kKeyTile;
   const long long key_end = min(d.N, key_begin + (long long)plan.tiles_per_split * kKeyTile);
   const int ntiles = key_end > key_begin ? (int)((key_end - key_begin + kKeyTile - 1) / kKeyTile) : 0;
 
-  if (tid == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], NCW);
+  if (init_bars) {
+    if (tid == 0) {
+      for (int s = 0; s < STAGES; ++s) {
+        mbar_init(&full_bar[s], 1);
+        mbar_init(&empty_bar[s], NCW);
+      }
+      mbar_init(&sh.fin_bar, 1);
+      fence_mbar_init();
     }
-    mbar_init(&fin_bar, 1);
-    fence_mbar_init();
+    __syncthreads();
   }
-  __syncthreads();
+  bool ok = true;
 
   if (warp == C::kProducerWarp) {
     // ---------------- producer warp: TMA loads into the ring ----------------
     if (lane == 0 && ntiles > 0) {
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
-        const int s = i % STAGES;
-        const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
-        if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, args.err, DEV_ERR_WAIT_EMPTY)) break;
+        const long long gi = tile_base + i;  // ring position across work items
+        const int s = (int)(gi % STAGES);
+        const uint32_t ph = (uint32_t)(gi / STAGES) & 1u;
+        if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, args.err, DEV_ERR_WAIT_EMPTY)) {
+          ok = false;
+          break;
+        }
         mbar_arrive_expect_tx(&full_bar[s], C::kStageBytes);
         const int key0 = (int)(key_begin + (long long)i * kKeyTile);
         uint8_t* st = smem + s * C::kStageBytes;
 #pragma unroll
-        for (int h = 0; h < D / 64; ++h) tma_load_3d(st + h * (kKeyTile * 128), &tmK, &full_bar[s], h * 64, key0, bg);
+        for (int h = 0; h < D / 64; ++h) tma_load_3d(st + h * (kKeyTile * 128), tmK, &full_bar[s], h * 64, key0, bg);
 #pragma unroll
         for (int h = 0; h < D / 64; ++h)
-          tma_load_3d(st + C::kTileBytes + h * (kKeyTile * 128), &tmV, &full_bar[s], h * 64, key0, bg);
+          tma_load_3d(st + C::kTileBytes + h * (kKeyTile * 128), tmV, &full_bar[s], h * 64, key0, bg);
         ++issued;
       }
       // Do not leave while copies issued by this CTA may still be landing.
-      for (int i = max(0, issued - STAGES); i < issued; ++i)
-        mbar_wait_bounded(&full_bar[i % STAGES], (uint32_t)(i / STAGES) & 1u, args.err, DEV_ERR_WAIT_FULL);
+      for (int i = max(0, issued - STAGES); i < issued; ++i) {
+        const long long gi = tile_base + i;
+        ok &= mbar_wait_bounded(&full_bar[gi % STAGES], (uint32_t)(gi / STAGES) & 1u, args.err, DEV_ERR_WAIT_FULL);
+      }
     }
-    return;
+    return ok;
   }
 
   if (warp == C::kAuxWarp) {
@@ -225,11 +243,11 @@ __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
     for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
     const float sl2 = d.scale * 1.4426950408889634f;  // scale * log2(e)
-    bool ok = true;
 
     for (int i = 0; i < ntiles && ok; ++i) {
-      const int s = i % STAGES;
-      if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(i / STAGES) & 1u, args.err, DEV_ERR_WAIT_FULL)) {
+      const long long gi = tile_base + i;
+      const int s = (int)(gi % STAGES);
+      if (!mbar_wait_bounded(&full_bar[s], (uint32_t)(gi / STAGES) & 1u, args.err, DEV_ERR_WAIT_FULL)) {
         ok = false;
         break;
       }
@@ -392,31 +410,107 @@ __global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
   split_rows(rows_valid, plan.splits, split, r0, r1);
   const Epilogue sep = step_epilogue(args);
   const size_t nunits = (size_t)d.b * d.hkv * plan.n_row_tiles;
-  uint32_t fin_phase = 0;
   coop_finish_rows<D, C::kFinishThreads>(args.partials + unit * plan.splits * RT * (D + 4), plan.splits, RT, r0, r1,
                                          args.step.enabled ? args.inblock + unit * RT * (D + 4) : nullptr, s_flags,
                                          grow0, args.ep, args.step.enabled ? &sep : nullptr, smem, C::kRingBytes,
-                                         &fin_bar, &fin_phase, args.counters + unit, args.counters + nunits + unit,
+                                         &sh.fin_bar, &fin_phase, args.counters + unit, args.counters + nunits + unit,
                                          args.err, ftid, kBarFinish);
-  if (args.step.enabled && split == 0)
-    record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, s_M, args.step.dec_M, args.step.dec_reuse,
+  if (args.step.enabled && !args.step.reuse_done && split == 0)
+    record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, sh.M, args.step.dec_M, args.step.dec_reuse,
                      kvh == 0 && rt == 0, ftid, C::kFinishThreads);
+  return ok;
+}
+
+
+// PERSIST = false: one work item per CTA, grid (splits, row tiles, b * H_kv).
+// PERSIST = true: the batched fused step's persistent CTAs (plan.persistent).
+template <int D, int WARPS_M, int WARPS_N, int STAGES, bool PERSIST>
+__global__ void __launch_bounds__(Cfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1)
+    pass_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const PassArgs args) {
+  using C = Cfg<D, WARPS_M, WARPS_N, STAGES>;
+  constexpr int RT = C::kRowTile;
+  static_assert(STAGES <= 8, "PassShared holds up to 8 stages");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) PassShared<RT> sh;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (warp == C::kProducerWarp && lane == 0) {
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+  }
+  uint32_t fin_phase = 0;
+  const SplitPlan& plan = args.plan;
+  if constexpr (!PERSIST) {
+    pass_unit<D, WARPS_M, WARPS_N, STAGES>(&tmK, &tmV, args, blockIdx.x, blockIdx.y, blockIdx.z, smem, sh,
+                                           fin_phase, 0, true);
+    return;
+  }
+  // Persistent CTA (one split per tile, many tiles): work items u = blockIdx.x + k * gridDim.x.
+  // First the gate of each of them, one thread per item, so that items whose rows all
+  // reuse cost no pass at all; then the remaining items one after another.
+  __shared__ int s_units[kMaxUnitsPerCta];
+  __shared__ int s_nunits, s_abort;
+  const Dims& d = args.d;
+  const GateParams& g = args.gate;
+  if (tid == 0) {
+    s_nunits = 0;
+    s_abort = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&sh.full_bar[s], 1);
+      mbar_init(&sh.empty_bar[s], C::kConsumerWarps);
+    }
+    mbar_init(&sh.fin_bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const long long units = (long long)d.b * d.hkv * plan.n_row_tiles;
+  for (long long u = blockIdx.x + (long long)tid * gridDim.x; u < units; u += (long long)C::kThreads * gridDim.x) {
+    const int bg = (int)(u / plan.n_row_tiles), rt = (int)(u - (long long)bg * plan.n_row_tiles);
+    const int b = bg / d.hkv, kvh = bg - b * d.hkv;
+    const int row0 = rt * RT, rows_valid = min(RT, d.R - row0);
+    bool need = true;
+    if (g.enabled) {
+      int M = 0;
+      for (int i = 0; i < d.B; ++i) M += g.mask[(size_t)b * d.B + i] != 0;
+      const bool tau_ok = tau_reuse(g, M);
+      need = false;
+      const int h0 = kvh * d.G + row0 / d.B, h1 = kvh * d.G + (row0 + rows_valid - 1) / d.B;
+      for (int h = h0; h <= h1 && !need; ++h) need = !head_reuse(g, tau_ok, b, d.hq, h);
+    }
+    if (need) s_units[atomicAdd(&s_nunits, 1)] = (int)u;
+  }
+  __syncthreads();
+  const int n = s_nunits;
+  long long tile_base = 0;
+  for (int li = 0; li < n; ++li) {
+    const int u = s_units[li];
+    const int bg = u / plan.n_row_tiles, rt = u - bg * plan.n_row_tiles;
+    const bool ok =
+        pass_unit<D, WARPS_M, WARPS_N, STAGES>(&tmK, &tmV, args, 0, rt, bg, smem, sh, fin_phase, tile_base, false);
+    tile_base += plan.tiles_per_split;
+    fence_proxy_async_smem();  // generic writes to the ring (scratch, staging) before the next item's TMA loads
+    if (!ok) s_abort = 1;
+    __syncthreads();
+    if (s_abort) break;
+  }
 }
 
 template <int D, int WM, int WN, int STAGES>
 cudaError_t launch_cfg(const PassArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t s) {
   using C = Cfg<D, WM, WN, STAGES>;
-  auto kern = pass_bf16_kernel<D, WM, WN, STAGES>;
-  static bool attr_set[64] = {};
+  auto kern = a.plan.persistent ? pass_bf16_kernel<D, WM, WN, STAGES, true> : pass_bf16_kernel<D, WM, WN, STAGES, false>;
+  static bool attr_set[2][64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+  const int pi = a.plan.persistent ? 1 : 0;
+  if (dev < 0 || dev >= 64 || !attr_set[pi][dev]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    if (dev >= 0 && dev < 64) attr_set[pi][dev] = true;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.plan.splits, a.plan.n_row_tiles, a.d.b * a.d.hkv);
+  cfg.gridDim = a.plan.persistent ? dim3(a.plan.grid) : dim3(a.plan.splits, a.plan.n_row_tiles, a.d.b * a.d.hkv);
   cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = s;

@@ -59,8 +59,9 @@ __global__ void __launch_bounds__(kThreads) pass_f32_kernel(const PassArgs args)
   const size_t unit = (size_t)bg * plan.n_row_tiles + rt;
 
   if (!gate_row_flags(args.gate, d, b, kvh, row0, rows_valid, RT, &s_flags[0], s_red, &s_M)) {
-    // Every row reuses its cache: in a fused step, merge this split's rows with it.
-    if (args.step.enabled) {
+    // Every row reuses its cache: in a fused step, merge this split's rows with it
+    // (unless the reuse-rows kernel already did).
+    if (args.step.enabled && !args.step.reuse_done) {
       inblock_rows<float, D>(d, static_cast<const float*>(args.q), static_cast<const float*>(args.step.k_blk),
                              static_cast<const float*>(args.step.v_blk), b, kvh, row0, ib0, ib1, step_ep, warp,
                              kThreads / 32, lane);
@@ -157,8 +158,9 @@ __global__ void __launch_bounds__(kThreads) pass_f32_kernel(const PassArgs args)
   if (args.step.enabled) {
     __syncthreads();  // the recomputed cache rows are written
     merge_tile_from_ws<D>(step_ep, grow0, rows_valid, args.inblock + unit * RT * (D + 4), tid, kThreads);
-    record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, s_M, args.step.dec_M, args.step.dec_reuse,
-                     kvh == 0 && rt == 0, tid, kThreads);
+    if (!args.step.reuse_done)
+      record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, s_M, args.step.dec_M, args.step.dec_reuse,
+                       kvh == 0 && rt == 0, tid, kThreads);
   }
   if (tid == 0) args.counters[unit] = 0u;
 }

@@ -1,0 +1,111 @@
+// reuse.cu -- the reusing rows of a denoising step, for many problems at once.
+//
+// FlashBlock technical summary (gist.science 2602.05305), "2. Methodology / Core
+// mechanism": a row whose cache is reused gets A_full = merge(cached (A_out,
+// L_out), fresh in-block (A_in, L_in)); the prefix K/V are not read.  "Adaptive
+// reuse strategies": the row's head reuses iff the step is not the block's first,
+// M^{s+1} < tau and (with a per-head gate) its similarity is above gamma.
+//
+// When one call carries many independent (b, KV head) groups -- the batch of a
+// serving step, or every layer of a model stacked on the batch axis -- the pass
+// kernel's one-CTA-per-SM shared-memory ring would hold a whole SM per reusing
+// tile.  This kernel instead runs a group per CTA with no dynamic shared memory, so
+// several CTAs (and a warp per row) share each SM and the rows' loads overlap:
+// the gate, the decision record (dec_M, dec_reuse), and for every reusing row the
+// in-block attention merged with its cached row, in the same arithmetic as the
+// pass kernels' fused epilogue (inblock_merge_row), so the results agree bit for
+// bit.  Rows that recompute are left to the prefix pass that follows.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "fb_device.cuh"
+#include "fb_internal.h"
+
+namespace fb {
+namespace {
+
+constexpr int kReuseThreads = 256;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kReuseThreads, 3) reuse_rows_kernel(const PassArgs args) {
+  __shared__ int s_red[32];
+  const Dims& d = args.d;
+  const GateParams& g = args.gate;
+  const int bg = blockIdx.x, b = bg / d.hkv, kvh = bg - b * d.hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B;
+  {
+    // Pull the group's rows into L1 while the gate reads the mask, so each row's
+    // loads below hit L1 instead of paying a DRAM latency each: the q rows, the
+    // cached rows (A and L) and the block's keys and values.  Every prefetched
+    // address lies inside its buffer (a range's last byte covers its last line).
+    const char* base[5] = {reinterpret_cast<const char*>(static_cast<const T*>(args.q) + grow0 * D),
+                           reinterpret_cast<const char*>(args.ep.a_dst + grow0 * D),
+                           reinterpret_cast<const char*>(args.ep.l_dst + grow0),
+                           reinterpret_cast<const char*>(static_cast<const T*>(args.step.k_blk) + (size_t)bg * d.B * D),
+                           reinterpret_cast<const char*>(static_cast<const T*>(args.step.v_blk) + (size_t)bg * d.B * D)};
+    const size_t bytes[5] = {(size_t)d.R * D * sizeof(T), (size_t)d.R * D * 4, (size_t)d.R * 4,
+                             (size_t)d.B * D * sizeof(T), (size_t)d.B * D * sizeof(T)};
+#pragma unroll
+    for (int t = 0; t < 5; ++t) {
+      const int lines = (int)((bytes[t] + 127) / 128);
+      for (int i = tid; i <= lines; i += kReuseThreads)
+        prefetch_l1(base[t] + (i < lines ? (size_t)i * 128 : bytes[t] - 1));
+    }
+  }
+  const int M = block_updated_count(g.mask + (size_t)b * d.B, d.B, s_red);
+  const bool tau_ok = tau_reuse(g, M);
+  if (kvh == 0 && tid == 0 && args.step.dec_M) args.step.dec_M[b] = M;
+  if (args.step.dec_reuse)
+    for (int j = tid; j < d.G; j += kReuseThreads) {
+      const int h = kvh * d.G + j;
+      args.step.dec_reuse[(size_t)b * d.hq + h] = head_reuse(g, tau_ok, b, d.hq, h) ? 1 : 0;
+    }
+  if (!tau_ok) return;  // every head of this batch element recomputes: the prefix pass writes its rows
+
+  Epilogue ep;
+  ep.mode = 1;
+  ep.a_dst = nullptr;
+  ep.l_dst = nullptr;
+  ep.a_prev = args.ep.a_dst;  // the cache
+  ep.l_prev = args.ep.l_dst;
+  ep.a_full = args.step.a_full;
+  ep.l_full = args.step.l_full;
+  ep.out_bf16 = d.dtype == 1;
+  const T* q = static_cast<const T*>(args.q);
+  const T* kb = static_cast<const T*>(args.step.k_blk) + (size_t)bg * d.B * D;
+  const T* vb = static_cast<const T*>(args.step.v_blk) + (size_t)bg * d.B * D;
+  constexpr int kWarps = kReuseThreads / 32;
+  for (int r = warp; r < d.R; r += kWarps) {
+    if (!head_reuse(g, true, b, d.hq, kvh * d.G + r / d.B)) continue;  // warp-uniform
+    inblock_merge_row<T, D>(d, q, kb, vb, grow0 + r, ep, lane);
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_typed(const PassArgs& a, cudaStream_t s) {
+  reuse_rows_kernel<T, D><<<(unsigned)(a.d.b * a.d.hkv), kReuseThreads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int reuse_rows_supported(int dtype, int D) {
+  return dtype == 1 ? (D == 64 || D == 128) : (D == 32 || D == 64 || D == 96 || D == 128);
+}
+
+cudaError_t launch_reuse_rows(const PassArgs& a, cudaStream_t s) {
+  const int D = a.d.D;
+  if (a.d.dtype == 1) {
+    if (D == 128) return launch_typed<__nv_bfloat16, 128>(a, s);
+    if (D == 64) return launch_typed<__nv_bfloat16, 64>(a, s);
+  } else {
+    if (D == 128) return launch_typed<float, 128>(a, s);
+    if (D == 96) return launch_typed<float, 96>(a, s);
+    if (D == 64) return launch_typed<float, 64>(a, s);
+    if (D == 32) return launch_typed<float, 32>(a, s);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace fb

@@ -16,7 +16,8 @@ import torch
 __all__ = [
     "FBError", "Shape", "Gate", "load", "lib_path", "make_shape", "make_gate", "FB_F32", "FB_BF16",
     "fb_version", "fb_status_string", "fb_device_error", "fb_workspace_bytes", "fb_workspace_init",
-    "fb_gate_eval", "fb_prefix_attn", "fb_prefix_attn_noalloc", "fb_block_attn", "fb_merge", "fb_block_merge", "fb_step",
+    "fb_gate_eval", "fb_prefix_attn", "fb_prefix_attn_noalloc", "fb_block_attn", "fb_merge", "fb_merge_partials",
+    "fb_block_merge", "fb_step",
     "fb_page_minmax", "fb_append_block", "fb_similarity_workspace_bytes", "fb_head_similarity",
     "fb_refresh_reference", "fb_losa_step", "LosaLayer", "fb_sparse_workspace_bytes", "fb_sparse_select", "fb_sparse_step", "Sparse",
     "SparseResidualLayer", "CachedAttentionLayer", "EXPORTED",
@@ -81,6 +82,7 @@ EXPORTED = {
     "fb_block_merge": (_i, [_PS, _vp, _vp, _vp, _PG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fb_step": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _PG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fb_prefix_attn_noalloc": (_i, [_PS, _vp, _vp, _vp, _PG, _vp, _vp, _vp]),
+    "fb_merge_partials": (_i, [_PS, _vp, ctypes.c_int64, _vp, ctypes.c_int64, _i, _PG, _vp, _vp, _vp]),
     "fb_page_cap": (_i, [_PS, _i]),
     "fb_page_minmax": (_i, [_PS, _vp, _i, _vp, _vp, _vp]),
     "fb_append_block": (_i, [_PS, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
@@ -122,6 +124,15 @@ def _ptr(t: Optional[torch.Tensor]):
         raise ValueError("libfb takes device tensors")
     if not t.is_contiguous():
         raise ValueError("libfb takes contiguous tensors (strides go through the shape)")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _ptr_any(t: Optional[torch.Tensor]):
+    """Device pointer of a tensor that may be a strided view (the strides go in the call)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libfb takes device tensors")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -200,6 +211,13 @@ def fb_block_attn(shape, q, k_blk, v_blk, a_in, l_in, ws=None):
 def fb_merge(shape, a1, l1, a2, l2, a_full, l_full=None):
     _check("fb_merge", load().fb_merge(ctypes.byref(shape), _ptr(a1), _ptr(l1), _ptr(a2), _ptr(l2), _ptr(a_full),
                                        _ptr(l_full), _stream()))
+
+
+def fb_merge_partials(shape, a_parts, a_part_stride, l_parts, l_part_stride, n_parts, gate, a_out, l_out):
+    """Cache rows of recomputing heads = log-space merge of n_parts partials (strides in elements)."""
+    _check("fb_merge_partials", load().fb_merge_partials(
+        ctypes.byref(shape), _ptr_any(a_parts), int(a_part_stride), _ptr_any(l_parts), int(l_part_stride),
+        int(n_parts), _gref(gate), _ptr(a_out), _ptr(l_out), _stream()))
 
 
 def fb_block_merge(shape, q, k_blk, v_blk, gate, a_out, l_out, a_full, l_full=None, dec_M=None, dec_reuse=None,

@@ -124,10 +124,12 @@ int fb_workspace_init(void* ws, size_t ws_bytes, fb_stream_t stream);
 int fb_gate_eval(const fb_shape* shape, const fb_gate* gate, int32_t* dec_M, uint8_t* dec_reuse,
                  fb_stream_t stream);
 
-/* Out-of-block attention (split-KV pass, split combine, cache write): (A_out, L_out)
- * of every query row over the whole prefix J_out, computed split-KV and reduced in
- * log space.  With gate ==
- * NULL every row is recomputed; otherwise only rows of heads whose decision is
+/* Out-of-block attention (split-KV pass, split combine, cache write).  Passage:
+ * FlashBlock technical summary, "2. Methodology / Core mechanism" -- A_out and
+ * L_out = log Z_out over J_out (the tokens outside the current block), computed
+ * once and cached.  (A_out, L_out) of every query row over the whole prefix J_out,
+ * computed split-KV and reduced in log space.  With gate == NULL every row is
+ * recomputed; otherwise only rows of heads whose decision is
  * "recompute" are written, and rows of reusing heads are left bit-for-bit
  * untouched (the decision is taken on the device; no host synchronisation).
  * ws: fb_workspace_bytes(shape) bytes. */
@@ -135,17 +137,42 @@ int fb_prefix_attn(const fb_shape* shape, const void* q, const void* k_cache, co
                    const fb_gate* gate, float* a_out, float* l_out, void* ws, size_t ws_bytes,
                    fb_stream_t stream);
 
-/* In-block attention: (A_in, L_in) of every query row over the B block keys,
- * bidirectional (no mask).  ws may be NULL when block <= 64; larger blocks need
+/* In-block attention.  Passage: FlashBlock technical summary, "2. Methodology /
+ * Core mechanism" -- the part over J_in, the tokens of the current block, that
+ * every denoising step computes afresh.  (A_in, L_in) of every query row over the
+ * B block keys, bidirectional (no mask).  ws may be NULL when block <= 64; larger blocks need
  * fb_workspace_bytes(shape) bytes. */
 int fb_block_attn(const fb_shape* shape, const void* q, const void* k_blk, const void* v_blk,
                   float* a_in, float* l_in, void* ws, size_t ws_bytes, fb_stream_t stream);
 
-/* Log-space merge, elementwise over [b, H_q, B] rows:
+/* Log-space merge.  Passage: FlashBlock technical summary, "2. Methodology /
+ * Core mechanism", the merge equation (also the split-KV reduction: every split is
+ * a subset of J_out).  Elementwise over [b, H_q, B] rows:
  * A_full = merge((a1, l1), (a2, l2)) in the shape's dtype; l_full (nullable) gets
  * m + ln(e^{l1-m} + e^{l2-m}).  Two empty inputs give (0, -inf). */
 int fb_merge(const fb_shape* shape, const float* a1, const float* l1, const float* a2,
              const float* l2, void* a_full, float* l_full, fb_stream_t stream);
+
+/* Context-parallel combine of the out-of-block part.  Passage: FlashBlock
+ * technical summary, "2. Methodology / Core mechanism", the merge equation: the
+ * log-space merge of partial results over disjoint key sets is the result over
+ * their union, so J_out may be cut into P key ranges -- one per GPU, each GPU
+ * holding its range of the prefix K/V -- whose partial (A, L) are computed apart
+ * (fb_prefix_attn on the range) and merged here.  Partial p (p = 0 .. n_parts-1)
+ * is A_p = a_parts + p * a_part_stride ([b, H_q, B, D] fp32) and L_p = l_parts +
+ * p * l_part_stride ([b, H_q, B] fp32, natural log); the caller gathers them into
+ * these buffers (e.g. one all-gather).  For every row of a head whose gate decision
+ * is "recompute" (every row when gate == NULL):
+ *     M = max_p L_p,  e_p = e^{L_p - M},  den = sum_p e_p   (p ascending)
+ *     A_out = (sum_p e_p A_p) / den,  L_out = M + ln den
+ * written to a_out / l_out (the cache); rows of reusing heads are left untouched.
+ * Empty ranges (L = -inf) are allowed; all empty gives (0, -inf).  The merge runs
+ * in range order, so the result does not depend on timing.  a_part_stride must be
+ * a multiple of 4 (16-byte aligned partials) and, with n_parts > 1, at least
+ * b*H_q*B*D; l_part_stride at least b*H_q*B. */
+int fb_merge_partials(const fb_shape* shape, const float* a_parts, int64_t a_part_stride,
+                      const float* l_parts, int64_t l_part_stride, int n_parts, const fb_gate* gate,
+                      float* a_out, float* l_out, fb_stream_t stream);
 
 /* Second half of a step (gate, in-block attention, merge): evaluates the gate, records dec_M /
  * dec_reuse (nullable), computes (A_in, L_in) and merges it with the cache
@@ -156,7 +183,10 @@ int fb_block_merge(const fb_shape* shape, const void* q, const void* k_blk, cons
                    float* l_full, int32_t* dec_M, uint8_t* dec_reuse, void* ws, size_t ws_bytes,
                    fb_stream_t stream);
 
-/* One denoising step of one attention layer: fb_prefix_attn(gate) refreshes the
+/* One denoising step of one attention layer.  Passages: FlashBlock technical
+ * summary, "2. Methodology / Core mechanism" (cache, in-block part, merge) and
+ * "Adaptive reuse strategies" (the tau and gamma gates that decide whether the
+ * cache is reused).  fb_prefix_attn(gate) refreshes the
  * cache rows that recompute, then fb_block_merge writes A_full, L_full and the
  * decisions.  On a reuse step the prefix K/V are not read.  gate is required. */
 int fb_step(const fb_shape* shape, const void* q, const void* k_cache, const void* v_cache,
@@ -238,12 +268,14 @@ int fb_losa_step(const fb_shape* shape, const void* q, const void* q_prev, const
  * queries q [b, H_q, B, D] and the reference queries q_ref (same layout and dtype:
  * the queries the head's cache was last computed with), i.e.
  * <Q, R> / sqrt(<Q, Q> <R, R>) in float64 rounded to float32 (0 when a norm is 0).
- * The sums run in one fixed order -- per row ascending d, rows in chunks of 256 as a
- * pairwise tree, chunk totals in ascending order -- so the result, and the gate
- * decision sim > gamma taken on it, is reproducible bit for bit.  sim [b, H_q]
+ * The sums run in one plain order -- each row's products in ascending d give the
+ * row's dot product, and the row dot products are added one after another in
+ * ascending row order -- so the result, and the gate decision sim > gamma taken on
+ * it, is reproducible bit for bit.  sim [b, H_q]
  * float32 device memory, then usable as fb_gate.head_sim.  Workspace: at least
- * fb_similarity_workspace_bytes(shape) bytes, zeroed once (fb_workspace_init); its
- * counters return to zero after each call.  Asynchronous on `stream`. */
+ * fb_similarity_workspace_bytes(shape) bytes (arrival counters and 32 bytes per
+ * query row), zeroed once (fb_workspace_init); its counters return to zero after
+ * each call.  Asynchronous on `stream`. */
 size_t fb_similarity_workspace_bytes(const fb_shape* shape);
 int fb_head_similarity(const fb_shape* shape, const void* q, const void* q_ref, float* sim, void* ws,
                        size_t ws_bytes, fb_stream_t stream);
@@ -304,10 +336,15 @@ int fb_sparse_step(const fb_shape* shape, const void* q, const void* k_cache, co
  * call.  The caller still passes q, the KV cache and the outputs, with the same
  * meaning, layout and gate as fb_prefix_attn.
  *
- *  - Shapes whose workspace (fb_workspace_bytes for the prefix pass) exceeds
- *    FB_STATIC_SCRATCH_BYTES are rejected with FB_ERR_WORKSPACE before any launch.
- *  - The first call on a device looks up the array's device address (with that
- *    device current); make that first call before any stream capture.
+ *  - Shapes whose prefix-pass scratch exceeds FB_STATIC_SCRATCH_BYTES are
+ *    rejected with FB_ERR_WORKSPACE before any launch.  The limit applies to the
+ *    split-KV scratch of the prefix pass alone -- what fb_prefix_attn itself uses
+ *    for the shape -- which can be smaller than fb_workspace_bytes(shape): that
+ *    figure also covers the in-block rows of the fused step (fb_step).
+ *  - Each call looks up the array's device address with the current device
+ *    (a host-side query, so nothing goes stale after a device reset).  The first
+ *    call on a device may load the library's device code: make it before any
+ *    stream capture.
  *  - All calls on a device share the one array, and it keeps the last call's
  *    contents: each call first clears the arrival counters it needs on `stream`.
  *    Calls that overlap on the GPU (other streams, other threads) race on the
