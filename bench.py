@@ -51,6 +51,35 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+_READ_PEAK = {}
+
+
+def read_peak_gbs(dev, gib: int = 4, reps: int = 5):
+    """Read-only streaming bandwidth of this GPU, measured here: a sum over `gib` GiB
+    of fp32 (torch's reduction kernel, 16-byte loads), best of `reps` with the events
+    on the current stream.  A kernel that only reads (the prefix pass) can exceed the
+    copy bandwidth of MEASURED_PEAKS.json, whose bytes are half writes; this figure
+    is reported beside it, not instead of it."""
+    key = str(dev)
+    if key in _READ_PEAK:
+        return _READ_PEAK[key]
+    x = torch.ones((gib << 28,), device=dev, dtype=torch.float32)
+    out = torch.empty((), device=dev, dtype=torch.float32)
+    torch.sum(x, dim=0, out=out)
+    best = 0.0
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch.sum(x, dim=0, out=out)
+        e1.record()
+        torch.cuda.synchronize()
+        best = max(best, x.numel() * 4 / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    del x
+    torch.cuda.empty_cache()
+    _READ_PEAK[key] = best
+    return best
+
+
 def tensor_roofline(tflops: float) -> dict:
     """Tensor roofline of a step whose launch is timed alone (L2 flushed between
     steps): against the measured burst cuBLAS bf16 figure, with the sustained one
@@ -86,8 +115,13 @@ def kernel_source_hash(kernel: Optional[str] = None) -> str:
 
 def ncu_traffic(workload: str):
     """DRAM bytes per launch of the profiled kernel from the committed ncu summary,
-    or None when the summary is absent or was taken on other sources of that kernel."""
-    path = os.path.join(ROOT, "profiles", f"prefix_pass_{workload}.md")
+    or None when the summary is absent or was taken on other sources of that kernel.
+    A long-context length without its own summary takes the long_200k capture scaled
+    by the algorithmic bytes of a recompute launch (the traffic is the prefix K/V
+    read once, so it grows in proportion)."""
+    own = os.path.join(ROOT, "profiles", f"prefix_pass_{workload}.md")
+    ref = "long_200k" if workload.startswith("long_") else workload
+    path = own if os.path.exists(own) else os.path.join(ROOT, "profiles", f"prefix_pass_{ref}.md")
     if not os.path.exists(path):
         return None
     vals = {}
@@ -99,9 +133,12 @@ def ncu_traffic(workload: str):
     if kernel not in KERNEL_SOURCES or vals.get("kernel_source_sha") != kernel_source_hash(kernel):
         return None
     try:
-        return float(vals["dram_bytes_per_launch"])
+        traffic = float(vals["dram_bytes_per_launch"])
     except (KeyError, ValueError):
         return None
+    if path != own:
+        traffic *= step_bytes(W.get(workload))[0] / step_bytes(W.get(ref))[0]
+    return traffic
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -575,6 +612,7 @@ def device_arm(args, rank, world, w: Optional[W.Workload] = None, kv=None, extra
         sim_gbs = 2 * qa.numel() * qa.element_size() / (sim_us * 1e-6) / 1e9
 
     reuse_batched = batched_reuse(fb, w, flush) if extras else None
+    read_peak = read_peak_gbs(dev)
     reuse_ms = [step_ms[i] for i in reuse_steps]
     roofline_reuse = None
     if reuse_ms and not dw.losa:
@@ -607,6 +645,7 @@ def device_arm(args, rank, world, w: Optional[W.Workload] = None, kv=None, extra
                       frac=(achieved / hbm) if achieved else None,
                       peak_source=f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
                       frac_of_8tbs=(achieved / 8000.0) if achieved else None,
+                      read_peak=read_peak, frac_of_read_peak=(achieved / read_peak) if achieved else None,
                       alg_bytes_per_launch=alg, launches=len(rec_ms),
                       avg_launch_us=(sum(rec_ms) / len(rec_ms) * 1e3) if rec_ms else None,
                       traffic=traffic),
@@ -860,7 +899,8 @@ def sweep_entry(r: dict) -> dict:
         workload=r["config"]["workload"], n_prefix=r["config"]["n_prefix"], steps_per_s=r["value"],
         ms_per_step=r["ms_per_step"], steps=r["steps"],
         roofline=dict(achieved=rf["achieved"], peak=rf["peak"], unit=rf["unit"], frac=rf["frac"],
-                      frac_of_8tbs=rf.get("frac_of_8tbs"), alg_bytes_per_launch=rf["alg_bytes_per_launch"],
+                      frac_of_8tbs=rf.get("frac_of_8tbs"), frac_of_read_peak=rf.get("frac_of_read_peak"),
+                      alg_bytes_per_launch=rf["alg_bytes_per_launch"],
                       launches=rf["launches"], avg_launch_us=rf["avg_launch_us"], traffic=rf.get("traffic")),
         roofline_reuse=bd.get("roofline_reuse"),
         recompute_steps=bd["recompute_steps"], reuse_steps=bd["reuse_steps"],

@@ -49,9 +49,10 @@ __global__ void __launch_bounds__(kSmallThreads) small_block_kernel(const SmallB
       if (a.dec_M && h == 0) a.dec_M[b] = M;
     }
   }
+  extern __shared__ __align__(16) uint8_t tile_smem[];  // bf16: a tile memory per warp
   inblock_rows<T, D>(d, static_cast<const T*>(a.q), static_cast<const T*>(a.k_blk),
                      static_cast<const T*>(a.v_blk), b, kvh, (h - kvh * d.G) * d.B, 0, d.B, a.ep, tid >> 5,
-                     kSmallThreads / 32, tid & 31);
+                     kSmallThreads / 32, tid & 31, tile_smem);
 }
 
 __global__ void gate_kernel(const Dims d, const GateParams g, int32_t* dec_M, uint8_t* dec_reuse) {
@@ -145,17 +146,35 @@ __global__ void append_block_kernel(const Dims d, uint8_t* k_cache, uint8_t* v_c
   }
 }
 
+template <typename T, int DC>
+cudaError_t launch_small_dc(const SmallBlockArgs& a, const dim3& grid, cudaStream_t s) {
+  // bf16 takes a tensor-core tile memory per warp (dynamic shared memory)
+  constexpr size_t smem = std::is_same<T, __nv_bfloat16>::value ? (kSmallThreads / 32) * TileSmem<32 * DC>::kBytes : 0;
+  if (smem > 48 * 1024) {
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(small_block_kernel<T, DC>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+      if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+  }
+  small_block_kernel<T, DC><<<grid, kSmallThreads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t launch_small_t(const SmallBlockArgs& a, cudaStream_t s) {
   dim3 grid(a.d.hq, a.d.b);
   switch (a.d.D / 32) {
-    case 1: small_block_kernel<T, 1><<<grid, kSmallThreads, 0, s>>>(a); break;
-    case 2: small_block_kernel<T, 2><<<grid, kSmallThreads, 0, s>>>(a); break;
-    case 3: small_block_kernel<T, 3><<<grid, kSmallThreads, 0, s>>>(a); break;
-    case 4: small_block_kernel<T, 4><<<grid, kSmallThreads, 0, s>>>(a); break;
+    case 1: return launch_small_dc<T, 1>(a, grid, s);
+    case 2: return launch_small_dc<T, 2>(a, grid, s);
+    case 3: return launch_small_dc<T, 3>(a, grid, s);
+    case 4: return launch_small_dc<T, 4>(a, grid, s);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace

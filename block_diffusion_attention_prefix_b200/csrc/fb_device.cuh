@@ -13,6 +13,8 @@
 #include <cuda_runtime.h>
 #include <math_constants.h>
 
+#include <type_traits>
+
 #include "fb_internal.h"
 #include "fb_ptx.cuh"
 
@@ -233,26 +235,55 @@ __device__ __forceinline__ void load_vec(const __nv_bfloat16* p, float (&x)[DC])
   }
 }
 
+// Store DC consecutive floats (as fp32, or rounded to bf16) with one vector store
+// where the width allows (the caller's offset is DC-element aligned).
+template <int DC>
+__device__ __forceinline__ void store_vec(float* p, const float (&x)[DC]) {
+  if constexpr (DC == 4) {
+    *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+  } else if constexpr (DC == 2) {
+    *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
+  } else {
+#pragma unroll
+    for (int t = 0; t < DC; ++t) p[t] = x[t];
+  }
+}
+template <int DC>
+__device__ __forceinline__ void store_vec(__nv_bfloat16* p, const float (&x)[DC]) {
+  if constexpr (DC == 4) {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(x[0], x[1]), hi = __floats2bfloat162_rn(x[2], x[3]);
+    uint2 u;
+    u.x = *reinterpret_cast<const uint32_t*>(&lo);
+    u.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(p) = u;
+  } else if constexpr (DC == 2) {
+    *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(x[0], x[1]);
+  } else {
+#pragma unroll
+    for (int t = 0; t < DC; ++t) p[t] = __float2bfloat16_rn(x[t]);
+  }
+}
+
 // In-block attention of one query row by one warp (FlashBlock "Core mechanism":
 // A_in over J_in, the B tokens of the current block, bidirectional; fp32 math).
-// Lane l owns dims [l*DC, l*DC + DC).  Keys go in chunks of 8 whose dot products
+// Lane l owns dims [l*DC, l*DC + DC).  Keys go in chunks of KC whose dot products
 // are reduced across the warp together (independent butterflies), with an online
 // softmax across chunks.  Returns L_in (natural log); `a` gets the lane's dims of
 // the normalised A_in.  `kb` / `vb` point at the KV group's [B][D] block keys.
-template <typename T, int D>
-__device__ __forceinline__ float inblock_row(const T* qrow, const T* kb, const T* vb, int B, float scale,
-                                             float (&a)[D / 32], int lane) {
+template <typename T, int D, int KC>
+__device__ __forceinline__ float inblock_row_kc(const T* qrow, const T* kb, const T* vb, int B, float scale,
+                                                float (&a)[D / 32], int lane) {
   constexpr int DC = D / 32;
   float q[DC];
   load_vec<DC>(qrow + lane * DC, q);
   float m = -CUDART_INF_F, l = 0.f, acc[DC];
 #pragma unroll
   for (int t = 0; t < DC; ++t) acc[t] = 0.f;
-  for (int j0 = 0; j0 < B; j0 += 8) {
-    const int nj = min(8, B - j0);
-    float s[8], v[8][DC];
+  for (int j0 = 0; j0 < B; j0 += KC) {
+    const int nj = min(KC, B - j0);
+    float s[KC], v[KC][DC];
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
+    for (int jj = 0; jj < KC; ++jj) {
       s[jj] = 0.f;
 #pragma unroll
       for (int t = 0; t < DC; ++t) v[jj][t] = 0.f;
@@ -267,11 +298,11 @@ __device__ __forceinline__ float inblock_row(const T* qrow, const T* kb, const T
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) s[jj] += __shfl_xor_sync(0xffffffffu, s[jj], o);
+      for (int jj = 0; jj < KC; ++jj) s[jj] += __shfl_xor_sync(0xffffffffu, s[jj], o);
     }
     float cm = -CUDART_INF_F;
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
+    for (int jj = 0; jj < KC; ++jj) {
       s[jj] = jj < nj ? s[jj] * scale : -CUDART_INF_F;
       cm = fmaxf(cm, s[jj]);
     }
@@ -281,7 +312,7 @@ __device__ __forceinline__ float inblock_row(const T* qrow, const T* kb, const T
 #pragma unroll
     for (int t = 0; t < DC; ++t) acc[t] *= alpha;
 #pragma unroll
-    for (int jj = 0; jj < 8; ++jj) {
+    for (int jj = 0; jj < KC; ++jj) {
       const float p = jj < nj ? expf(s[jj] - mn) : 0.f;
       l += p;
 #pragma unroll
@@ -294,6 +325,275 @@ __device__ __forceinline__ float inblock_row(const T* qrow, const T* kb, const T
   for (int t = 0; t < DC; ++t) a[t] = acc[t] * inv;
   return m + logf(l);
 }
+
+// In-block row with chunks of 8 keys.  Blocks of at most 4 keys take chunks of 4:
+// the same result bit for bit (a chunk's unused key slots add exact zeros to the
+// row sum and the accumulators, and -inf to the chunk max), with half the shuffles.
+template <typename T, int D>
+__device__ __forceinline__ float inblock_row(const T* qrow, const T* kb, const T* vb, int B, float scale,
+                                             float (&a)[D / 32], int lane) {
+  if (B <= 4) return inblock_row_kc<T, D, 4>(qrow, kb, vb, B, scale, a, lane);
+  return inblock_row_kc<T, D, 8>(qrow, kb, vb, B, scale, a, lane);
+}
+
+// ---------------------------------------------------------------------------
+// In-block attention on the tensor cores (bf16): 16 query rows of one KV group by
+// one warp.  FlashBlock "Core mechanism": (A_in, L_in) over J_in, the B tokens of
+// the current block, bidirectional.  The operands are staged in the warp's own
+// shared memory with coalesced 16-byte async copies (one pass over the 16 query
+// rows, then the keys and values 16 at a time), and mma.sync m16n8k16 (bf16
+// operands, fp32 accumulation) reads them with ldmatrix:
+//   S = Q K^T over D in k16 steps, keys in chunks of 16 (two n8 tiles);
+//   online softmax across the chunks in fp32, base 2 (scale * log2 e folded in),
+//   keys past B masked; the running max m, sum l and the output are rescaled by
+//   2^(m_old - m_new) when a chunk raises the max;
+//   O += P V with P split into bf16 hi and lo parts (P = hi + lo to about 2^-17),
+//   two products per step, so the rounding of P to bf16 costs no accuracy;
+//   A_in = O / l, L_in = (m + log2 l) ln 2.
+// Each row's result depends only on that row's query and the block's keys and
+// values (the MMA computes each output element the same way for every row, and the
+// row reductions run inside the row's thread quad), so every caller that covers a
+// row with any 16-row tile gets the same bits.
+// Output, accumulator layout: thread (g = lane / 4, c = lane % 4) holds for d-tile n
+// o[n][0..1] = A_in[row g][8n + 2c, +1] and o[n][2..3] = the same of row g + 8, and
+// L[0] / L[1] = L_in of rows g / g + 8 (tile rows).
+
+// One warp's shared memory for in-block tiles: 16 staged query rows, 16 keys, 16
+// values (bf16 rows padded to D + 8 elements: 16-byte aligned, ldmatrix without bank
+// conflicts) and 16 cached rows of D + 4 floats (the merge of mode 1).
+template <int D>
+struct TileSmem {
+  static constexpr int kRow = D + 8;                       // bf16 elements per staged row
+  static constexpr int kQOff = 0;                          // bytes
+  static constexpr int kKOff = kQOff + 16 * kRow * 2;
+  static constexpr int kVOff = kKOff + 16 * kRow * 2;
+  static constexpr int kCacheOff = kVOff + 16 * kRow * 2;
+  static constexpr int kBytes = kCacheOff + 16 * (D + 4) * 4;
+  static constexpr int kOperandBytes = kCacheOff;  // enough for callers that merge nothing (to_ws, mode 0)
+  static_assert(kBytes % 16 == 0 && kOperandBytes % 16 == 0, "16-byte aligned regions");
+};
+
+// 16 rows [row0, row0 + 16) of a [n][D] bf16 array into a staged [16][D + 8] tile;
+// rows >= n are zero-filled.  Asynchronous (cp.async); the caller waits.
+template <int D>
+__device__ __forceinline__ void stage_rows16(__nv_bfloat16* dst, const __nv_bfloat16* src, int row0, int n,
+                                             int lane) {
+  constexpr int kChunks = D / 8;  // 16-byte chunks per row
+  for (int i = lane; i < 16 * kChunks; i += 32) {
+    const int r = i / kChunks, c = i - r * kChunks;
+    const bool valid = row0 + r < n;
+    const __nv_bfloat16* g = src + (size_t)(valid ? row0 + r : 0) * D + c * 8;
+    cp_async16_zfill(dst + r * TileSmem<D>::kRow + c * 8, g, valid);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void inblock_tile_tc(const __nv_bfloat16* q, int R, int row0, const __nv_bfloat16* kb,
+                                                const __nv_bfloat16* vb, int B, float scale, float (&o)[D / 8][4],
+                                                float (&L)[2], int lane, uint8_t* wsm) {
+  using TS = TileSmem<D>;
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(wsm + TS::kQOff);
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(wsm + TS::kKOff);
+  __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(wsm + TS::kVOff);
+  const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+  const int c = lane & 3;
+  __syncwarp();  // the warp's previous reads of its tile memory are done
+  stage_rows16<D>(sQ, q, row0, R, lane);
+  const float sl2 = scale * 1.4426950408889634f;
+  float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  uint32_t qf[D / 16][4];
+  for (int k0 = 0; k0 < B; k0 += 16) {
+    if (k0 > 0) __syncwarp();  // the previous chunk's reads of sK / sV are done
+    stage_rows16<D>(sK, kb, k0, B, lane);
+    stage_rows16<D>(sV, vb, k0, B, lane);
+    cp_async_wait_all();
+    __syncwarp();
+    if (k0 == 0) {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        ldsm_x4(aQ + (uint32_t)(((lane & 15) * TS::kRow + kk * 16 + (lane >> 4) * 8) * 2), qf[kk][0], qf[kk][1],
+                qf[kk][2], qf[kk][3]);
+    }
+    // S for this chunk's 16 keys (n-tiles 0: keys k0..k0+7, 1: k0+8..k0+15)
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      uint32_t b0, b1, b2, b3;
+      const int key = (lane & 7) + ((lane >> 4) << 3);
+      const int col = kk * 16 + ((lane >> 3) & 1) * 8;
+      ldsm_x4(aK + (uint32_t)((key * TS::kRow + col) * 2), b0, b1, b2, b3);
+      mma_bf16_16816_free(s[0], qf[kk], b0, b1);
+      mma_bf16_16816_free(s[1], qf[kk], b2, b3);
+    }
+    float cm0 = -CUDART_INF_F, cm1 = -CUDART_INF_F;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int key = k0 + j * 8 + 2 * c + (e & 1);
+        const float v = key < B ? s[j][e] * sl2 : -CUDART_INF_F;
+        s[j][e] = v;
+        if (e < 2) cm0 = fmaxf(cm0, v); else cm1 = fmaxf(cm1, v);
+      }
+    }
+    cm0 = fmaxf(cm0, __shfl_xor_sync(0xffffffffu, cm0, 1));
+    cm0 = fmaxf(cm0, __shfl_xor_sync(0xffffffffu, cm0, 2));
+    cm1 = fmaxf(cm1, __shfl_xor_sync(0xffffffffu, cm1, 1));
+    cm1 = fmaxf(cm1, __shfl_xor_sync(0xffffffffu, cm1, 2));
+    const float n0 = fmaxf(m0, cm0), n1 = fmaxf(m1, cm1);  // every chunk has a valid key: finite
+    const float al0 = ex2_approx(m0 - n0), al1 = ex2_approx(m1 - n1);  // 0 on the first chunk
+    float cs0 = 0.f, cs1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      s[j][0] = ex2_approx(s[j][0] - n0);
+      s[j][1] = ex2_approx(s[j][1] - n0);
+      s[j][2] = ex2_approx(s[j][2] - n1);
+      s[j][3] = ex2_approx(s[j][3] - n1);
+      cs0 += s[j][0] + s[j][1];
+      cs1 += s[j][2] + s[j][3];
+    }
+    cs0 += __shfl_xor_sync(0xffffffffu, cs0, 1);
+    cs0 += __shfl_xor_sync(0xffffffffu, cs0, 2);
+    cs1 += __shfl_xor_sync(0xffffffffu, cs1, 1);
+    cs1 += __shfl_xor_sync(0xffffffffu, cs1, 2);
+    l0 = l0 * al0 + cs0;
+    l1 = l1 * al1 + cs1;
+    m0 = n0;
+    m1 = n1;
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) {
+      o[n][0] *= al0;
+      o[n][1] *= al0;
+      o[n][2] *= al1;
+      o[n][3] *= al1;
+    }
+    // O += P V, P = hi + lo in bf16
+    uint32_t hi[4], lo[4];
+    {
+      const float pv[8] = {s[0][0], s[0][1], s[0][2], s[0][3], s[1][0], s[1][1], s[1][2], s[1][3]};
+      float rest[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) rest[e] = pv[e] - __bfloat162float(__float2bfloat16_rn(pv[e]));
+      hi[0] = pack_bf16x2(pv[0], pv[1]);
+      hi[1] = pack_bf16x2(pv[2], pv[3]);
+      hi[2] = pack_bf16x2(pv[4], pv[5]);
+      hi[3] = pack_bf16x2(pv[6], pv[7]);
+      lo[0] = pack_bf16x2(rest[0], rest[1]);
+      lo[1] = pack_bf16x2(rest[2], rest[3]);
+      lo[2] = pack_bf16x2(rest[4], rest[5]);
+      lo[3] = pack_bf16x2(rest[6], rest[7]);
+    }
+#pragma unroll
+    for (int dn = 0; dn < D / 8; dn += 2) {
+      uint32_t b0, b1, b2, b3;
+      const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int col = dn * 8 + (lane >> 4) * 8;
+      ldsm_x4_t(aV + (uint32_t)((key * TS::kRow + col) * 2), b0, b1, b2, b3);
+      mma_bf16_16816_free(o[dn], hi, b0, b1);
+      mma_bf16_16816_free(o[dn], lo, b0, b1);
+      mma_bf16_16816_free(o[dn + 1], hi, b2, b3);
+      mma_bf16_16816_free(o[dn + 1], lo, b2, b3);
+    }
+  }
+  const float i0 = 1.f / l0, i1 = 1.f / l1;
+#pragma unroll
+  for (int n = 0; n < D / 8; ++n) {
+    o[n][0] *= i0;
+    o[n][1] *= i0;
+    o[n][2] *= i1;
+    o[n][3] *= i1;
+  }
+  L[0] = (m0 + __log2f(l0)) * 0.6931471805599453f;
+  L[1] = (m1 + __log2f(l1)) * 0.6931471805599453f;
+}
+
+// The in-block rows [r_begin, r_end) of KV group (b, kvh) (group rows, 0 .. G*B),
+// computed on the tensor cores in 16-row tiles by warps [warp, nwarps); for each
+// tile row r that `keep(r)` accepts, the threads holding it write their columns.
+// `wsm`: this warp's TileSmem<D>::kBytes of shared memory (16-byte aligned).  In
+// mode 1 the tile's cached rows are copied there asynchronously while the tile is
+// computed.  Modes:
+//   to_ws: (A_in, L_in) into slot rows r - slot_row0 ([.][D + 4] fp32, L at col D);
+//   ep mode 0: (A_in, L_in) into ep.a_dst / ep.l_dst;
+//   ep mode 1: A_full = merge(cache row, in-block row) into ep.a_full / ep.l_full.
+struct TileOut {
+  int kind;            // 0: workspace slot, 1: epilogue
+  float* slot;         // kind 0
+  int slot_row0;       // kind 0: group row of slot row 0
+  Epilogue ep;         // kind 1
+};
+
+template <int D, typename Keep>
+__device__ void inblock_rows_tc(const Dims& d, const __nv_bfloat16* q, const __nv_bfloat16* k_blk,
+                                const __nv_bfloat16* v_blk, int b, int kvh, int r_begin, int r_end,
+                                const TileOut& out, Keep keep, int warp, int nwarps, int lane, uint8_t* wsm) {
+  using TS = TileSmem<D>;
+  const __nv_bfloat16* kb = k_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
+  const __nv_bfloat16* vb = v_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
+  const size_t grow_base = (size_t)(b * d.hq + kvh * d.G) * d.B;  // global row of group row 0
+  const __nv_bfloat16* qg = q + grow_base * D;
+  float* sC = reinterpret_cast<float*>(wsm + TS::kCacheOff);
+  const int g = lane >> 2, c = lane & 3;
+  for (int t0 = r_begin + warp * 16; t0 < r_end; t0 += nwarps * 16) {
+    const bool merge = out.kind == 1 && out.ep.mode == 1;
+    if (merge) {
+      // the tile's cached rows are needed after the in-block math: copy them now
+      __syncwarp();  // the previous tile's reads of sC are done
+      const int nr = min(16, r_end - t0);
+      for (int i = lane; i < nr * (D / 4); i += 32) {
+        const int rr = i / (D / 4), c4 = i - rr * (D / 4);
+        cp_async16(sC + rr * (D + 4) + c4 * 4, out.ep.a_prev + (grow_base + t0 + rr) * D + c4 * 4);
+      }
+      for (int rr = lane; rr < nr; rr += 32) cp_async4(sC + rr * (D + 4) + D, out.ep.l_prev + grow_base + t0 + rr);
+    }
+    float o[D / 8][4], L[2];
+    inblock_tile_tc<D>(qg, min(r_end, d.R), t0, kb, vb, d.B, d.scale, o, L, lane, wsm);
+    if (merge) {
+      cp_async_wait_all();
+      __syncwarp();
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = t0 + g + 8 * h;
+      if (r >= r_end || !keep(r)) continue;
+      const size_t grow = grow_base + r;
+      if (out.kind == 0) {
+        float* dst = out.slot + (size_t)(r - out.slot_row0) * (D + 4);
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n)
+          *reinterpret_cast<float2*>(dst + n * 8 + 2 * c) = make_float2(o[n][2 * h], o[n][2 * h + 1]);
+        if (c == 0) dst[D] = L[h];
+      } else if (out.ep.mode == 0) {
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n)
+          *reinterpret_cast<float2*>(out.ep.a_dst + grow * D + n * 8 + 2 * c) =
+              make_float2(o[n][2 * h], o[n][2 * h + 1]);
+        if (c == 0) out.ep.l_dst[grow] = L[h];
+      } else {
+        const float* srow = sC + (r - t0) * (D + 4);
+        const MergeRow w = merge_row(srow[D], L[h]);
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          const size_t off = grow * D + n * 8 + 2 * c;
+          const float2 ap = *reinterpret_cast<const float2*>(srow + n * 8 + 2 * c);
+          const float v0 = merge_val(w, ap.x, o[n][2 * h]), v1 = merge_val(w, ap.y, o[n][2 * h + 1]);
+          if (out.ep.out_bf16)
+            *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(out.ep.a_full) + off) =
+                __floats2bfloat162_rn(v0, v1);
+          else
+            *reinterpret_cast<float2*>(static_cast<float*>(out.ep.a_full) + off) = make_float2(v0, v1);
+        }
+        if (c == 0 && out.ep.l_full) out.ep.l_full[grow] = w.l;
+      }
+    }
+  }
+}
+
+struct KeepAll {
+  __device__ bool operator()(int) const { return true; }
+};
 
 // One in-block row of a step, by one warp: A_full = merge(cache row, in-block
 // row) (mode 1), or (A_in, L_in) written out (mode 0).  `grow` indexes [b, H_q, B];
@@ -316,30 +616,40 @@ __device__ __forceinline__ void inblock_merge_row(const Dims& d, const T* q, con
   const float L = inblock_row<T, D>(q + grow * D, kb, vb, d.B, d.scale, a, lane);
   const size_t off = grow * D + (size_t)lane * DC;
   if (ep.mode == 0) {
-#pragma unroll
-    for (int t = 0; t < DC; ++t) ep.a_dst[off + t] = a[t];
+    store_vec<DC>(ep.a_dst + off, a);
     if (lane == 0) ep.l_dst[grow] = L;
     return;
   }
   const MergeRow w = merge_row(lp, L);
+  float o[DC];
 #pragma unroll
-  for (int t = 0; t < DC; ++t) {
-    const float v = merge_val(w, ap[t], a[t]);
-    if (ep.out_bf16)
-      static_cast<__nv_bfloat16*>(ep.a_full)[off + t] = __float2bfloat16_rn(v);
-    else
-      static_cast<float*>(ep.a_full)[off + t] = v;
-  }
+  for (int t = 0; t < DC; ++t) o[t] = merge_val(w, ap[t], a[t]);
+  if (ep.out_bf16)
+    store_vec<DC>(static_cast<__nv_bfloat16*>(ep.a_full) + off, o);
+  else
+    store_vec<DC>(static_cast<float*>(ep.a_full) + off, o);
   if (lane == 0 && ep.l_full) ep.l_full[grow] = w.l;
 }
 
 // In-block rows [r_begin, r_end) of tile rows (group rows row0 + r) of KV group
 // (b, kvh), one warp per row (inblock_merge_row), executed by warps [0, nwarps) of
 // the CTA.
+// `tsm` (bf16 only): shared memory of TileSmem<D>::kBytes per warp (warp w uses
+// tsm + w * TileSmem<D>::kBytes) for the tensor-core tiles.
 template <typename T, int D>
 __device__ void inblock_rows(const Dims& d, const T* q, const T* k_blk, const T* v_blk, int b, int kvh,
                              int row0, int r_begin, int r_end, const Epilogue& ep, int warp, int nwarps,
-                             int lane) {
+                             int lane, uint8_t* tsm = nullptr) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {  // bf16: tensor-core tiles
+    TileOut out;
+    out.kind = 1;
+    out.slot = nullptr;
+    out.slot_row0 = 0;
+    out.ep = ep;
+    inblock_rows_tc<D>(d, q, k_blk, v_blk, b, kvh, row0 + r_begin, row0 + r_end, out, KeepAll(), warp, nwarps,
+                       lane, tsm + (size_t)warp * TileSmem<D>::kBytes);
+    return;
+  }
   const T* kb = k_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
   const T* vb = v_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
   const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B + row0;
@@ -348,10 +658,20 @@ __device__ void inblock_rows(const Dims& d, const T* q, const T* k_blk, const T*
 
 // In-block rows [r_begin, r_end) of one tile written as (A_in, L_in) into the
 // tile's [RT][D + 4] fp32 slot of the workspace (the fused step merges them later).
+// `tsm` as for inblock_rows.
 template <typename T, int D>
 __device__ void inblock_rows_to_ws(const Dims& d, const T* q, const T* k_blk, const T* v_blk, int b, int kvh,
                                    int row0, int r_begin, int r_end, float* slot, int warp, int nwarps,
-                                   int lane) {
+                                   int lane, uint8_t* tsm = nullptr) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {  // bf16: tensor-core tiles
+    TileOut out;
+    out.kind = 0;
+    out.slot = slot;
+    out.slot_row0 = row0;
+    inblock_rows_tc<D>(d, q, k_blk, v_blk, b, kvh, row0 + r_begin, row0 + r_end, out, KeepAll(), warp, nwarps,
+                       lane, tsm + (size_t)warp * TileSmem<D>::kBytes);
+    return;
+  }
   constexpr int DC = D / 32;
   const T* kb = k_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
   const T* vb = v_blk + (size_t)(b * d.hkv + kvh) * d.B * D;

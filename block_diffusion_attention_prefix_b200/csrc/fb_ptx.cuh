@@ -158,6 +158,44 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Transpose of an 8x8 b16 matrix held one row pair per thread: thread t gives
+// {M[t/4][2(t%4)], M[t/4][2(t%4)+1]} and gets {M[2(t%4)][t/4], M[2(t%4)+1][t/4]}.
+// A pure register operation (not volatile), so the compiler may schedule the loads
+// that feed it early.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// mma.sync as a pure register operation (not volatile): same instruction as
+// mma_bf16_16816, free for the compiler to schedule around the loads that feed it.
+__device__ __forceinline__ void mma_bf16_16816_free(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                                    uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Asynchronous global -> shared copies of 16 or 4 bytes (cp.async), completed by
+// cp_async_wait_all() in the issuing thread.
+__device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 16;" ::"r"(smem_u32(sdst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* sdst, const void* gsrc) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sdst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// 16-byte async copy that zero-fills the destination when `valid` is false (no bytes
+// are read then; gsrc must still be a valid address).  Through L1 (.ca), so lines
+// an earlier prefetch brought into L1 are served from there.
+__device__ __forceinline__ void cp_async16_zfill(void* sdst, const void* gsrc, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(sdst)), "l"(gsrc),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+
 // 2^x with the hardware approximation (inputs here are <= 0 or -inf).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

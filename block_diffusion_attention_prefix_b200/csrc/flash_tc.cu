@@ -67,7 +67,8 @@ constexpr int kPBytes = 128 * kKT * 2;           // P_w: [128 rows][64 keys] bf1
 constexpr int kQOff = 0;
 constexpr int kStageOff = kQBytes;
 constexpr int kPOff = kStageOff + kStages * kStageBytes;
-constexpr int kSmemBytes = kPOff + 2 * kPBytes + 1024;
+constexpr int kAuxOff = kPOff + 2 * kPBytes;     // the aux warp's in-block tile memory
+constexpr int kSmemBytes = kAuxOff + TileSmem<kD>::kOperandBytes + 1024;
 constexpr int kBufBytes = kSmemBytes - 1024;  // all of it, reused by the split combine
 
 // Shared-memory matrix descriptor, 128-byte swizzle (layout type 2, version 1).
@@ -193,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int r0, r1;
     split_rows(rows_valid, plan.splits, split, r0, r1);
     constexpr int kLinesRow = kD * (int)sizeof(bf16) / 128;  // 128-byte lines per bf16 row
-    const int nq = (r1 - r0) * kLinesRow;
+    const int nq = (min(r0 + 16, d.R - row0) - r0) * kLinesRow;  // the 16-row tile the in-block part stages
     const int nkv = d.B * kLinesRow;  // per tensor
     const int nc = (r1 - r0) * (kD * 4 / 128);
     const bf16* kb = k_blk + (size_t)(b * d.hkv + kvh) * d.B * kD;
@@ -218,8 +219,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (SPLIT && args.step.enabled) {
       int r0, r1;
       split_rows(rows_valid, plan.splits, split, r0, r1);
-      inblock_rows<bf16, kD>(d, q, k_blk, v_blk, b, kvh, row0, r0, r1, step_epilogue(args), warp, kThreads / 32,
-                             lane);
+      constexpr int kTileWarps = 8;  // tile memories that fit the idle shared memory
+      static_assert(kTileWarps * TileSmem<kD>::kBytes <= kSmemBytes - 1024, "tile memory per warp");
+      if (warp < kTileWarps)
+        inblock_rows<bf16, kD>(d, q, k_blk, v_blk, b, kvh, row0, r0, r1, step_epilogue(args), warp, kTileWarps,
+                               lane, smem);  // nothing else uses shared memory here
       if (split == 0)
         record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, s_M, args.step.dec_M,
                          args.step.dec_reuse, kvh == 0 && rt == 0, tid, kThreads);
@@ -325,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int r0, r1;
       split_rows(rows_valid, plan.splits, split, r0, r1);
       inblock_rows_to_ws<bf16, kD>(d, q, k_blk, v_blk, b, kvh, row0, r0, r1, args.inblock + unit * RT * (kD + 4),
-                                   0, 1, lane);
+                                   0, 1, lane, smem + kAuxOff);
     }
   } else {
     // ---------------- softmax warpgroups: one query row per thread ----------------

@@ -63,7 +63,10 @@ struct Cfg {
   static constexpr int kStageBytes = 2 * kTileBytes;  // K then V
   static constexpr int kScratchBytes = kConsumerWarps * 16 * (D + 2) * 4;
   static constexpr int kRingBytes = STAGES * kStageBytes;
-  static constexpr int kSmemBytes = (kRingBytes > kScratchBytes ? kRingBytes : kScratchBytes) + 1024;
+  // the aux warp's in-block tile memory, past the ring (which is busy while it works)
+  static constexpr int kAuxOff = kRingBytes > kScratchBytes ? kRingBytes : kScratchBytes;
+  static constexpr int kSmemBytes = kAuxOff + TileSmem<D>::kOperandBytes + 1024;
+  static_assert(kConsumerWarps + 2 <= kRingBytes / TileSmem<D>::kBytes, "reuse path: a tile memory per warp");
   static_assert(KW % 16 == 0, "each warp needs whole k16 steps of keys");
   static_assert(D % 64 == 0, "D must be a multiple of 64");
   // The combine stages (rows x (splits + 1)) partial rows, rows <= ceil(RT / splits):
@@ -126,7 +129,7 @@ __device__ __forceinline__ bool pass_unit(const CUtensorMap* tmK, const CUtensor
     int r0, r1;
     split_rows(rows_valid, plan.splits, split, r0, r1);
     const int lines_row = D * (int)sizeof(bf16) / 128;  // 128-byte lines per bf16 row
-    const int nq = (r1 - r0) * lines_row;
+    const int nq = (min(r0 + 16, d.R - row0) - r0) * lines_row;  // the 16-row tile the in-block part stages
     const int nkv = d.B * lines_row;  // per tensor
     const int nc = (r1 - r0) * (D * 4 / 128);
     const bf16* kb = k_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
@@ -153,7 +156,7 @@ __device__ __forceinline__ bool pass_unit(const CUtensorMap* tmK, const CUtensor
       int r0, r1;
       split_rows(rows_valid, plan.splits, split, r0, r1);
       inblock_rows<bf16, D>(d, q, k_blk, v_blk, b, kvh, row0, r0, r1, step_epilogue(args), warp, C::kThreads / 32,
-                            lane);
+                            lane, smem);  // the ring is idle: a tile memory per warp
       if (split == 0)
         record_decisions(args.gate, d, b, kvh, row0, rows_valid, s_flags, sh.M, args.step.dec_M,
                          args.step.dec_reuse, kvh == 0 && rt == 0, tid, C::kThreads);
@@ -215,7 +218,7 @@ __device__ __forceinline__ bool pass_unit(const CUtensorMap* tmK, const CUtensor
       int r0, r1;
       split_rows(rows_valid, plan.splits, split, r0, r1);
       inblock_rows_to_ws<bf16, D>(d, q, k_blk, v_blk, b, kvh, row0, r0, r1, args.inblock + unit * RT * (D + 4),
-                                  0, 1, lane);
+                                  0, 1, lane, smem + C::kAuxOff);
     }
   } else {
     // ---------------------------- consumer warps ----------------------------

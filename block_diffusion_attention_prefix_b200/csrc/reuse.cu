@@ -9,14 +9,21 @@
 // When one call carries many independent (b, KV head) groups -- the batch of a
 // serving step, or every layer of a model stacked on the batch axis -- the pass
 // kernel's one-CTA-per-SM shared-memory ring would hold a whole SM per reusing
-// tile.  This kernel instead runs a group per CTA with no dynamic shared memory, so
-// several CTAs (and a warp per row) share each SM and the rows' loads overlap:
-// the gate, the decision record (dec_M, dec_reuse), and for every reusing row the
-// in-block attention merged with its cached row, in the same arithmetic as the
-// pass kernels' fused epilogue (inblock_merge_row), so the results agree bit for
-// bit.  Rows that recompute are left to the prefix pass that follows.
+// tile.  These kernels instead need no dynamic shared memory: the gate, the
+// decision record (dec_M, dec_reuse), and for every reusing row the in-block
+// attention merged with its cached row, in the same arithmetic as the pass kernels'
+// fused epilogue, so the results agree bit for bit.  Rows that recompute are left to
+// the prefix pass that follows.
+//  * bf16 (reuse_tiles_kernel): a warp per 16-row tile of a group, the in-block
+//    part on the tensor cores (inblock_rows_tc), four tiles per CTA and three CTAs
+//    per SM; each warp
+//    first pulls its tile's rows into L1 so one DRAM latency covers the tile.
+//  * fp32 (reuse_rows_kernel): a CTA per group, a warp per row on CUDA cores
+//    (inblock_merge_row), three CTAs per SM.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <type_traits>
 
 #include "fb_device.cuh"
 #include "fb_internal.h"
@@ -82,9 +89,84 @@ __global__ void __launch_bounds__(kReuseThreads, 3) reuse_rows_kernel(const Pass
   }
 }
 
+constexpr int kTileWarps = 4;
+
+template <int D>
+__global__ void __launch_bounds__(kTileWarps * 32, 3) reuse_tiles_kernel(const PassArgs args, long long items) {
+  using bf16 = __nv_bfloat16;
+  const Dims& d = args.d;
+  const GateParams& g = args.gate;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles = (d.R + 15) >> 4;
+  const long long item = (long long)blockIdx.x * kTileWarps + warp;
+  if (item >= items) return;
+  const int bg = (int)(item / tiles), t = (int)(item - (long long)bg * tiles);
+  const int b = bg / d.hkv, kvh = bg - b * d.hkv;
+  const int r0 = t * 16, r1 = min(d.R, r0 + 16);
+  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B;
+  {
+    // the tile's q rows, cached rows and L, and the group's block K/V into L1 while
+    // the gate reads the mask (every address inside its buffer)
+    const char* base[5] = {reinterpret_cast<const char*>(static_cast<const bf16*>(args.q) + (grow0 + r0) * D),
+                           reinterpret_cast<const char*>(args.ep.a_dst + (grow0 + r0) * D),
+                           reinterpret_cast<const char*>(args.ep.l_dst + grow0 + r0),
+                           reinterpret_cast<const char*>(static_cast<const bf16*>(args.step.k_blk) + (size_t)bg * d.B * D),
+                           reinterpret_cast<const char*>(static_cast<const bf16*>(args.step.v_blk) + (size_t)bg * d.B * D)};
+    const size_t bytes[5] = {(size_t)(r1 - r0) * D * 2, (size_t)(r1 - r0) * D * 4, (size_t)(r1 - r0) * 4,
+                             (size_t)d.B * D * 2, (size_t)d.B * D * 2};
+#pragma unroll
+    for (int k = 0; k < 5; ++k) {
+      const int lines = (int)((bytes[k] + 127) / 128);
+      for (int i = lane; i <= lines; i += 32) prefetch_l1(base[k] + (i < lines ? (size_t)i * 128 : bytes[k] - 1));
+    }
+  }
+  int cnt = 0;
+  for (int i = lane; i < d.B; i += 32) cnt += g.mask[(size_t)b * d.B + i] != 0;
+  const int M = warp_sum_int(cnt);
+  const bool tau_ok = tau_reuse(g, M);
+  if (t == 0) {
+    if (kvh == 0 && lane == 0 && args.step.dec_M) args.step.dec_M[b] = M;
+    if (args.step.dec_reuse)
+      for (int j = lane; j < d.G; j += 32)
+        args.step.dec_reuse[(size_t)b * d.hq + kvh * d.G + j] = head_reuse(g, tau_ok, b, d.hq, kvh * d.G + j) ? 1 : 0;
+  }
+  if (!tau_ok) return;  // every head of this batch element recomputes: the prefix pass writes its rows
+  TileOut out;
+  out.kind = 1;
+  out.slot = nullptr;
+  out.slot_row0 = 0;
+  out.ep.mode = 1;
+  out.ep.a_dst = nullptr;
+  out.ep.l_dst = nullptr;
+  out.ep.a_prev = args.ep.a_dst;  // the cache
+  out.ep.l_prev = args.ep.l_dst;
+  out.ep.a_full = args.step.a_full;
+  out.ep.l_full = args.step.l_full;
+  out.ep.out_bf16 = 1;
+  auto keep = [&](int r) { return head_reuse(g, true, b, d.hq, kvh * d.G + r / d.B); };
+  extern __shared__ __align__(16) uint8_t tile_smem[];  // a tile memory per warp
+  inblock_rows_tc<D>(d, static_cast<const bf16*>(args.q), static_cast<const bf16*>(args.step.k_blk),
+                     static_cast<const bf16*>(args.step.v_blk), b, kvh, r0, r1, out, keep, 0, 1, lane,
+                     tile_smem + (size_t)warp * TileSmem<D>::kBytes);
+}
+
 template <typename T, int D>
 cudaError_t launch_typed(const PassArgs& a, cudaStream_t s) {
-  reuse_rows_kernel<T, D><<<(unsigned)(a.d.b * a.d.hkv), kReuseThreads, 0, s>>>(a);
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+    const long long items = (long long)a.d.b * a.d.hkv * ((a.d.R + 15) / 16);
+    constexpr int smem = kTileWarps * TileSmem<D>::kBytes;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+      const cudaError_t e = cudaFuncSetAttribute(reuse_tiles_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return e;
+      if (dev >= 0 && dev < 64) attr_set[dev] = true;
+    }
+    reuse_tiles_kernel<D><<<(unsigned)((items + kTileWarps - 1) / kTileWarps), kTileWarps * 32, smem, s>>>(a, items);
+  } else {
+    reuse_rows_kernel<T, D><<<(unsigned)(a.d.b * a.d.hkv), kReuseThreads, 0, s>>>(a);
+  }
   return cudaGetLastError();
 }
 

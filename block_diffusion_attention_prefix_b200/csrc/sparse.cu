@@ -463,7 +463,9 @@ struct SCfg {
   static constexpr int kStageBytes = 2 * kTileBytes;       // K then V
   static constexpr int kScratchBytes = kConsumerWarps * 16 * (D + 2) * 4 * 2;  // sel and res
   static constexpr int kRingBytes = STAGES * kStageBytes;
-  static constexpr int kSmemBytes = (kRingBytes > kScratchBytes ? kRingBytes : kScratchBytes) + 1024;
+  // the aux warp's in-block tile memory, past the ring (which is busy while it works)
+  static constexpr int kAuxOff = kRingBytes > kScratchBytes ? kRingBytes : kScratchBytes;
+  static constexpr int kSmemBytes = kAuxOff + TileSmem<D>::kOperandBytes + 1024;
   static_assert(KW % 16 == 0, "whole k16 steps per warp");
   // The split combine stages rows x (2 splits + 1) partial rows (rows <= ceil(RT / splits)):
   // at most 2 (2 RT + 149) + RT rows for up to 148 splits (it reads the workspace otherwise).
@@ -1082,7 +1084,7 @@ __global__ void __launch_bounds__(SCfg<D, WARPS_M, WARPS_N, STAGES>::kThreads, 1
     const int r0 = min(rows_valid, split * per), r1 = min(rows_valid, r0 + per);
     inblock_rows_to_ws<bf16, D>(d, q, static_cast<const bf16*>(args.step.k_blk),
                                 static_cast<const bf16*>(args.step.v_blk), b, kvh, row0, r0, r1,
-                                args.inblock + unit * RT * rs, 0, 1, lane);
+                                args.inblock + unit * RT * rs, 0, 1, lane, smem + C::kAuxOff);
   } else {
     // ---------------------------- consumers ----------------------------
     const int wm = warp / WARPS_N, wn = warp - (warp / WARPS_N) * WARPS_N;
