@@ -387,27 +387,41 @@ __device__ __forceinline__ void stage_rows16(__nv_bfloat16* dst, const __nv_bflo
   }
 }
 
+// The first copies of a tile: its 16 query rows and the block's first 16 keys and
+// values, into the warp's tile memory (asynchronous).
+template <int D>
+__device__ __forceinline__ void inblock_tile_stage(const __nv_bfloat16* q, int R, int row0, const __nv_bfloat16* kb,
+                                                   const __nv_bfloat16* vb, int B, int lane, uint8_t* wsm) {
+  using TS = TileSmem<D>;
+  __syncwarp();  // the warp's previous reads of its tile memory are done
+  stage_rows16<D>(reinterpret_cast<__nv_bfloat16*>(wsm + TS::kQOff), q, row0, R, lane);
+  stage_rows16<D>(reinterpret_cast<__nv_bfloat16*>(wsm + TS::kKOff), kb, 0, B, lane);
+  stage_rows16<D>(reinterpret_cast<__nv_bfloat16*>(wsm + TS::kVOff), vb, 0, B, lane);
+}
+
+// `staged`: inblock_tile_stage already ran for this tile (same arguments).
 template <int D>
 __device__ __forceinline__ void inblock_tile_tc(const __nv_bfloat16* q, int R, int row0, const __nv_bfloat16* kb,
                                                 const __nv_bfloat16* vb, int B, float scale, float (&o)[D / 8][4],
-                                                float (&L)[2], int lane, uint8_t* wsm) {
+                                                float (&L)[2], int lane, uint8_t* wsm, bool staged = false) {
   using TS = TileSmem<D>;
   __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(wsm + TS::kQOff);
   __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(wsm + TS::kKOff);
   __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(wsm + TS::kVOff);
   const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
   const int c = lane & 3;
-  __syncwarp();  // the warp's previous reads of its tile memory are done
-  stage_rows16<D>(sQ, q, row0, R, lane);
+  if (!staged) inblock_tile_stage<D>(q, R, row0, kb, vb, B, lane, wsm);
   const float sl2 = scale * 1.4426950408889634f;
   float m0 = -CUDART_INF_F, m1 = -CUDART_INF_F, l0 = 0.f, l1 = 0.f;
 #pragma unroll
   for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   uint32_t qf[D / 16][4];
   for (int k0 = 0; k0 < B; k0 += 16) {
-    if (k0 > 0) __syncwarp();  // the previous chunk's reads of sK / sV are done
-    stage_rows16<D>(sK, kb, k0, B, lane);
-    stage_rows16<D>(sV, vb, k0, B, lane);
+    if (k0 > 0) {  // the first chunk came with the query rows
+      __syncwarp();  // the previous chunk's reads of sK / sV are done
+      stage_rows16<D>(sK, kb, k0, B, lane);
+      stage_rows16<D>(sV, vb, k0, B, lane);
+    }
     cp_async_wait_all();
     __syncwarp();
     if (k0 == 0) {
@@ -525,10 +539,35 @@ struct TileOut {
   Epilogue ep;         // kind 1
 };
 
+// The copies inblock_rows_tc makes first for this warp's first tile (query rows, the
+// first 16 keys and values, and in mode 1 the cached rows), issued ahead -- e.g. while
+// the gate is still being read; the matching call then passes prestaged = true.
+template <int D>
+__device__ void inblock_rows_prestage(const Dims& d, const __nv_bfloat16* q, const __nv_bfloat16* k_blk,
+                                      const __nv_bfloat16* v_blk, int b, int kvh, int r_begin, int r_end,
+                                      const TileOut& out, int warp, int lane, uint8_t* wsm) {
+  using TS = TileSmem<D>;
+  const int t0 = r_begin + warp * 16;
+  if (t0 >= r_end) return;
+  const size_t grow_base = (size_t)(b * d.hq + kvh * d.G) * d.B;
+  if (out.kind == 1 && out.ep.mode == 1) {
+    float* sC = reinterpret_cast<float*>(wsm + TS::kCacheOff);
+    const int nr = min(16, r_end - t0);
+    for (int i = lane; i < nr * (D / 4); i += 32) {
+      const int rr = i / (D / 4), c4 = i - rr * (D / 4);
+      cp_async16(sC + rr * (D + 4) + c4 * 4, out.ep.a_prev + (grow_base + t0 + rr) * D + c4 * 4);
+    }
+    for (int rr = lane; rr < nr; rr += 32) cp_async4(sC + rr * (D + 4) + D, out.ep.l_prev + grow_base + t0 + rr);
+  }
+  inblock_tile_stage<D>(q + grow_base * D, min(r_end, d.R), t0, k_blk + (size_t)(b * d.hkv + kvh) * d.B * D,
+                        v_blk + (size_t)(b * d.hkv + kvh) * d.B * D, d.B, lane, wsm);
+}
+
 template <int D, typename Keep>
 __device__ void inblock_rows_tc(const Dims& d, const __nv_bfloat16* q, const __nv_bfloat16* k_blk,
                                 const __nv_bfloat16* v_blk, int b, int kvh, int r_begin, int r_end,
-                                const TileOut& out, Keep keep, int warp, int nwarps, int lane, uint8_t* wsm) {
+                                const TileOut& out, Keep keep, int warp, int nwarps, int lane, uint8_t* wsm,
+                                bool prestaged = false) {
   using TS = TileSmem<D>;
   const __nv_bfloat16* kb = k_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
   const __nv_bfloat16* vb = v_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
@@ -538,7 +577,8 @@ __device__ void inblock_rows_tc(const Dims& d, const __nv_bfloat16* q, const __n
   const int g = lane >> 2, c = lane & 3;
   for (int t0 = r_begin + warp * 16; t0 < r_end; t0 += nwarps * 16) {
     const bool merge = out.kind == 1 && out.ep.mode == 1;
-    if (merge) {
+    const bool pre = prestaged && t0 == r_begin + warp * 16;
+    if (merge && !pre) {
       // the tile's cached rows are needed after the in-block math: copy them now
       __syncwarp();  // the previous tile's reads of sC are done
       const int nr = min(16, r_end - t0);
@@ -549,7 +589,7 @@ __device__ void inblock_rows_tc(const Dims& d, const __nv_bfloat16* q, const __n
       for (int rr = lane; rr < nr; rr += 32) cp_async4(sC + rr * (D + 4) + D, out.ep.l_prev + grow_base + t0 + rr);
     }
     float o[D / 8][4], L[2];
-    inblock_tile_tc<D>(qg, min(r_end, d.R), t0, kb, vb, d.B, d.scale, o, L, lane, wsm);
+    inblock_tile_tc<D>(qg, min(r_end, d.R), t0, kb, vb, d.B, d.scale, o, L, lane, wsm, pre);
     if (merge) {
       cp_async_wait_all();
       __syncwarp();
@@ -589,6 +629,15 @@ __device__ void inblock_rows_tc(const Dims& d, const __nv_bfloat16* q, const __n
       }
     }
   }
+}
+
+__device__ __forceinline__ TileOut tile_out_ep(const Epilogue& ep) {
+  TileOut out;
+  out.kind = 1;
+  out.slot = nullptr;
+  out.slot_row0 = 0;
+  out.ep = ep;
+  return out;
 }
 
 struct KeepAll {
@@ -639,7 +688,7 @@ __device__ __forceinline__ void inblock_merge_row(const Dims& d, const T* q, con
 template <typename T, int D>
 __device__ void inblock_rows(const Dims& d, const T* q, const T* k_blk, const T* v_blk, int b, int kvh,
                              int row0, int r_begin, int r_end, const Epilogue& ep, int warp, int nwarps,
-                             int lane, uint8_t* tsm = nullptr) {
+                             int lane, uint8_t* tsm = nullptr, bool prestaged = false) {
   if constexpr (std::is_same<T, __nv_bfloat16>::value) {  // bf16: tensor-core tiles
     TileOut out;
     out.kind = 1;
@@ -647,7 +696,7 @@ __device__ void inblock_rows(const Dims& d, const T* q, const T* k_blk, const T*
     out.slot_row0 = 0;
     out.ep = ep;
     inblock_rows_tc<D>(d, q, k_blk, v_blk, b, kvh, row0 + r_begin, row0 + r_end, out, KeepAll(), warp, nwarps,
-                       lane, tsm + (size_t)warp * TileSmem<D>::kBytes);
+                       lane, tsm + (size_t)warp * TileSmem<D>::kBytes, prestaged);
     return;
   }
   const T* kb = k_blk + (size_t)(b * d.hkv + kvh) * d.B * D;

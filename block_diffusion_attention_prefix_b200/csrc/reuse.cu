@@ -15,9 +15,10 @@
 // fused epilogue, so the results agree bit for bit.  Rows that recompute are left to
 // the prefix pass that follows.
 //  * bf16 (reuse_tiles_kernel): a warp per 16-row tile of a group, the in-block
-//    part on the tensor cores (inblock_rows_tc), four tiles per CTA and three CTAs
-//    per SM; each warp
-//    first pulls its tile's rows into L1 so one DRAM latency covers the tile.
+//    part on the tensor cores (inblock_rows_tc), two tiles per CTA and five CTAs per
+//    SM (their tile memories fill shared memory); each warp starts
+//    its tile's copies into its shared memory while it reads the gate, so one DRAM
+//    latency covers the tile.
 //  * fp32 (reuse_rows_kernel): a CTA per group, a warp per row on CUDA cores
 //    (inblock_merge_row), three CTAs per SM.
 #include <cuda_bf16.h>
@@ -89,10 +90,10 @@ __global__ void __launch_bounds__(kReuseThreads, 3) reuse_rows_kernel(const Pass
   }
 }
 
-constexpr int kTileWarps = 4;
+constexpr int kTileWarps = 2;
 
 template <int D>
-__global__ void __launch_bounds__(kTileWarps * 32, 3) reuse_tiles_kernel(const PassArgs args, long long items) {
+__global__ void __launch_bounds__(kTileWarps * 32, 5) reuse_tiles_kernel(const PassArgs args, long long items) {
   using bf16 = __nv_bfloat16;
   const Dims& d = args.d;
   const GateParams& g = args.gate;
@@ -103,23 +104,24 @@ __global__ void __launch_bounds__(kTileWarps * 32, 3) reuse_tiles_kernel(const P
   const int bg = (int)(item / tiles), t = (int)(item - (long long)bg * tiles);
   const int b = bg / d.hkv, kvh = bg - b * d.hkv;
   const int r0 = t * 16, r1 = min(d.R, r0 + 16);
-  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B;
-  {
-    // the tile's q rows, cached rows and L, and the group's block K/V into L1 while
-    // the gate reads the mask (every address inside its buffer)
-    const char* base[5] = {reinterpret_cast<const char*>(static_cast<const bf16*>(args.q) + (grow0 + r0) * D),
-                           reinterpret_cast<const char*>(args.ep.a_dst + (grow0 + r0) * D),
-                           reinterpret_cast<const char*>(args.ep.l_dst + grow0 + r0),
-                           reinterpret_cast<const char*>(static_cast<const bf16*>(args.step.k_blk) + (size_t)bg * d.B * D),
-                           reinterpret_cast<const char*>(static_cast<const bf16*>(args.step.v_blk) + (size_t)bg * d.B * D)};
-    const size_t bytes[5] = {(size_t)(r1 - r0) * D * 2, (size_t)(r1 - r0) * D * 4, (size_t)(r1 - r0) * 4,
-                             (size_t)d.B * D * 2, (size_t)d.B * D * 2};
-#pragma unroll
-    for (int k = 0; k < 5; ++k) {
-      const int lines = (int)((bytes[k] + 127) / 128);
-      for (int i = lane; i <= lines; i += 32) prefetch_l1(base[k] + (i < lines ? (size_t)i * 128 : bytes[k] - 1));
-    }
-  }
+  Epilogue ep;
+  ep.mode = 1;
+  ep.a_dst = nullptr;
+  ep.l_dst = nullptr;
+  ep.a_prev = args.ep.a_dst;  // the cache
+  ep.l_prev = args.ep.l_dst;
+  ep.a_full = args.step.a_full;
+  ep.l_full = args.step.l_full;
+  ep.out_bf16 = 1;
+  const TileOut out = tile_out_ep(ep);
+  const bf16* q = static_cast<const bf16*>(args.q);
+  const bf16* kb = static_cast<const bf16*>(args.step.k_blk);
+  const bf16* vb = static_cast<const bf16*>(args.step.v_blk);
+  extern __shared__ __align__(16) uint8_t tile_smem[];  // a tile memory per warp
+  uint8_t* wsm = tile_smem + (size_t)warp * TileSmem<D>::kBytes;
+  // the tile's copies (query rows, block keys and values, cached rows) start while
+  // the gate reads the mask
+  inblock_rows_prestage<D>(d, q, kb, vb, b, kvh, r0, r1, out, 0, lane, wsm);
   int cnt = 0;
   for (int i = lane; i < d.B; i += 32) cnt += g.mask[(size_t)b * d.B + i] != 0;
   const int M = warp_sum_int(cnt);
@@ -130,24 +132,12 @@ __global__ void __launch_bounds__(kTileWarps * 32, 3) reuse_tiles_kernel(const P
       for (int j = lane; j < d.G; j += 32)
         args.step.dec_reuse[(size_t)b * d.hq + kvh * d.G + j] = head_reuse(g, tau_ok, b, d.hq, kvh * d.G + j) ? 1 : 0;
   }
-  if (!tau_ok) return;  // every head of this batch element recomputes: the prefix pass writes its rows
-  TileOut out;
-  out.kind = 1;
-  out.slot = nullptr;
-  out.slot_row0 = 0;
-  out.ep.mode = 1;
-  out.ep.a_dst = nullptr;
-  out.ep.l_dst = nullptr;
-  out.ep.a_prev = args.ep.a_dst;  // the cache
-  out.ep.l_prev = args.ep.l_dst;
-  out.ep.a_full = args.step.a_full;
-  out.ep.l_full = args.step.l_full;
-  out.ep.out_bf16 = 1;
+  if (!tau_ok) {  // every head of this batch element recomputes: the prefix pass writes its rows
+    cp_async_wait_all();  // no copy may still be landing when the warp leaves
+    return;
+  }
   auto keep = [&](int r) { return head_reuse(g, true, b, d.hq, kvh * d.G + r / d.B); };
-  extern __shared__ __align__(16) uint8_t tile_smem[];  // a tile memory per warp
-  inblock_rows_tc<D>(d, static_cast<const bf16*>(args.q), static_cast<const bf16*>(args.step.k_blk),
-                     static_cast<const bf16*>(args.step.v_blk), b, kvh, r0, r1, out, keep, 0, 1, lane,
-                     tile_smem + (size_t)warp * TileSmem<D>::kBytes);
+  inblock_rows_tc<D>(d, q, kb, vb, b, kvh, r0, r1, out, keep, 0, 1, lane, wsm, true);
 }
 
 template <typename T, int D>
