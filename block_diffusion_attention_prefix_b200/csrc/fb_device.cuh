@@ -358,28 +358,33 @@ __device__ __forceinline__ float inblock_row(const T* qrow, const T* kb, const T
 // o[n][0..1] = A_in[row g][8n + 2c, +1] and o[n][2..3] = the same of row g + 8, and
 // L[0] / L[1] = L_in of rows g / g + 8 (tile rows).
 
-// One warp's shared memory for in-block tiles: 16 staged query rows, 16 keys, 16
-// values (bf16 rows padded to D + 8 elements: 16-byte aligned, ldmatrix without bank
-// conflicts) and 16 cached rows of D + 4 floats (the merge of mode 1).
+// One warp's shared memory for in-block tiles: 16 staged query rows, the keys and
+// values of one chunk (16 rows, or 8 when the block has at most 8 keys; bf16 rows
+// padded to D + 8 elements: 16-byte aligned, ldmatrix without bank conflicts) and 16
+// cached rows of D + 4 floats (the merge of mode 1).  kBytes / kOperandBytes are the
+// sizes for any block (16-row chunks); bytes(B) / operand_bytes(B) for a given B.
 template <int D>
 struct TileSmem {
-  static constexpr int kRow = D + 8;                       // bf16 elements per staged row
-  static constexpr int kQOff = 0;                          // bytes
-  static constexpr int kKOff = kQOff + 16 * kRow * 2;
-  static constexpr int kVOff = kKOff + 16 * kRow * 2;
-  static constexpr int kCacheOff = kVOff + 16 * kRow * 2;
-  static constexpr int kBytes = kCacheOff + 16 * (D + 4) * 4;
-  static constexpr int kOperandBytes = kCacheOff;  // enough for callers that merge nothing (to_ws, mode 0)
-  static_assert(kBytes % 16 == 0 && kOperandBytes % 16 == 0, "16-byte aligned regions");
+  static constexpr int kRow = D + 8;  // bf16 elements per staged row
+  static constexpr int kQBytes = 16 * kRow * 2;
+  __host__ __device__ static constexpr int kv_rows(int B) { return B <= 8 ? 8 : 16; }
+  __host__ __device__ static constexpr int k_off(int) { return kQBytes; }
+  __host__ __device__ static constexpr int v_off(int B) { return kQBytes + kv_rows(B) * kRow * 2; }
+  __host__ __device__ static constexpr int cache_off(int B) { return kQBytes + 2 * kv_rows(B) * kRow * 2; }
+  __host__ __device__ static constexpr int operand_bytes(int B) { return cache_off(B); }
+  __host__ __device__ static constexpr int bytes(int B) { return cache_off(B) + 16 * (D + 4) * 4; }
+  static constexpr int kBytes = bytes(64);
+  static constexpr int kOperandBytes = operand_bytes(64);  // enough for callers that merge nothing
+  static_assert(kBytes % 16 == 0 && kOperandBytes % 16 == 0 && bytes(1) % 16 == 0, "16-byte aligned regions");
 };
 
-// 16 rows [row0, row0 + 16) of a [n][D] bf16 array into a staged [16][D + 8] tile;
-// rows >= n are zero-filled.  Asynchronous (cp.async); the caller waits.
+// `rows` rows [row0, row0 + rows) of a [n][D] bf16 array into a staged [rows][D + 8]
+// tile; rows >= n are zero-filled.  Asynchronous (cp.async); the caller waits.
 template <int D>
-__device__ __forceinline__ void stage_rows16(__nv_bfloat16* dst, const __nv_bfloat16* src, int row0, int n,
-                                             int lane) {
+__device__ __forceinline__ void stage_rows(__nv_bfloat16* dst, const __nv_bfloat16* src, int row0, int n, int rows,
+                                           int lane) {
   constexpr int kChunks = D / 8;  // 16-byte chunks per row
-  for (int i = lane; i < 16 * kChunks; i += 32) {
+  for (int i = lane; i < rows * kChunks; i += 32) {
     const int r = i / kChunks, c = i - r * kChunks;
     const bool valid = row0 + r < n;
     const __nv_bfloat16* g = src + (size_t)(valid ? row0 + r : 0) * D + c * 8;
@@ -393,10 +398,11 @@ template <int D>
 __device__ __forceinline__ void inblock_tile_stage(const __nv_bfloat16* q, int R, int row0, const __nv_bfloat16* kb,
                                                    const __nv_bfloat16* vb, int B, int lane, uint8_t* wsm) {
   using TS = TileSmem<D>;
+  const int kvr = TS::kv_rows(B);
   __syncwarp();  // the warp's previous reads of its tile memory are done
-  stage_rows16<D>(reinterpret_cast<__nv_bfloat16*>(wsm + TS::kQOff), q, row0, R, lane);
-  stage_rows16<D>(reinterpret_cast<__nv_bfloat16*>(wsm + TS::kKOff), kb, 0, B, lane);
-  stage_rows16<D>(reinterpret_cast<__nv_bfloat16*>(wsm + TS::kVOff), vb, 0, B, lane);
+  stage_rows<D>(reinterpret_cast<__nv_bfloat16*>(wsm), q, row0, R, 16, lane);
+  stage_rows<D>(reinterpret_cast<__nv_bfloat16*>(wsm + TS::k_off(B)), kb, 0, B, kvr, lane);
+  stage_rows<D>(reinterpret_cast<__nv_bfloat16*>(wsm + TS::v_off(B)), vb, 0, B, kvr, lane);
 }
 
 // `staged`: inblock_tile_stage already ran for this tile (same arguments).
@@ -405,9 +411,10 @@ __device__ __forceinline__ void inblock_tile_tc(const __nv_bfloat16* q, int R, i
                                                 const __nv_bfloat16* vb, int B, float scale, float (&o)[D / 8][4],
                                                 float (&L)[2], int lane, uint8_t* wsm, bool staged = false) {
   using TS = TileSmem<D>;
-  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(wsm + TS::kQOff);
-  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(wsm + TS::kKOff);
-  __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(wsm + TS::kVOff);
+  const bool narrow = TS::kv_rows(B) == 8;  // at most 8 keys: one n8 tile of scores, 8 value rows
+  __nv_bfloat16* sQ = reinterpret_cast<__nv_bfloat16*>(wsm);
+  __nv_bfloat16* sK = reinterpret_cast<__nv_bfloat16*>(wsm + TS::k_off(B));
+  __nv_bfloat16* sV = reinterpret_cast<__nv_bfloat16*>(wsm + TS::v_off(B));
   const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
   const int c = lane & 3;
   if (!staged) inblock_tile_stage<D>(q, R, row0, kb, vb, B, lane, wsm);
@@ -417,10 +424,10 @@ __device__ __forceinline__ void inblock_tile_tc(const __nv_bfloat16* q, int R, i
   for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   uint32_t qf[D / 16][4];
   for (int k0 = 0; k0 < B; k0 += 16) {
-    if (k0 > 0) {  // the first chunk came with the query rows
+    if (k0 > 0) {  // the first chunk came with the query rows (chunks past it: 16 rows)
       __syncwarp();  // the previous chunk's reads of sK / sV are done
-      stage_rows16<D>(sK, kb, k0, B, lane);
-      stage_rows16<D>(sV, vb, k0, B, lane);
+      stage_rows<D>(sK, kb, k0, B, 16, lane);
+      stage_rows<D>(sV, vb, k0, B, 16, lane);
     }
     cp_async_wait_all();
     __syncwarp();
@@ -430,16 +437,24 @@ __device__ __forceinline__ void inblock_tile_tc(const __nv_bfloat16* q, int R, i
         ldsm_x4(aQ + (uint32_t)(((lane & 15) * TS::kRow + kk * 16 + (lane >> 4) * 8) * 2), qf[kk][0], qf[kk][1],
                 qf[kk][2], qf[kk][3]);
     }
-    // S for this chunk's 16 keys (n-tiles 0: keys k0..k0+7, 1: k0+8..k0+15)
+    // S for this chunk's 16 keys (n-tiles 0: keys k0..k0+7, 1: k0+8..k0+15).  With at
+    // most 8 keys the second n-tile is all masked and is not computed (its scores are
+    // -inf either way; the skipped products are exact zeros in the sums).
     float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      uint32_t b0, b1, b2, b3;
       const int key = (lane & 7) + ((lane >> 4) << 3);
       const int col = kk * 16 + ((lane >> 3) & 1) * 8;
-      ldsm_x4(aK + (uint32_t)((key * TS::kRow + col) * 2), b0, b1, b2, b3);
-      mma_bf16_16816_free(s[0], qf[kk], b0, b1);
-      mma_bf16_16816_free(s[1], qf[kk], b2, b3);
+      if (narrow) {
+        uint32_t b0, b1;
+        ldsm_x2(aK + (uint32_t)(((lane & 7) * TS::kRow + col) * 2), b0, b1);
+        mma_bf16_16816_free(s[0], qf[kk], b0, b1);
+      } else {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(aK + (uint32_t)((key * TS::kRow + col) * 2), b0, b1, b2, b3);
+        mma_bf16_16816_free(s[0], qf[kk], b0, b1);
+        mma_bf16_16816_free(s[1], qf[kk], b2, b3);
+      }
     }
     float cm0 = -CUDART_INF_F, cm1 = -CUDART_INF_F;
 #pragma unroll
@@ -501,10 +516,14 @@ __device__ __forceinline__ void inblock_tile_tc(const __nv_bfloat16* q, int R, i
     }
 #pragma unroll
     for (int dn = 0; dn < D / 8; dn += 2) {
-      uint32_t b0, b1, b2, b3;
-      const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
-      const int col = dn * 8 + (lane >> 4) * 8;
-      ldsm_x4_t(aV + (uint32_t)((key * TS::kRow + col) * 2), b0, b1, b2, b3);
+      uint32_t b0, b1 = 0u, b2, b3 = 0u;  // with at most 8 keys, value rows 8..15 are zero
+      if (narrow) {
+        ldsm_x2_t(aV + (uint32_t)(((lane & 7) * TS::kRow + dn * 8 + ((lane >> 3) & 1) * 8) * 2), b0, b2);
+      } else {
+        const int key = (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int col = dn * 8 + (lane >> 4) * 8;
+        ldsm_x4_t(aV + (uint32_t)((key * TS::kRow + col) * 2), b0, b1, b2, b3);
+      }
       mma_bf16_16816_free(o[dn], hi, b0, b1);
       mma_bf16_16816_free(o[dn], lo, b0, b1);
       mma_bf16_16816_free(o[dn + 1], hi, b2, b3);
@@ -551,7 +570,7 @@ __device__ void inblock_rows_prestage(const Dims& d, const __nv_bfloat16* q, con
   if (t0 >= r_end) return;
   const size_t grow_base = (size_t)(b * d.hq + kvh * d.G) * d.B;
   if (out.kind == 1 && out.ep.mode == 1) {
-    float* sC = reinterpret_cast<float*>(wsm + TS::kCacheOff);
+    float* sC = reinterpret_cast<float*>(wsm + TS::cache_off(d.B));
     const int nr = min(16, r_end - t0);
     for (int i = lane; i < nr * (D / 4); i += 32) {
       const int rr = i / (D / 4), c4 = i - rr * (D / 4);
@@ -573,7 +592,7 @@ __device__ void inblock_rows_tc(const Dims& d, const __nv_bfloat16* q, const __n
   const __nv_bfloat16* vb = v_blk + (size_t)(b * d.hkv + kvh) * d.B * D;
   const size_t grow_base = (size_t)(b * d.hq + kvh * d.G) * d.B;  // global row of group row 0
   const __nv_bfloat16* qg = q + grow_base * D;
-  float* sC = reinterpret_cast<float*>(wsm + TS::kCacheOff);
+  float* sC = reinterpret_cast<float*>(wsm + TS::cache_off(d.B));
   const int g = lane >> 2, c = lane & 3;
   for (int t0 = r_begin + warp * 16; t0 < r_end; t0 += nwarps * 16) {
     const bool merge = out.kind == 1 && out.ep.mode == 1;

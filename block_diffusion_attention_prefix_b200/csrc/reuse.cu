@@ -15,8 +15,8 @@
 // fused epilogue, so the results agree bit for bit.  Rows that recompute are left to
 // the prefix pass that follows.
 //  * bf16 (reuse_tiles_kernel): a warp per 16-row tile of a group, the in-block
-//    part on the tensor cores (inblock_rows_tc), two tiles per CTA and five CTAs per
-//    SM (their tile memories fill shared memory); each warp starts
+//    part on the tensor cores (inblock_rows_tc), two tiles per CTA and up to six CTAs
+//    per SM (their tile memories fill shared memory); each warp starts
 //    its tile's copies into its shared memory while it reads the gate, so one DRAM
 //    latency covers the tile.
 //  * fp32 (reuse_rows_kernel): a CTA per group, a warp per row on CUDA cores
@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(kReuseThreads, 3) reuse_rows_kernel(const Pass
 constexpr int kTileWarps = 2;
 
 template <int D>
-__global__ void __launch_bounds__(kTileWarps * 32, 5) reuse_tiles_kernel(const PassArgs args, long long items) {
+__global__ void __launch_bounds__(kTileWarps * 32, 6) reuse_tiles_kernel(const PassArgs args, long long items) {
   using bf16 = __nv_bfloat16;
   const Dims& d = args.d;
   const GateParams& g = args.gate;
@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(kTileWarps * 32, 5) reuse_tiles_kernel(const P
   const bf16* kb = static_cast<const bf16*>(args.step.k_blk);
   const bf16* vb = static_cast<const bf16*>(args.step.v_blk);
   extern __shared__ __align__(16) uint8_t tile_smem[];  // a tile memory per warp
-  uint8_t* wsm = tile_smem + (size_t)warp * TileSmem<D>::kBytes;
+  uint8_t* wsm = tile_smem + (size_t)warp * TileSmem<D>::bytes(d.B);
   // the tile's copies (query rows, block keys and values, cached rows) start while
   // the gate reads the mask
   inblock_rows_prestage<D>(d, q, kb, vb, b, kvh, r0, r1, out, 0, lane, wsm);
@@ -144,12 +144,13 @@ template <typename T, int D>
 cudaError_t launch_typed(const PassArgs& a, cudaStream_t s) {
   if constexpr (std::is_same<T, __nv_bfloat16>::value) {
     const long long items = (long long)a.d.b * a.d.hkv * ((a.d.R + 15) / 16);
-    constexpr int smem = kTileWarps * TileSmem<D>::kBytes;
+    const int smem = kTileWarps * TileSmem<D>::bytes(a.d.B);  // narrower for blocks of at most 8 keys
     static bool attr_set[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-      const cudaError_t e = cudaFuncSetAttribute(reuse_tiles_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      const cudaError_t e = cudaFuncSetAttribute(reuse_tiles_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kTileWarps * TileSmem<D>::kBytes);
       if (e != cudaSuccess) return e;
       if (dev >= 0 && dev < 64) attr_set[dev] = true;
     }
