@@ -236,8 +236,8 @@ int run_pass(const Dims& d0, long long keys, const void* q, const void* k, const
     CUtensorMap tq, tk, tv;
     const long long qrows = (long long)d.b * d.hq * d.B;
     FB_TRY(encode_kv_map(&tq, q, d.D, qrows, d.D, qrows * d.D, 1, 128));
-    FB_TRY(encode_kv_map(&tk, k, d.D, keys, row_stride, head_stride, d.b * d.hkv, 64));
-    FB_TRY(encode_kv_map(&tv, v, d.D, keys, row_stride, head_stride, d.b * d.hkv, 64));
+    FB_TRY(encode_kv_map(&tk, k, d.D, keys, row_stride, head_stride, d.b * d.hkv, a.plan.key_tile));
+    FB_TRY(encode_kv_map(&tv, v, d.D, keys, row_stride, head_stride, d.b * d.hkv, a.plan.key_tile));
     return cuda_status(launch_pass_tc(a, tq, tk, tv, stream));
   }
   if (d.dtype == FB_BF16) {
@@ -294,7 +294,7 @@ SplitPlan plan_split(int R, int D, long long N, int b, int hkv, int dtype, int n
     // contraction: tcgen05 (M = 128, rows past the tile padded); otherwise mma.sync.
     p.tc = (allow_tc && D == 128 && R > 16) ? 1 : 0;
     p.row_tile = p.tc ? (R <= 32 ? 32 : (R <= 64 ? 64 : 128)) : (R <= 16 ? 16 : (R <= 32 ? 32 : 64));
-    p.key_tile = 64;
+    p.key_tile = p.tc ? 128 : 64;
   } else {
     p.row_tile = 16;
     p.key_tile = 32;
@@ -453,6 +453,15 @@ int fb_merge(const fb_shape* shape, const float* a1, const float* l1, const floa
   FB_TRY(check_ptr(a_full));
   if (!l1 || !l2) return FB_ERR_NULL;
   return cuda_status(launch_merge(d, a1, l1, a2, l2, a_full, l_full, (cudaStream_t)stream));
+}
+
+int fb_exp2_fma(const float* x, float* y, int64_t n, fb_stream_t stream) {
+  if (n == 0) return FB_OK;
+  if (!x || !y) return FB_ERR_NULL;
+  if ((reinterpret_cast<uintptr_t>(x) & 3u) || (reinterpret_cast<uintptr_t>(y) & 3u)) return FB_ERR_ALIGN;
+  if (n < 0 || n >= (int64_t(1) << 31)) return FB_ERR_SHAPE;
+  if (current_device() < 0) return FB_ERR_CUDA;
+  return cuda_status(launch_exp2_fma(x, y, n, (cudaStream_t)stream));
 }
 
 int fb_merge_partials(const fb_shape* shape, const float* a_parts, int64_t a_part_stride, const float* l_parts,

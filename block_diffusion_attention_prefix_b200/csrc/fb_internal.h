@@ -181,6 +181,7 @@ cudaError_t launch_small_block(const SmallBlockArgs& a, cudaStream_t s);
 cudaError_t launch_gate_eval(const Dims& d, const GateParams& g, int32_t* dec_M, uint8_t* dec_reuse,
                              cudaStream_t s);
 // Context-parallel combine: cache rows of recomputing heads = merge of P partials.
+cudaError_t launch_exp2_fma(const float* x, float* y, long long n, cudaStream_t s);
 cudaError_t launch_merge_parts(const Dims& d, const GateParams& g, const float* a_parts, long long a_stride,
                                const float* l_parts, long long l_stride, int P, float* a_out, float* l_out,
                                cudaStream_t s);

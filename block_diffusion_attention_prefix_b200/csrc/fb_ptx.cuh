@@ -211,6 +211,78 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// 2^x on the FMA and integer pipes, for softmax exponentials that would otherwise
+// queue on the special-function unit.  Range reduction x = n + f with n = round(x)
+// (adding and subtracting 1.5 * 2^23 rounds to the nearest integer and leaves n in
+// the low mantissa bits of the sum), f in [-1/2, 1/2]; 2^f by a cubic with p(0) = 1
+// whose coefficients minimise the largest relative error on [-1/2, 1/2] (Lawson's
+// iteratively reweighted least squares; gen_exp2_poly.py in this folder refits
+// them); then 2^n is added into the exponent field.  Relative error <= 1.02e-4 for
+// x in [-125, 2^22) (below bf16's half ulp, the precision P is kept in); exact at
+// integers; 0 for x < -125 and for -inf.
+__device__ __forceinline__ float exp2_fma(float x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const float t = __fadd_rn(x, kRound);
+  const float f = __fsub_rn(x, __fsub_rn(t, kRound));
+  const float p = fmaf(f, fmaf(f, fmaf(f, 0.05500892966239863f, 0.2422109719919523f), 0.6932829287944439f), 1.0f);
+  const float r = __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
+  return x < -125.0f ? 0.0f : r;
+}
+
+// Packed pairs of floats for the sm_100 two-wide fp32 instructions (one issue slot
+// per pair): f2_pack / f2_unpack only rename registers.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// exp2_fma on a pair, its float steps two-wide: the same roundings, so each half
+// equals exp2_fma of that half bit for bit.
+__device__ __forceinline__ void exp2_fma2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kRound = 12582912.0f;
+  const uint64_t X = f2_pack(x0, x1);
+  const uint64_t R = f2_pack(kRound, kRound);
+  const uint64_t T = f2_add(X, R);
+  const uint64_t F = f2_sub(X, f2_sub(T, R));
+  uint64_t P = f2_fma(F, f2_pack(0.05500892966239863f, 0.05500892966239863f),
+                      f2_pack(0.2422109719919523f, 0.2422109719919523f));
+  P = f2_fma(F, P, f2_pack(0.6932829287944439f, 0.6932829287944439f));
+  P = f2_fma(F, P, f2_pack(1.0f, 1.0f));
+  float p0, p1, t0, t1;
+  f2_unpack(P, p0, p1);
+  f2_unpack(T, t0, t1);
+  const float r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  const float r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+  y0 = x0 < -125.0f ? 0.0f : r0;
+  y1 = x1 < -125.0f ? 0.0f : r1;
+}
+
+// Largest of three (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

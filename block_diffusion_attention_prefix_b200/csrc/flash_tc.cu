@@ -1,8 +1,8 @@
 // flash_tc.cu -- attention pass on the 5th-generation tensor cores (tcgen05 + TMEM).
 //
 // Used when more than 16 query rows share a KV head (GQA packing: B x G rows), so
-// the tiles are a real dense contraction: 128 x 64 x 128 score tiles and
-// 128 x 128 x 64 output tiles on tcgen05.mma with fp32 accumulators in tensor
+// the tiles are a real dense contraction: 128 x 128 x 128 score tiles and
+// 128 x 128 x 128 output tiles on tcgen05.mma with fp32 accumulators in tensor
 // memory.  Same contract as the mma.sync pass (prefix_bf16.cu): (A, L) per query
 // row over a key set -- the out-of-block part over J_out, or the in-block part
 // over J_in -- and, in a fused step, the in-block rows, the merge with the cache
@@ -18,25 +18,35 @@
 //           epilogue -- small blocks, where row tiles alone cannot fill the GPU;
 //   !SPLIT: all keys, epilogue directly (large blocks: video, 4680 rows per head).
 // 352 threads:
-//   warp 0     TMA producer: Q once; 64-key K and V tiles into a 4-stage ring
-//              (128-byte swizzle, no multicast).
+//   warp 0     TMA producer: Q once; 128-key K tiles into a 3-slot ring and V tiles
+//              into a 2-slot ring (128-byte swizzle, no multicast).  A K slot frees
+//              when its score MMAs finish, a V slot when its output MMAs do.
 //   warp 1     TMEM owner and MMA issuer (one thread):
-//                S_w  = Q K_j^T   (M=128, N=64 keys, K=128 d; A, B K-major)
-//                O_w += P_w V_j   (M=128, N=128 d,  K=64 keys; A = P K-major,
-//                                  B = V MN-major)
+//                S_w  = Q K_j^T   (M=128, N=128 keys, K=128 d; A, B K-major in
+//                                  shared memory)
+//                O_w += P_w V_j   (M=128, N=128 d,  K=128 keys; A = P_w in TMEM,
+//                                  B = V MN-major in shared memory)
 //              for key tiles j split between two softmax warpgroups w = j % 2,
 //              so that one group's softmax overlaps the other's MMAs;
-//              completions signalled with tcgen05.commit on mbarriers.
+//              completions signalled with tcgen05.commit on mbarriers.  An MMA
+//              with N = 64 runs at half the rate of N = 128 on this tensor core,
+//              which is why the key tile is 128 wide.
 //   warps 2-5, 6-9  softmax warpgroups a and b, one query row per thread (TMEM
-//              lane = row): read S_w with tcgen05.ld, online softmax in base 2, P_w
-//              (bf16) into shared memory.  O_w is rescaled in TMEM only when a row's
-//              max grows by more than 2^8 (otherwise the stale max is kept; p <= 2^8
-//              is exact enough in bf16 and cannot overflow fp32).  At the end group a
-//              merges the two partial results (the FlashBlock log-space merge).
+//              lane = row): read S_w with tcgen05.ld, online softmax in base 2, and
+//              P_w as bf16 pairs written back over the first half of S_w's columns
+//              (tcgen05.st), where the output MMA reads it; the next score MMA of
+//              the group is issued after that output MMA, and MMAs of one thread
+//              run in issue order.  A quarter of the exponentials run on the FMA
+//              pipe (exp2_fma), the rest on the special-function unit.  O_w is
+//              rescaled in TMEM only when a row's max grows by more than 2^8
+//              (otherwise the stale max is kept; p <= 2^8 is exact enough in bf16
+//              and cannot overflow fp32).  At the end group a merges the two
+//              partial results (the FlashBlock log-space merge).
 //   warp 10    fused step: this split's share of the tile's in-block rows.
-// TMEM: 512 columns (S_a [0,64), S_b [64,128), O_a [128,256), O_b [256,384)).
-// Every mbarrier wait is time bounded; on expiry the roles fall through to the
-// common exit, which frees TMEM.
+// TMEM: 512 columns (S_a / P_a [0,128), S_b / P_b [128,256), O_a [256,384),
+// O_b [384,512)).  Every mbarrier wait is time bounded; on expiry the roles fall
+// through to the common exit, which frees TMEM.
+#include <algorithm>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -50,39 +60,49 @@ namespace fb {
 namespace {
 
 constexpr int kM = 128;
-constexpr int kKT = 64;   // keys per tile
+constexpr int kKT = 128;  // keys per tile
 constexpr int kD = 128;
-constexpr int kStages = 4;
+constexpr int kKSlots = 3;  // K ring
+constexpr int kVSlots = 2;  // V ring
 constexpr int kThreads = 352;  // 11 warps
 constexpr int kAuxWarp = 10;
 constexpr int kBarSoftmax = 1;  // the 8 softmax warps
 constexpr int kBarFinish = 2;   // every warp (split combine)
 constexpr uint32_t kTmemCols = 512;
+// Pairs of keys (t, t + 1) within a 32-key chunk whose exponentials run on the FMA
+// pipe (exp2_fma2) instead of the special-function unit.  None: on the video
+// workload every fraction tried (1/4, 3/8, 1/2) made the pass slower (0.55, 0.54,
+// 0.52 of the burst tensor peak against 0.59 with none) -- the softmax is bound by
+// issue slots and latency, not by the special-function unit.
+__host__ __device__ constexpr bool kPolyPair(int) { return false; }
+constexpr uint32_t kOCol = 256;                  // O_a at column 256, O_b at 384
 constexpr int kQBlock = 128 * 128;               // Q: [128 rows][128 B] per 64-column block
 constexpr int kQBytes = 2 * kQBlock;
-constexpr int kKVBlock = kKT * 128;              // K or V: [64 keys][128 B] per 64-column block
-constexpr int kKVBytes = 2 * kKVBlock;           // one 64 x 128 tile
-constexpr int kStageBytes = 2 * kKVBytes;        // K then V
-constexpr int kPBytes = 128 * kKT * 2;           // P_w: [128 rows][64 keys] bf16 = one 128-B block
+constexpr int kKVBlock = kKT * 128;              // K or V: [128 keys][128 B] per 64-column block
+constexpr int kKVBytes = 2 * kKVBlock;           // one 128 x 128 tile
 constexpr int kQOff = 0;
-constexpr int kStageOff = kQBytes;
-constexpr int kPOff = kStageOff + kStages * kStageBytes;
-constexpr int kAuxOff = kPOff + 2 * kPBytes;     // the aux warp's in-block tile memory
+constexpr int kKOff = kQBytes;
+constexpr int kVOff = kKOff + kKSlots * kKVBytes;
+constexpr int kAuxOff = kVOff + kVSlots * kKVBytes;  // the aux warp's in-block tile memory
 constexpr int kSmemBytes = kAuxOff + TileSmem<kD>::kOperandBytes + 1024;
 constexpr int kBufBytes = kSmemBytes - 1024;  // all of it, reused by the split combine
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
-// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2, version 1).
-// K-major: 8-row groups 1024 B apart (SBO); LBO unused (1).  MN-major: LBO is the
-// stride between 64-element blocks along M/N, SBO the stride between 8-row groups
-// along K.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
+// Shared-memory matrix descriptor, 128-byte swizzle (layout type 2, version 1),
+// as two 32-bit words.  Low word: start address >> 4 (bits 0-13) and the leading
+// byte offset >> 4 (bits 16-29); high word: the stride byte offset >> 4 (bits 0-13),
+// the version bit (14) and the swizzle mode (bits 29-31).  K-major: 8-row groups
+// 1024 B apart (SBO); LBO unused (1).  MN-major: LBO is the stride between
+// 64-element blocks along M/N, SBO the stride between 8-row groups along K.
+// Shared addresses are below 2^18, so adding (byte offset >> 4) to the low word
+// moves the start without a carry into the LBO field: one add per MMA.
+__host__ __device__ constexpr uint32_t desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
 }
+__host__ __device__ constexpr uint32_t desc_hi(uint32_t sbo_bytes) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (2u << 29);
+}
+__device__ __forceinline__ uint64_t desc(uint32_t lo, uint32_t hi) { return ((uint64_t)hi << 32) | lo; }
 
 // Instruction descriptor of kind::f16: fp32 accumulate, bf16 A and B, A K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
@@ -95,6 +115,17 @@ __device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t a, uint64_t b, ui
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
           d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// Same MMA with A read from tensor memory: a_tmem addresses the 128 x 16 A slice,
+// row m in lane m, two bf16 of a row per 32-bit column in k order (low half first).
+__device__ __forceinline__ void umma_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                            uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
 
@@ -137,6 +168,15 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -157,8 +197,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t q_full;
-  __shared__ __align__(8) uint64_t kv_full[kStages];
-  __shared__ __align__(8) uint64_t kv_empty[kStages];
+  __shared__ __align__(8) uint64_t k_full[kKSlots];
+  __shared__ __align__(8) uint64_t k_empty[kKSlots];
+  __shared__ __align__(8) uint64_t v_full[kVSlots];
+  __shared__ __align__(8) uint64_t v_empty[kVSlots];
   __shared__ __align__(8) uint64_t s_full[2];
   __shared__ __align__(8) uint64_t p_full[2];
   __shared__ __align__(8) uint64_t o_done[2];
@@ -233,9 +275,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(&q_full, 1);
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < kKSlots; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kVSlots; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int w = 0; w < 2; ++w) {
       mbar_init(&s_full[w], 1);
@@ -265,62 +311,100 @@ __global__ void __launch_bounds__(kThreads, 1)
       prefetch_tmap(&tmV);
       mbar_arrive_expect_tx(&q_full, kQBytes);
       for (int h = 0; h < 2; ++h) tma_load_3d(smem + kQOff + h * kQBlock, &tmQ, &q_full, h * 64, (int)grow0, 0);
-      int issued = 0;
-      for (int j = 0; j < T; ++j) {
-        const int s = j % kStages;
-        if (!mbar_wait_bounded(&kv_empty[s], ((uint32_t)(j / kStages) & 1u) ^ 1u, args.err, DEV_ERR_WAIT_EMPTY))
-          break;
-        mbar_arrive_expect_tx(&kv_full[s], kStageBytes);
-        uint8_t* st = smem + kStageOff + s * kStageBytes;
-        const int key0 = (int)(key_begin + (long long)j * kKT);
-        for (int h = 0; h < 2; ++h) {
-          tma_load_3d(st + h * kKVBlock, &tmK, &kv_full[s], h * 64, key0, bg);
-          tma_load_3d(st + kKVBytes + h * kKVBlock, &tmV, &kv_full[s], h * 64, key0, bg);
+      // K tiles run up to three ahead, V tiles two: K(j + 3) once the score MMAs of
+      // tile j are done, then V(j + 2) once its output MMAs are.
+      auto load_k = [&](int n) -> bool {
+        const int sl = n % kKSlots;
+        if (!mbar_wait_bounded(&k_empty[sl], ((uint32_t)(n / kKSlots) & 1u) ^ 1u, args.err, DEV_ERR_WAIT_EMPTY))
+          return false;
+        mbar_arrive_expect_tx(&k_full[sl], kKVBytes);
+        uint8_t* st = smem + kKOff + sl * kKVBytes;
+        const int key0 = (int)(key_begin + (long long)n * kKT);
+        for (int h = 0; h < 2; ++h) tma_load_3d(st + h * kKVBlock, &tmK, &k_full[sl], h * 64, key0, bg);
+        return true;
+      };
+      auto load_v = [&](int n) -> bool {
+        const int sl = n % kVSlots;
+        if (!mbar_wait_bounded(&v_empty[sl], ((uint32_t)(n / kVSlots) & 1u) ^ 1u, args.err, DEV_ERR_WAIT_EMPTY))
+          return false;
+        mbar_arrive_expect_tx(&v_full[sl], kKVBytes);
+        uint8_t* st = smem + kVOff + sl * kKVBytes;
+        const int key0 = (int)(key_begin + (long long)n * kKT);
+        for (int h = 0; h < 2; ++h) tma_load_3d(st + h * kKVBlock, &tmV, &v_full[sl], h * 64, key0, bg);
+        return true;
+      };
+      int nk = 0, nv = 0;  // tiles issued
+      bool ok = true;
+      for (; nk < min(T, kKSlots) && ok; ++nk) ok = load_k(nk);
+      for (; nv < min(T, kVSlots) && ok; ++nv) ok = load_v(nv);
+      while (ok && (nk < T || nv < T)) {
+        if (nk < T) {
+          ok = load_k(nk);
+          if (ok) ++nk;
         }
-        ++issued;
+        if (ok && nv < T) {
+          ok = load_v(nv);
+          if (ok) ++nv;
+        }
       }
-      for (int j = max(0, issued - kStages); j < issued; ++j)
-        mbar_wait_bounded(&kv_full[j % kStages], (uint32_t)(j / kStages) & 1u, args.err, DEV_ERR_WAIT_FULL);
+      // No copy may still be landing when the CTA leaves (on a timeout above too).
+      for (int n = max(0, nk - kKSlots); n < nk; ++n)
+        mbar_wait_bounded(&k_full[n % kKSlots], (uint32_t)(n / kKSlots) & 1u, args.err, DEV_ERR_WAIT_FULL);
+      for (int n = max(0, nv - kVSlots); n < nv; ++n)
+        mbar_wait_bounded(&v_full[n % kVSlots], (uint32_t)(n / kVSlots) & 1u, args.err, DEV_ERR_WAIT_FULL);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && T > 0) {
       constexpr uint32_t kIdQK = idesc_bf16(kM, kKT, false);
       constexpr uint32_t kIdPV = idesc_bf16(kM, kD, true);
-      auto issue_qk = [&](int j) -> bool {
-        if (!mbar_wait_bounded(&kv_full[j % kStages], (uint32_t)(j / kStages) & 1u, args.err, DEV_ERR_WAIT_FULL))
-          return false;
-        const uint32_t sK = smem_u32(smem + kStageOff + (j % kStages) * kStageBytes);
+      const uint32_t q_lo = desc_lo(sQ, 16);
+      const uint32_t k_lo = desc_lo(smem_u32(smem + kKOff), 16);
+      const uint32_t v_lo = desc_lo(smem_u32(smem + kVOff), kKVBlock);
+      auto wait_k = [&](int j) -> bool {
+        return mbar_wait_bounded(&k_full[j % kKSlots], (uint32_t)(j / kKSlots) & 1u, args.err, DEV_ERR_WAIT_FULL);
+      };
+      auto issue_qk = [&](int j) {  // K_j has landed
+        const int sl = j % kKSlots;
+        const uint32_t b_lo = k_lo + (uint32_t)sl * (kKVBytes >> 4);
         const uint32_t tS = tmem + (uint32_t)((j & 1) * kKT);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint64_t a = sdesc(sQ + (kk >> 2) * kQBlock + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc(sK + (kk >> 2) * kKVBlock + (kk & 3) * 32, 16, 1024);
-          umma(tS, a, bd, kIdQK, kk > 0 ? 1u : 0u);
+          constexpr uint32_t kHi = desc_hi(1024);
+          const uint32_t off = (uint32_t)(((kk >> 2) * kKVBlock + (kk & 3) * 32) >> 4);
+          const uint32_t aoff = (uint32_t)(((kk >> 2) * kQBlock + (kk & 3) * 32) >> 4);
+          umma(tS, desc(q_lo + aoff, kHi), desc(b_lo + off, kHi), kIdQK, kk > 0 ? 1u : 0u);
         }
+        umma_commit(&k_empty[sl]);
         umma_commit(&s_full[j & 1]);
-        return true;
       };
-      bool ok = mbar_wait_bounded(&q_full, 0u, args.err, DEV_ERR_WAIT_FULL);
-      if (ok) ok = issue_qk(0);
-      if (ok && T > 1) ok = issue_qk(1);
+      bool ok = mbar_wait_bounded(&q_full, 0u, args.err, DEV_ERR_WAIT_FULL) && wait_k(0);
+      if (ok) issue_qk(0);
+      if (ok && T > 1) {
+        ok = wait_k(1);
+        if (ok) issue_qk(1);
+      }
       for (int j = 0; j < T && ok; ++j) {
         const int w = j & 1;
+        // The tiles this step reads (V_j, K_{j+2}) are normally in place long before
+        // group w hands over P_w: wait for them first, so that only the hand-over
+        // stands between the previous MMAs and these.
+        const int sl = j % kVSlots;
+        if (!mbar_wait_bounded(&v_full[sl], (uint32_t)(j / kVSlots) & 1u, args.err, DEV_ERR_WAIT_FULL)) break;
+        if (j + 2 < T && !wait_k(j + 2)) break;
         // O_w += P_w V_j once group w has written P_w for tile j.
         if (!mbar_wait_bounded(&p_full[w], (uint32_t)(j >> 1) & 1u, args.err, DEV_ERR_WAIT_FULL)) break;
         tc_fence_after();
-        const uint32_t sV = smem_u32(smem + kStageOff + (j % kStages) * kStageBytes + kKVBytes);
-        const uint32_t sP = smem_u32(smem + kPOff + w * kPBytes);
-        const uint32_t tO = tmem + 128u + (uint32_t)(w * kD);
+        const uint32_t b_lo = v_lo + (uint32_t)sl * (kKVBytes >> 4);
+        const uint32_t tP = tmem + (uint32_t)(w * kKT);
+        const uint32_t tO = tmem + kOCol + (uint32_t)(w * kD);
 #pragma unroll
-        for (int kk = 0; kk < kKT / 16; ++kk) {
-          const uint64_t a = sdesc(sP + kk * 32, 16, 1024);
-          const uint64_t bd = sdesc(sV + kk * 2048, kKVBlock, 1024);
-          umma(tO, a, bd, kIdPV, (j >= 2 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&kv_empty[j % kStages]);
+        for (int kk = 0; kk < kKT / 16; ++kk)
+          umma_tmem_a(tO, tP + (uint32_t)(kk * 8), desc(b_lo + (uint32_t)(kk * (2048 >> 4)), desc_hi(1024)), kIdPV,
+                      (j >= 2 || kk > 0) ? 1u : 0u);
+        umma_commit(&v_empty[sl]);
         umma_commit(&o_done[w]);
-        if (j + 2 < T) ok = issue_qk(j + 2);  // S_w is free: group w has read it
+        if (j + 2 < T) issue_qk(j + 2);  // after this group's output MMA, in issue order
       }
     }
   } else if (warp == kAuxWarp) {
@@ -339,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;
     const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
     const uint32_t tS = tmem + (uint32_t)(w * kKT) + lane_addr;
-    const uint32_t tO = tmem + 128u + (uint32_t)(w * kD) + lane_addr;
+    const uint32_t tO = tmem + kOCol + (uint32_t)(w * kD) + lane_addr;
     const float sl2 = d.scale * 1.4426950408889634f;
     const int ntiles = (real && T > w) ? (T - w + 1) / 2 : 0;
     float m_used = -CUDART_INF_F, l = 0.f;
@@ -351,36 +435,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      float s[kKT];
-#pragma unroll
-      for (int c = 0; c < kKT / 32; ++c) {
-        float v[32];
-        tmem_ld32(tS + c * 32, v);
-#pragma unroll
-        for (int t = 0; t < 32; ++t) s[c * 32 + t] = v[t];
-      }
-      tmem_wait_ld();
       // Raw scores; the scale (> 0) is applied in the exponent.  Keys past the end
-      // of the range (only in its last tile) are masked.
+      // of the range (only in its last tile) are masked.  S_w is read twice (for
+      // the max, then chunk by chunk for the exponentials), which keeps a row's
+      // registers to two 32-column chunks.
       const long long kleft = key_end - key_begin - (long long)j * kKT;
-      if (kleft < kKT) {
+      auto mask32 = [&](float (&v)[32], int c) {
+        if (kleft < kKT) {
 #pragma unroll
-        for (int c = 0; c < kKT; ++c) s[c] = c < kleft ? s[c] : -CUDART_INF_F;
-      }
-      float mx0 = s[0], mx1 = s[1];
-#pragma unroll
-      for (int c = 2; c < kKT; c += 2) {
-        mx0 = fmaxf(mx0, s[c]);
-        mx1 = fmaxf(mx1, s[c + 1]);
-      }
-      const float mt = fmaxf(mx0, mx1) * sl2;
-      if (i > 0) {  // PV of this group's previous tile must be done: P_w is overwritten, O_w may be rescaled
-        if (!warp_wait(&o_done[w], (uint32_t)(i - 1) & 1u, args.err)) {
-          ok = false;
-          break;
+          for (int t = 0; t < 32; ++t) v[t] = c * 32 + t < kleft ? v[t] : -CUDART_INF_F;
         }
-        tc_fence_after();
+      };
+      float mx[8];  // eight independent max chains, then a tree
+#pragma unroll
+      for (int t = 0; t < 8; ++t) mx[t] = -CUDART_INF_F;
+#pragma unroll
+      for (int c = 0; c < kKT / 32; c += 2) {
+        float v0[32], v1[32];
+        tmem_ld32(tS + c * 32, v0);
+        tmem_ld32(tS + (c + 1) * 32, v1);
+        tmem_wait_ld();
+        mask32(v0, c);
+        mask32(v1, c + 1);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) mx[t & 7] = fmax3(mx[t & 7], v0[t], v1[t]);
       }
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                       sl2;
+      // The output MMA of this group's previous tile is complete: it was issued before
+      // the score MMA of this tile, and s_full[w] completes only once every MMA issued
+      // before its commit has.  So O_w may be rescaled and P_w overwritten here.
       if (mt != -CUDART_INF_F && (m_used == -CUDART_INF_F || mt > m_used + 8.f)) {
         const float alpha = m_used == -CUDART_INF_F ? 0.f : ex2_approx(m_used - mt);
         l *= alpha;
@@ -399,25 +484,41 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_used = mt;
       }
       const float nbase = m_used == -CUDART_INF_F ? 0.f : -m_used;
-      float ps = 0.f;
-      uint8_t* prow = smem + kPOff + w * kPBytes + r * 128;
+      uint64_t ps[4] = {0, 0, 0, 0};  // pairs of partial row sums (+0.f bits)
+      const uint64_t SL2 = f2_pack(sl2, sl2), NB = f2_pack(nbase, nbase);
+      // P over the first half of S_w: keys [32c, 32c + 32) into columns [16c, 16c + 16),
+      // whose scores were read in this or an earlier chunk.  Keys 6 and 7 of every 8
+      // take the FMA-pipe exponential.
+      float v[2][32];
+      tmem_ld32(tS, v[0]);
 #pragma unroll
-      for (int ch = 0; ch < kKT / 8; ++ch) {  // 8 chunks of 8 keys
-        float p[8];
+      for (int c = 0; c < kKT / 32; ++c) {
+        tmem_wait_ld();
+        if (c + 1 < kKT / 32) tmem_ld32(tS + (c + 1) * 32, v[(c + 1) & 1]);
+        float (&x)[32] = v[c & 1];
+        mask32(x, c);
+        uint32_t u[16];
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          p[t] = ex2_approx(fmaf(s[ch * 8 + t], sl2, nbase));
-          ps += p[t];
+        for (int t = 0; t < 32; t += 2) {
+          float x0, x1, p0, p1;
+          f2_unpack(f2_fma(f2_pack(x[t], x[t + 1]), SL2, NB), x0, x1);
+          if (kPolyPair(t)) {
+            exp2_fma2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          ps[(t >> 1) & 3] = f2_add(ps[(t >> 1) & 3], f2_pack(p0, p1));
+          u[t >> 1] = pack_bf16x2(p0, p1);
         }
-        uint4 u;
-        u.x = pack_bf16x2(p[0], p[1]);
-        u.y = pack_bf16x2(p[2], p[3]);
-        u.z = pack_bf16x2(p[4], p[5]);
-        u.w = pack_bf16x2(p[6], p[7]);
-        *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = u;
+        tmem_st16(tS + (uint32_t)(c * 16), u);
       }
-      l += ps;
-      fence_proxy_async_smem();  // P visible to the tensor core (async proxy)
+      {
+        float s0, s1;
+        f2_unpack(f2_add(f2_add(ps[0], ps[1]), f2_add(ps[2], ps[3])), s0, s1);
+        l += s0 + s1;
+      }
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[w]);
@@ -452,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < kD / 32; ++c) {
         float va[32], vb[32];
         if (has) tmem_ld32(tO + c * 32, va);
-        if (has_b) tmem_ld32(tmem + 128u + kD + lane_addr + c * 32, vb);
+        if (has_b) tmem_ld32(tmem + kOCol + kD + lane_addr + c * 32, vb);
         if (has || has_b) tmem_wait_ld();
         if (!mine) continue;
 #pragma unroll
@@ -525,7 +626,26 @@ cudaError_t launch_tc(const PassArgs& a, const CUtensorMap& tq, const CUtensorMa
   return cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, a);
 }
 
+// The pass's pairwise form on pairs (x[2i], x[2i + 1]); an odd last element alone.
+__global__ void exp2_fma_kernel(const float* x, float* y, long long n) {
+  const long long pairs = n / 2;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < pairs; i += (long long)gridDim.x * blockDim.x) {
+    float y0, y1;
+    exp2_fma2(x[2 * i], x[2 * i + 1], y0, y1);
+    y[2 * i] = y0;
+    y[2 * i + 1] = y1;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0 && (n & 1)) y[n - 1] = exp2_fma(x[n - 1]);
+}
+
 }  // namespace
+
+cudaError_t launch_exp2_fma(const float* x, float* y, long long n, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const long long blocks = std::min<long long>((n + 255) / 256, 148 * 8);
+  exp2_fma_kernel<<<(unsigned)blocks, 256, 0, s>>>(x, y, n);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_pass_tc(const PassArgs& a, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                            cudaStream_t s) {

@@ -16,7 +16,7 @@ import torch
 __all__ = [
     "FBError", "Shape", "Gate", "load", "lib_path", "make_shape", "make_gate", "FB_F32", "FB_BF16",
     "fb_version", "fb_status_string", "fb_device_error", "fb_workspace_bytes", "fb_workspace_init",
-    "fb_gate_eval", "fb_prefix_attn", "fb_prefix_attn_noalloc", "fb_block_attn", "fb_merge", "fb_merge_partials",
+    "fb_gate_eval", "fb_prefix_attn", "fb_prefix_attn_noalloc", "fb_block_attn", "fb_merge", "fb_merge_partials", "fb_exp2_fma",
     "fb_block_merge", "fb_step",
     "fb_page_minmax", "fb_append_block", "fb_similarity_workspace_bytes", "fb_head_similarity",
     "fb_refresh_reference", "fb_losa_step", "LosaLayer", "fb_sparse_workspace_bytes", "fb_sparse_select", "fb_sparse_step", "Sparse",
@@ -83,6 +83,7 @@ EXPORTED = {
     "fb_step": (_i, [_PS, _vp, _vp, _vp, _vp, _vp, _PG, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fb_prefix_attn_noalloc": (_i, [_PS, _vp, _vp, _vp, _PG, _vp, _vp, _vp]),
     "fb_merge_partials": (_i, [_PS, _vp, ctypes.c_int64, _vp, ctypes.c_int64, _i, _PG, _vp, _vp, _vp]),
+    "fb_exp2_fma": (_i, [_vp, _vp, ctypes.c_int64, _vp]),
     "fb_page_cap": (_i, [_PS, _i]),
     "fb_page_minmax": (_i, [_PS, _vp, _i, _vp, _vp, _vp]),
     "fb_append_block": (_i, [_PS, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp]),
@@ -218,6 +219,15 @@ def fb_merge_partials(shape, a_parts, a_part_stride, l_parts, l_part_stride, n_p
     _check("fb_merge_partials", load().fb_merge_partials(
         ctypes.byref(shape), _ptr_any(a_parts), int(a_part_stride), _ptr_any(l_parts), int(l_part_stride),
         int(n_parts), _gref(gate), _ptr(a_out), _ptr(l_out), _stream()))
+
+
+def fb_exp2_fma(x: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = 2^x elementwise (float32, on the device) in the FMA-pipe arithmetic of the tcgen05 pass."""
+    if x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous float32 tensor")
+    y = torch.empty_like(x) if y is None else y
+    _check("fb_exp2_fma", load().fb_exp2_fma(_ptr(x), _ptr(y), x.numel(), _stream()))
+    return y
 
 
 def fb_block_merge(shape, q, k_blk, v_blk, gate, a_out, l_out, a_full, l_full=None, dec_M=None, dec_reuse=None,

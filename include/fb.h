@@ -354,6 +354,17 @@ int fb_prefix_attn_noalloc(const fb_shape* shape, const void* q, const void* k_c
                            const void* v_cache, const fb_gate* gate, float* a_out, float* l_out,
                            fb_stream_t stream);
 
+/* Diagnostics: evaluates on the device, element by element, y[i] = 2^x[i] in the
+ * arithmetic the tcgen05 attention pass uses for a quarter of its softmax
+ * exponentials (those it keeps off the special-function unit): x = n + f with
+ * n = round(x), a cubic in f fitted for the least largest relative error on
+ * [-1/2, 1/2] with p(0) = 1, then n added to the exponent.  Relative error at
+ * most 1.02e-4 for x in [-125, 2^22); exact at integers; 0 for x < -125 and -inf.
+ * x and y are device arrays of n floats (they may alias; NULL when n == 0);
+ * n >= 0.  For tests of that error bound.  FB_ERR_NULL, FB_ERR_ALIGN (4-byte alignment), FB_ERR_SHAPE
+ * (n < 0 or n >= 2^31). */
+int fb_exp2_fma(const float* x, float* y, int64_t n, fb_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
