@@ -75,6 +75,9 @@ constexpr uint32_t kTmemCols = 512;
 // 0.52 of the burst tensor peak against 0.59 with none) -- the softmax is bound by
 // issue slots and latency, not by the special-function unit.
 __host__ __device__ constexpr bool kPolyPair(int) { return false; }
+// First TMEM column (within S_w) of the P of keys [32c, 32c + 32), c = 0..3: the
+// softmax writes each chunk over scores it has already read.
+__device__ constexpr uint32_t kPCol[4] = {112, 0, 16, 96};
 constexpr uint32_t kOCol = 256;                  // O_a at column 256, O_b at 384
 constexpr int kQBlock = 128 * 128;               // Q: [128 rows][128 B] per 64-column block
 constexpr int kQBytes = 2 * kQBlock;
@@ -399,9 +402,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t tP = tmem + (uint32_t)(w * kKT);
         const uint32_t tO = tmem + kOCol + (uint32_t)(w * kD);
 #pragma unroll
-        for (int kk = 0; kk < kKT / 16; ++kk)
-          umma_tmem_a(tO, tP + (uint32_t)(kk * 8), desc(b_lo + (uint32_t)(kk * (2048 >> 4)), desc_hi(1024)), kIdPV,
-                      (j >= 2 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kKT / 16; ++kk)  // keys [16kk, 16kk + 16): P where the softmax placed them
+          umma_tmem_a(tO, tP + kPCol[kk >> 1] + (uint32_t)(8 * (kk & 1)),
+                      desc(b_lo + (uint32_t)(kk * (2048 >> 4)), desc_hi(1024)), kIdPV, (j >= 2 || kk > 0) ? 1u : 0u);
         umma_commit(&v_empty[sl]);
         umma_commit(&o_done[w]);
         if (j + 2 < T) issue_qk(j + 2);  // after this group's output MMA, in issue order
@@ -436,9 +439,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       // Raw scores; the scale (> 0) is applied in the exponent.  Keys past the end
-      // of the range (only in its last tile) are masked.  S_w is read twice (for
-      // the max, then chunk by chunk for the exponentials), which keeps a row's
-      // registers to two 32-column chunks.
+      // of the range (only in its last tile) are masked.  The max reads all of S_w
+      // and keeps the last 32-key chunk in registers; the exponentials take it first,
+      // writing its P over columns already read, then read the other chunks again,
+      // each P chunk going to columns whose scores are consumed: P of keys [96, 128)
+      // in columns [96, 112), [0, 32) in [112, 128), [32, 64) in [0, 16) and
+      // [64, 96) in [16, 32).  The output MMA reads P in that placement (pcol).
       const long long kleft = key_end - key_begin - (long long)j * kKT;
       auto mask32 = [&](float (&v)[32], int c) {
         if (kleft < kKT) {
@@ -447,19 +453,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       };
       float mx[8];  // eight independent max chains, then a tree
+      float va[32], vb[32];
+      tmem_ld32(tS, va);
+      tmem_ld32(tS + 32, vb);
+      tmem_wait_ld();
+      mask32(va, 0);
+      mask32(vb, 1);
 #pragma unroll
-      for (int t = 0; t < 8; ++t) mx[t] = -CUDART_INF_F;
+      for (int t = 0; t < 8; ++t) mx[t] = fmaxf(va[t], vb[t]);
 #pragma unroll
-      for (int c = 0; c < kKT / 32; c += 2) {
-        float v0[32], v1[32];
-        tmem_ld32(tS + c * 32, v0);
-        tmem_ld32(tS + (c + 1) * 32, v1);
-        tmem_wait_ld();
-        mask32(v0, c);
-        mask32(v1, c + 1);
+      for (int t = 8; t < 32; ++t) mx[t & 7] = fmax3(mx[t & 7], va[t], vb[t]);
+      tmem_ld32(tS + 64, va);
+      tmem_ld32(tS + 96, vb);
+      tmem_wait_ld();
+      mask32(va, 2);
+      mask32(vb, 3);
 #pragma unroll
-        for (int t = 0; t < 32; ++t) mx[t & 7] = fmax3(mx[t & 7], v0[t], v1[t]);
-      }
+      for (int t = 0; t < 32; ++t) mx[t & 7] = fmax3(mx[t & 7], va[t], vb[t]);
       const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                              fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
                        sl2;
@@ -486,17 +496,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float nbase = m_used == -CUDART_INF_F ? 0.f : -m_used;
       uint64_t ps[4] = {0, 0, 0, 0};  // pairs of partial row sums (+0.f bits)
       const uint64_t SL2 = f2_pack(sl2, sl2), NB = f2_pack(nbase, nbase);
-      // P over the first half of S_w: keys [32c, 32c + 32) into columns [16c, 16c + 16),
-      // whose scores were read in this or an earlier chunk.  Keys 6 and 7 of every 8
-      // take the FMA-pipe exponential.
-      float v[2][32];
-      tmem_ld32(tS, v[0]);
-#pragma unroll
-      for (int c = 0; c < kKT / 32; ++c) {
-        tmem_wait_ld();
-        if (c + 1 < kKT / 32) tmem_ld32(tS + (c + 1) * 32, v[(c + 1) & 1]);
-        float (&x)[32] = v[c & 1];
-        mask32(x, c);
+      // One 32-key chunk: exponentials, row-sum pairs, P as bf16 pairs into 16 columns.
+      auto exp_chunk = [&](const float (&x)[32], uint32_t col) {
         uint32_t u[16];
 #pragma unroll
         for (int t = 0; t < 32; t += 2) {
@@ -511,8 +512,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           ps[(t >> 1) & 3] = f2_add(ps[(t >> 1) & 3], f2_pack(p0, p1));
           u[t >> 1] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(tS + (uint32_t)(c * 16), u);
-      }
+        tmem_st16(tS + col, u);
+      };
+      tmem_ld32(tS, va);  // chunk 0 again, under chunk 3
+      exp_chunk(vb, kPCol[3]);
+      tmem_wait_ld();
+      tmem_ld32(tS + 32, vb);  // chunk 1, under chunk 0
+      mask32(va, 0);
+      exp_chunk(va, kPCol[0]);
+      tmem_wait_ld();
+      tmem_ld32(tS + 64, va);  // chunk 2, under chunk 1
+      mask32(vb, 1);
+      exp_chunk(vb, kPCol[1]);
+      tmem_wait_ld();
+      mask32(va, 2);
+      exp_chunk(va, kPCol[2]);
       {
         float s0, s1;
         f2_unpack(f2_add(f2_add(ps[0], ps[1]), f2_add(ps[2], ps[3])), s0, s1);
