@@ -598,12 +598,14 @@ int sparse_layout(const Dims& d, int sms, SparseLayout* L) {
   return FB_OK;
 }
 
-// Pages the K cache's row capacity holds (the page stride of the bounds layout):
-// rows r with r * row_stride + D <= head_stride, at least N.
+// Pages the K cache's row capacity holds (rows r with r * row_stride + D <=
+// head_stride, at least N), rounded up to a multiple of 8: the page stride of the
+// bounds layout, so that every channel row of the bounds starts on 16 bytes.
 int page_capacity(const Dims& d) {
   long long rows = d.row_stride > 0 ? (d.head_stride - d.D) / d.row_stride + 1 : d.N;
   if (rows < d.N) rows = d.N;
-  return (int)((rows + kSparsePage - 1) / kSparsePage);
+  const long long pages = (rows + kSparsePage - 1) / kSparsePage;
+  return (int)((pages + 7) / 8 * 8);
 }
 
 int sparse_check(const fb_shape* shape, const fb_gate* gate, const fb_sparse* sp, Dims* d, GateParams* gp) {

@@ -144,106 +144,165 @@ __global__ void __launch_bounds__(32 * (D / 16)) page_minmax_kernel(const Sparse
 
 // ------------------------------------------------------------------ page estimates
 
-constexpr int kEstPages = 256;  // pages per CTA
-constexpr int kEstRowLanes = 2; // threads per page, each taking every other chunk of rows
-constexpr int kEstRows = 8;     // rows per chunk
-constexpr int kEstThreads = kEstPages * kEstRowLanes;
+constexpr int kEstVec = 2;      // consecutive pages per thread: one 4-byte load per bound row
+constexpr int kEstRows = 8;     // rows per thread
+constexpr int kEstAhead = 16;   // channels of bound loads in flight (a shared-memory ring per thread)
+constexpr int kEstThreads = 128;
+constexpr int kEstPages = kEstThreads * kEstVec;  // pages per CTA
+constexpr bool kEstSplitSign = true;  // q as (max(q, 0), min(q, 0)) pairs instead of a select
 
-// Page estimates of pages [p_lo, p_hi) of KV group bg for all R rows of the group,
-// by threads [0, NT); the group's q rows are in `sq` as float64 ([R rounded up to
-// 16][D]).  Two threads per page, 8 rows each per chunk; per row a float64 DFMA
-// chain in ascending d (each product exact), so the estimate is bit-identical to
-// the ordered sum.  The bounds of the next 8 channels are loaded while the current
-// 8 are consumed.
+// The rows to estimate (rows[0 .. n)) of KV group bg as float64 pairs
+// (max(q, 0), min(q, 0)), channel-major: sq2[2 (c Rp + k) + {0, 1}] for the k-th row;
+// rows n .. Rp are zero.  Every thread issues all its 16-byte loads (R <= 32 rows)
+// before it stores any of them, so their latencies overlap.
 template <int D, int NT>
-__device__ void estimate_pages(const SparseArgs& a, int bg, int p_lo, int p_hi, const double* sq, int tid,
-                               const int* rows, int nrows) {
+__device__ void load_group_q2(const SparseArgs& a, int bg, double* sq2, int Rp, const int* rows, int n, int tid) {
+  constexpr int kChunks = D / 8;                          // 16-byte chunks per row
+  constexpr int kPer = (32 * kChunks + NT - 1) / NT;      // chunks per thread at most
   const Dims& d = a.d;
-  const int R = nrows;  // rows[0 .. nrows) are the group rows to estimate
   const int b = bg / d.hkv, kvh = bg - b * d.hkv;
-  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B;
-  const int npg = p_hi - p_lo;
-  for (int it = tid; it < npg * kEstRowLanes; it += NT) {
-    const int p = p_lo + it % npg, rlane = it / npg;
-    const bf16* mn = a.kmin + (size_t)bg * D * a.Pcap + p;
-    const bf16* mx = a.kmax + (size_t)bg * D * a.Pcap + p;
-    for (int r0 = rlane * kEstRows; r0 < R; r0 += kEstRows * kEstRowLanes) {
-      double acc[kEstRows];
+  const bf16* qg = static_cast<const bf16*>(a.q) + (size_t)(b * d.hq + kvh * d.G) * d.B * D;
+  uint4 v[kPer];
 #pragma unroll
-      for (int j = 0; j < kEstRows; ++j) acc[j] = 0.0;
-      // Two register buffers (A, B) of 8 channels' bounds, ping-pong: the loads of
-      // the next 8 channels are in flight while the current 8 are consumed.
-      float an[8], ax[8], bn[8], bx[8];
-      auto load8 = [&](float (&n8)[8], float (&x8)[8], int c0) {
+  for (int j = 0; j < kPer; ++j) {
+    const int i = tid + j * NT;
+    v[j] = i < n * kChunks ? __ldg(reinterpret_cast<const uint4*>(qg + (size_t)rows[i / kChunks] * D) + i % kChunks)
+                           : make_uint4(0u, 0u, 0u, 0u);
+  }
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          n8[t] = __bfloat162float(__ldg(mn + (size_t)(c0 + t) * a.Pcap));
-          x8[t] = __bfloat162float(__ldg(mx + (size_t)(c0 + t) * a.Pcap));
-        }
-      };
-      auto use8 = [&](const float (&n8)[8], const float (&x8)[8], int c0) {
+  for (int j = 0; j < kPer; ++j) {
+    const int i = tid + j * NT;
+    if (i >= n * kChunks) break;
+    const int k = i / kChunks, c0 = (i % kChunks) * 8;
+    const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const double kmn = (double)n8[t], kmx = (double)x8[t];
-#pragma unroll
-          for (int j = 0; j < kEstRows; ++j) {
-            const double qv = sq[(size_t)rows[min(r0 + j, R - 1)] * D + c0 + t];
-            acc[j] = fma(qv, qv >= 0.0 ? kmx : kmn, acc[j]);  // exact product, one rounding
-          }
-        }
-      };
-      static_assert(D % 16 == 0, "channels in pairs of 8");
-      load8(an, ax, 0);
-#pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 16) {
-        load8(bn, bx, c0 + 8);
-        use8(an, ax, c0);
-        if (c0 + 16 < D) load8(an, ax, c0 + 16);
-        use8(bn, bx, c0 + 8);
-      }
-#pragma unroll
-      for (int j = 0; j < kEstRows; ++j)
-        if (r0 + j < R) a.est[(grow0 + rows[r0 + j]) * (size_t)a.P + p] = acc[j];
+    for (int e = 0; e < 8; ++e) {
+      const double q = (double)__uint_as_float(e & 1 ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+      double* dst = sq2 + 2 * ((size_t)(c0 + e) * Rp + k);
+      dst[0] = kEstSplitSign ? fmax(q, 0.0) : q;
+      dst[1] = kEstSplitSign ? fmin(q, 0.0) : q;
     }
+  }
+  for (int i = tid; i < (Rp - n) * D; i += NT) {  // padding rows
+    const int k = n + i / D, c = i % D;
+    sq2[2 * ((size_t)c * Rp + k)] = 0.0;
+    sq2[2 * ((size_t)c * Rp + k) + 1] = 0.0;
   }
 }
 
-// The q rows of KV group bg as float64 in shared memory (rows past R are zero).
-template <int D, int NT>
-__device__ void load_group_q(const SparseArgs& a, int bg, double* sq, int tid) {
-  const Dims& d = a.d;
-  const int R = d.R, Rp = (R + 15) / 16 * 16;
-  const int b = bg / d.hkv, kvh = bg - b * d.hkv;
-  const bf16* qg = static_cast<const bf16*>(a.q) + (size_t)(b * d.hq + kvh * d.G) * d.B * D;
-  for (int i = tid; i < Rp * D; i += NT) sq[i] = i < R * D ? (double)__bfloat162float(qg[i]) : 0.0;
-}
-
+// e for every (row, page) of recomputing batch elements: the bound of each channel
+// picked by the sign of q (max(q kmin, q kmax), exactly), summed in float64 in
+// ascending d.  With kEstSplitSign the pick is written without a select: q kmax is
+// added with max(q, 0) and q kmin with min(q, 0), one of which is a zero -- adding
+// q * 0 = +-0 leaves a sum unchanged (it is never -0: it starts at +0, and a rounded
+// sum is -0 only when both terms are), so every (row, page) chain rounds exactly as
+// the ordered sum of the picked products.  A thread owns 2 consecutive pages (one
+// 4-byte load per bound per channel, kEstAhead channels in flight) and 8 rows: 16
+// independent float64 chains, each bound widened to float64 once for 8 rows.
+// Grid: (page blocks, b * H_kv, chunks of 8 rows); a chunk past the rows to
+// estimate returns at once.
 template <int D>
 __global__ void __launch_bounds__(kEstThreads) page_estimate_kernel(const SparseArgs a) {
-  extern __shared__ double sq[];  // [R rounded up to 16][D] float64 copies of the group's q rows
+  extern __shared__ double sq2[];  // [D][rows rounded up to 8][2], then the bounds ring
   __shared__ int s_red[32];
+  __shared__ int s_rows[32];
+  __shared__ int s_nrows;
   const Dims& d = a.d;
-  const int bg = blockIdx.y, b = bg / d.hkv;
+  const int bg = blockIdx.y, b = bg / d.hkv, kvh = bg - b * d.hkv;
   if (!sparse_recompute(a.gate, b, d.B, s_red)) return;
   const int p0 = blockIdx.x * kEstPages;
   // The union of the group is rebuilt by the top-k: clear this chunk's words.
-  if (threadIdx.x < kEstPages / 32) {
+  if (blockIdx.z == 0 && threadIdx.x < kEstPages / 32) {
     const int w = p0 / 32 + threadIdx.x;
     if (w < a.words) a.union_bits[(size_t)bg * a.words + w] = 0u;
   }
-  // The group rows to estimate: all, or (LoSA) the rows of active tokens.
-  __shared__ int s_rows[1024];
-  __shared__ int s_nrows;
+  // The group rows to estimate: all, or (LoSA) the rows of active tokens (R <= 32).
   if (threadIdx.x == 0) {
     int n = 0;
-    for (int r = 0; r < d.R && r < 1024; ++r)
+    for (int r = 0; r < d.R; ++r)
       if (!a.active || a.active[(size_t)b * d.B + r % d.B]) s_rows[n++] = r;
     s_nrows = n;
   }
-  load_group_q<D, kEstThreads>(a, bg, sq, threadIdx.x);
   __syncthreads();
-  if (s_nrows > 0)
-    estimate_pages<D, kEstThreads>(a, bg, p0, min(a.P, p0 + kEstPages), sq, threadIdx.x, s_rows, s_nrows);
+  const int n = s_nrows;
+  if (n == 0) return;
+  const int Rp = (n + kEstRows - 1) / kEstRows * kEstRows;
+  load_group_q2<D, kEstThreads>(a, bg, sq2, Rp, s_rows, n, threadIdx.x);
+  __syncthreads();
+  const int pg = p0 + threadIdx.x * kEstVec;  // first of this thread's pages
+  if (pg >= a.P) return;
+  // Pcap is a multiple of 8 and pg of 2: 4-byte aligned, inside the allocation.
+  const uint32_t* mn = reinterpret_cast<const uint32_t*>(a.kmin + (size_t)bg * D * a.Pcap + pg);
+  const uint32_t* mx = reinterpret_cast<const uint32_t*>(a.kmax + (size_t)bg * D * a.Pcap + pg);
+  const size_t cstride = (size_t)a.Pcap / 2;  // words per channel row
+  const size_t grow0 = (size_t)(b * d.hq + kvh * d.G) * d.B;
+  auto widen = [](uint32_t u, double (&o)[kEstVec]) {
+    o[0] = (double)__uint_as_float(u << 16);
+    o[1] = (double)__uint_as_float(u & 0xFFFF0000u);
+  };
+  {
+    const int rc = blockIdx.z;  // this CTA's chunk of 8 rows
+    if (rc * kEstRows >= n) return;
+    double acc[kEstRows][kEstVec];
+#pragma unroll
+    for (int k = 0; k < kEstRows; ++k)
+#pragma unroll
+      for (int p = 0; p < kEstVec; ++p) acc[k][p] = 0.0;
+    // Bounds of the next kEstAhead channels in flight through cp.async into this
+    // thread's slots of the ring (a DRAM latency covers ~16 channels of work); a
+    // slot is refilled right after the thread has read it.
+    uint32_t* ring = reinterpret_cast<uint32_t*>(sq2 + 2 * (size_t)Rp * D);  // [kEstAhead][2][kEstThreads]
+    auto slot = [&](int c, int bound) { return ring + ((size_t)(c % kEstAhead) * 2 + bound) * kEstThreads + threadIdx.x; };
+#pragma unroll
+    for (int t = 0; t < kEstAhead; ++t) {
+      if (t < D) {
+        cp_async4(slot(t, 0), mn + t * cstride);
+        cp_async4(slot(t, 1), mx + t * cstride);
+      }
+      cp_async_commit();
+    }
+#pragma unroll 4
+    for (int c = 0; c < D; ++c) {
+      cp_async_wait_group<kEstAhead - 1>();  // channel c has landed
+      const uint32_t ln = *slot(c, 0), lx = *slot(c, 1);
+      double kn[kEstVec], kx[kEstVec];
+      widen(ln, kn);
+      widen(lx, kx);
+      if (c + kEstAhead < D) {
+        cp_async4(slot(c, 0), mn + (c + kEstAhead) * cstride);
+        cp_async4(slot(c, 1), mx + (c + kEstAhead) * cstride);
+      }
+      cp_async_commit();
+      const double2* qq = reinterpret_cast<const double2*>(sq2 + 2 * ((size_t)c * Rp + rc * kEstRows));
+      double2 q[kEstRows];
+#pragma unroll
+      for (int k = 0; k < kEstRows; ++k) q[k] = qq[k];
+      if (kEstSplitSign) {  // all the max(q, 0) terms, then all the min(q, 0) terms: independent FMAs apiece
+#pragma unroll
+        for (int k = 0; k < kEstRows; ++k)
+#pragma unroll
+          for (int p = 0; p < kEstVec; ++p) acc[k][p] = fma(q[k].x, kx[p], acc[k][p]);
+#pragma unroll
+        for (int k = 0; k < kEstRows; ++k)
+#pragma unroll
+          for (int p = 0; p < kEstVec; ++p) acc[k][p] = fma(q[k].y, kn[p], acc[k][p]);
+      } else {
+#pragma unroll
+        for (int k = 0; k < kEstRows; ++k)
+#pragma unroll
+          for (int p = 0; p < kEstVec; ++p) acc[k][p] = fma(q[k].x, q[k].x >= 0.0 ? kx[p] : kn[p], acc[k][p]);
+      }
+    }
+    cp_async_wait_all();
+#pragma unroll
+    for (int k = 0; k < kEstRows; ++k) {
+      if (rc * kEstRows + k >= n) break;
+      double* e = a.est + (grow0 + s_rows[rc * kEstRows + k]) * (size_t)a.P + pg;
+#pragma unroll
+      for (int p = 0; p < kEstVec; ++p)
+        if (pg + p < a.P) e[p] = acc[k][p];
+    }
+  }
 }
 
 // ------------------------------------------------------------------ top-k pages
@@ -331,9 +390,20 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
     if (tid == 0) s_unique = 0;
     __syncthreads();
     if (REG > 0) {
-      FB_FOR_MINE(t) {
-        const unsigned long long key = FB_KEY(t);
-        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      // When every lane's key of a warp falls in one bin (the leading bits of the
+      // estimates are nearly all equal), one atomic adds the warp's 32.
+      const int lane = tid & 31;
+#pragma unroll
+      for (int t = 0; t < (REG > 0 ? REG : 1); ++t) {
+        const unsigned long long key = kc.k[t];
+        const bool part = t < n && (key & mask) == prefix;
+        const unsigned bin = (unsigned)(key >> shift) & 255u;
+        const unsigned bin0 = __shfl_sync(0xffffffffu, bin, 0);
+        if (__all_sync(0xffffffffu, part && bin == bin0)) {
+          if (lane == 0) atomicAdd(&hist[bin], 32u);
+        } else if (part) {
+          atomicAdd(&hist[bin], 1u);
+        }
       }
     } else {
       for (int t = 0; t < n; ++t) {
@@ -411,11 +481,20 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
   int my_take = 0;
   {
     int r = eq_rank;
-    for (int t = 0; t < n; ++t) {
-      const unsigned long long key = REG > 0 ? desc_key(est[pb + t]) : FB_KEY(t);
-      const bool eq = key == T;
-      my_take += (key < T) || (eq && r < kk);
-      r += eq;
+    if (REG > 0) {
+      FB_FOR_MINE(t) {
+        const unsigned long long key = FB_KEY(t);
+        const bool eq = key == T;
+        my_take += (key < T) || (eq && r < kk);
+        r += eq;
+      }
+    } else {
+      for (int t = 0; t < n; ++t) {
+        const unsigned long long key = FB_KEY(t);
+        const bool eq = key == T;
+        my_take += (key < T) || (eq && r < kk);
+        r += eq;
+      }
     }
   }
   int pos = block_exclusive_scan(my_take, s_tmp);
@@ -424,15 +503,19 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
   {
     int r = eq_rank;
     int32_t* out = a.sel_idx + (size_t)row * a.k_sel;
-    for (int t = 0; t < n; ++t) {
+    auto take = [&](int t, unsigned long long key) {
       const int p = pb + t;
-      const unsigned long long key = desc_key(est[p]);
       const bool eq = key == T;
       if ((key < T) || (eq && r < kk)) {
         out[pos++] = p;
         atomicOr(&s_bits[p >> 5], 1u << (p & 31));
       }
       r += eq;
+    };
+    if (REG > 0) {
+      FB_FOR_MINE(t) take(t, FB_KEY(t));
+    } else {
+      for (int t = 0; t < n; ++t) take(t, FB_KEY(t));
     }
   }
 #undef FB_KEY
@@ -1271,8 +1354,9 @@ cudaError_t launch_page_minmax(const SparseArgs& a, cudaStream_t s) {
 }
 
 cudaError_t launch_sparse_select(const SparseArgs& a, cudaStream_t s) {
-  const size_t est_smem = (size_t)((a.d.R + 15) / 16 * 16) * a.d.D * sizeof(double);
-  dim3 g1((a.P + kEstPages - 1) / kEstPages, a.d.b * a.d.hkv);
+  const size_t est_smem = (size_t)((a.d.R + kEstRows - 1) / kEstRows * kEstRows) * a.d.D * 2 * sizeof(double) +
+                          (size_t)kEstAhead * 2 * kEstThreads * sizeof(uint32_t);
+  dim3 g1((a.P + kEstPages - 1) / kEstPages, a.d.b * a.d.hkv, (a.d.R + kEstRows - 1) / kEstRows);
   cudaError_t e;
   if (a.d.D == 128) {
     e = cudaFuncSetAttribute(page_estimate_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)est_smem);

@@ -216,7 +216,8 @@ typedef struct fb_sparse {
   int32_t n_select;       /* pages per query row, 1 .. n_pages */
   const void* kmin;       /* [b, H_kv, D, page_cap] bf16 page minima (fb_page_minmax), pages
                              [0, n_pages) valid; page_cap (fb_page_cap) = ceil(cap / page_size)
-                             with cap the K cache's row capacity per head (rows r with
+                             rounded up to a multiple of 8 (16-byte channel rows), with cap
+                             the K cache's row capacity per head (rows r with
                              r * kv_row_stride + head_dim <= kv_head_stride; = n_prefix for a
                              contiguous cache), so the layout survives fb_append_block */
   const void* kmax;       /* same layout, page maxima */
@@ -230,7 +231,8 @@ typedef struct fb_sparse {
 } fb_sparse;
 
 /* The page stride page_cap of the bounds layout (see fb_sparse.kmin) for this
- * shape: > 0, or a negative fb_status (bad shape, page_size != 16, n_prefix < 1).
+ * shape: > 0 and a multiple of 8, or a negative fb_status (bad shape,
+ * page_size != 16, n_prefix < 1).
  * Host only; allocate kmin / kmax as [b, H_kv, D, page_cap] bf16. */
 int fb_page_cap(const fb_shape* shape, int page_size);
 

@@ -123,8 +123,9 @@ def test_workspace_bytes_for_valid_and_invalid_shapes(lib):
     assert big >= n
 
 
-@pytest.mark.parametrize("n,cap,want", [
-    (1, None, 1), (16, None, 1), (17, None, 2), (65536, None, 4096), (65536, 65552, 4097), (1000, 2000, 125),
+@pytest.mark.parametrize("n,cap,want", [   # ceil(capacity / 16) rounded up to a multiple of 8
+    (1, None, 8), (16, None, 8), (17, None, 8), (65536, None, 4096), (65536, 65552, 4104), (1000, 2000, 128),
+    (2000, None, 128), (2048, None, 128), (2049, None, 136),
 ])
 def test_page_cap_is_the_pages_of_the_cache_capacity(lib, n, cap, want):
     kw = dict(n_prefix=n) if cap is None else dict(n_prefix=n, kv_head_stride=cap * 128)

@@ -72,7 +72,7 @@ def test_append_block_refreshes_touched_page_bounds(fb, N, B):
     kd, vd = k.cuda(), v.cuda()
     sh = fb.make_shape(b, 4 * hkv, hkv, D, B, N, "bf16", kv_head_stride=cap * D)
     page_cap = fb.fb_page_cap(sh)
-    assert page_cap == (cap + 15) // 16
+    assert page_cap == ((cap + 15) // 16 + 7) // 8 * 8
     kmin = torch.full((b, hkv, D, page_cap), 5.0, dtype=torch.bfloat16, device="cuda")
     kmax = kmin.clone()
     fb.fb_page_minmax(sh, kd, 16, kmin, kmax)
