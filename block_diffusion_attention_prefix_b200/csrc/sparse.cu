@@ -359,6 +359,7 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
   __shared__ unsigned hist[256];
   __shared__ int s_tmp[32];
   __shared__ unsigned long long s_prefix, s_key;
+  __shared__ unsigned long long s_kand[kTopkThreads / 32], s_kor[kTopkThreads / 32];
   __shared__ int s_kk, s_unique;
   const Dims& d = a.d;
   const int row = blockIdx.x;
@@ -384,7 +385,43 @@ __global__ void __launch_bounds__(kTopkThreads) topk_kernel(const SparseArgs a) 
   // then the k-th smallest itself.
   unsigned long long prefix = 0, mask = 0;
   int kk = a.k_sel;
-  for (int pass = 0; pass < 8; ++pass) {
+  int first_pass = 0;
+  if (REG > 0) {
+    // Whole leading bytes that every key shares (the estimates mostly share sign and
+    // exponent) would each cost a pass whose histogram has one bin: start past them.
+    unsigned long long kand = ~0ull, kor = 0ull;
+    FB_FOR_MINE(t) {
+      kand &= FB_KEY(t);
+      kor |= FB_KEY(t);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      kand &= __shfl_xor_sync(0xffffffffu, kand, o);
+      kor |= __shfl_xor_sync(0xffffffffu, kor, o);
+    }
+    if ((tid & 31) == 0) {
+      s_kand[tid >> 5] = kand;
+      s_kor[tid >> 5] = kor;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      unsigned long long ba = ~0ull, bo = 0ull;
+      for (int w = 0; w < kTopkThreads / 32; ++w) {
+        ba &= s_kand[w];
+        bo |= s_kor[w];
+      }
+      s_kand[0] = ba;
+      s_kor[0] = bo;
+    }
+    __syncthreads();
+    const unsigned long long diff = s_kand[0] ^ s_kor[0];
+    first_pass = diff ? __clzll((long long)diff) / 8 : 8;
+    if (first_pass > 0) {
+      mask = first_pass >= 8 ? ~0ull : ~0ull << (64 - 8 * first_pass);
+      prefix = s_kand[0] & mask;
+    }
+  }
+  for (int pass = first_pass; pass < 8; ++pass) {
     const int shift = 56 - 8 * pass;
     if (tid < 256) hist[tid] = 0u;
     if (tid == 0) s_unique = 0;
