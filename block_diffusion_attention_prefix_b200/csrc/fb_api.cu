@@ -733,7 +733,15 @@ extern "C" int fb_losa_step(const fb_shape* shape, const void* q, const void* q_
   FB_TRY(encode_kv_map(&tv, v_cache, d.D, d.N, d.row_stride, d.head_stride, d.b * d.hkv, kSparsePage));
   FB_TRY(encode_kv_map(&tk4, k_cache, d.D, d.N, d.row_stride, d.head_stride, d.b * d.hkv, 4 * kSparsePage));
   FB_TRY(encode_kv_map(&tv4, v_cache, d.D, d.N, d.row_stride, d.head_stride, d.b * d.hkv, 4 * kSparsePage));
-  FB_TRY(cuda_status(launch_token_mse(d, q, q_prev, delta, mse, dec_active, (cudaStream_t)stream)));
+  if (losa_score_in_estimate(d)) {
+    // the page estimate scores the tokens itself (one launch fewer)
+    a.q_prev = q_prev;
+    a.delta = delta;
+    a.mse = mse;
+    a.active_out = dec_active;
+  } else {
+    FB_TRY(cuda_status(launch_token_mse(d, q, q_prev, delta, mse, dec_active, (cudaStream_t)stream)));
+  }
   FB_TRY(cuda_status(launch_sparse_select(a, (cudaStream_t)stream)));
   return cuda_status(launch_sparse_pass(a, tk, tv, tk4, tv4, (cudaStream_t)stream));
 }

@@ -123,6 +123,12 @@ struct SparseArgs {
   uint32_t* union_bits;   // [b*H_kv][words]
   GateParams gate;        // tau only
   const uint8_t* active;  // LoSA mode: token activity [b, B] (NULL otherwise)
+  // LoSA mode with the locality score taken inside the page estimate (q_prev != NULL):
+  // each estimate CTA scores its batch element's tokens, one CTA writes mse / active.
+  const void* q_prev;     // [b, H_q, B, D] bf16, the previous step's queries
+  float delta;            // activity threshold
+  float* mse;             // optional output [b, B]
+  uint8_t* active_out;    // output [b, B] (the same buffer as `active`)
   float* a_res;           // residual cache [b, H_q, B, D] / [b, H_q, B]
   float* l_res;
   float* a_sel;           // optional
@@ -137,6 +143,7 @@ struct SparseArgs {
 int sparse_supported(int D, int row_tile);
 cudaError_t launch_page_minmax(const SparseArgs& a, cudaStream_t s);
 // LoSA: per-token locality score (float32 [b, B], nullable) and activity (score > delta).
+bool losa_score_in_estimate(const Dims& d);  // the page estimate can score the LoSA tokens itself
 cudaError_t launch_token_mse(const Dims& d, const void* q, const void* q_prev, float delta, float* mse,
                              uint8_t* active, cudaStream_t s);
 cudaError_t launch_sparse_select(const SparseArgs& a, cudaStream_t s);

@@ -63,45 +63,57 @@ __device__ __forceinline__ bool sparse_recompute(const GateParams& g, int b, int
 // then a rounded sum (no fused multiply-add: the products are not exact); thread 0
 // adds the heads in ascending order and divides by H_q * D.  Reading L1 of the LoSA
 // page ("2. Methodology": MSE between the queries of steps t and t - 1).
+// Sum over d (ascending) of (q - q_prev)^2 for one (batch element, head, token) row of D
+// channels, in float64, each term a rounded product then a rounded sum.
+__device__ __forceinline__ double head_sq_diff(const bf16* q, const bf16* qp, size_t off, int D) {
+  const uint4* qv = reinterpret_cast<const uint4*>(q + off);
+  const uint4* pv = reinterpret_cast<const uint4*>(qp + off);
+  double acc = 0.0;
+  for (int c0 = 0; c0 < D / 8; c0 += 8) {  // 64 channels' loads in flight, then their terms in order
+    uint4 xa[8], xb[8];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      xa[c] = c0 + c < D / 8 ? __ldg(qv + c0 + c) : make_uint4(0, 0, 0, 0);
+      xb[c] = c0 + c < D / 8 ? __ldg(pv + c0 + c) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      if (c0 + c >= D / 8) break;
+      const bf16* ea = reinterpret_cast<const bf16*>(&xa[c]);
+      const bf16* eb = reinterpret_cast<const bf16*>(&xb[c]);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const double diff = __dsub_rn((double)__bfloat162float(ea[e]), (double)__bfloat162float(eb[e]));
+        acc = __dadd_rn(acc, __dmul_rn(diff, diff));
+      }
+    }
+  }
+  return acc;
+}
+
+// The token's score from its heads' sums (ascending h), divided by H_q * D.
+__device__ __forceinline__ float token_score(const double* head_sums, int hq, int D) {
+  double tot = 0.0;
+  for (int h = 0; h < hq; ++h) tot = __dadd_rn(tot, head_sums[h]);
+  return (float)__ddiv_rn(tot, (double)hq * D);
+}
+
 __global__ void token_mse_kernel(const Dims d, const bf16* q, const bf16* qp, float delta, float* mse,
                                  uint8_t* active) {
   extern __shared__ double s_head[];
   const int i = blockIdx.x, b = blockIdx.y;
-  for (int h = threadIdx.x; h < d.hq; h += blockDim.x) {
-    const size_t off = (((size_t)b * d.hq + h) * d.B + i) * d.D;
-    const uint4* qv = reinterpret_cast<const uint4*>(q + off);
-    const uint4* pv = reinterpret_cast<const uint4*>(qp + off);
-    double acc = 0.0;
-    for (int c0 = 0; c0 < d.D / 8; c0 += 8) {  // 64 channels' loads in flight, then their terms in order
-      uint4 xa[8], xb[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        xa[c] = c0 + c < d.D / 8 ? __ldg(qv + c0 + c) : make_uint4(0, 0, 0, 0);
-        xb[c] = c0 + c < d.D / 8 ? __ldg(pv + c0 + c) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        if (c0 + c >= d.D / 8) break;
-        const bf16* ea = reinterpret_cast<const bf16*>(&xa[c]);
-        const bf16* eb = reinterpret_cast<const bf16*>(&xb[c]);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const double diff = __dsub_rn((double)__bfloat162float(ea[e]), (double)__bfloat162float(eb[e]));
-          acc = __dadd_rn(acc, __dmul_rn(diff, diff));
-        }
-      }
-    }
-    s_head[h] = acc;
-  }
+  for (int h = threadIdx.x; h < d.hq; h += blockDim.x)
+    s_head[h] = head_sq_diff(q, qp, (((size_t)b * d.hq + h) * d.B + i) * d.D, d.D);
   __syncthreads();
   if (threadIdx.x == 0) {
-    double tot = 0.0;
-    for (int h = 0; h < d.hq; ++h) tot = __dadd_rn(tot, s_head[h]);
-    const float m = (float)__ddiv_rn(tot, (double)d.hq * d.D);
+    const float m = token_score(s_head, d.hq, d.D);
     if (mse) mse[(size_t)b * d.B + i] = m;
     active[(size_t)b * d.B + i] = m > delta ? 1 : 0;
   }
 }
+
+// Largest number of (token, head) sums the page estimate keeps to score the tokens itself.
+constexpr int kEstScoreMax = 2048;
 
 // ------------------------------------------------------------------ page bounds
 
@@ -216,11 +228,35 @@ __global__ void __launch_bounds__(kEstThreads) page_estimate_kernel(const Sparse
     const int w = p0 / 32 + threadIdx.x;
     if (w < a.words) a.union_bits[(size_t)bg * a.words + w] = 0u;
   }
+  // LoSA with the score taken here: every CTA scores its batch element's B tokens
+  // (the same float64 arithmetic as token_mse_kernel, so every CTA agrees), and one
+  // CTA per batch element writes the scores and activity for the launches after it.
+  __shared__ uint8_t s_act[kSmallBlockMax];
+  __shared__ double s_hsum[kEstScoreMax];
+  const bool own_score = a.q_prev != nullptr;
+  if (own_score) {
+    const bf16* q = static_cast<const bf16*>(a.q);
+    const bf16* qp = static_cast<const bf16*>(a.q_prev);
+    for (int t = threadIdx.x; t < d.B * d.hq; t += kEstThreads) {
+      const int i = t / d.hq, h = t - i * d.hq;
+      s_hsum[t] = head_sq_diff(q, qp, (((size_t)b * d.hq + h) * d.B + i) * d.D, d.D);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < d.B; i += kEstThreads) {
+      const float m = token_score(s_hsum + (size_t)i * d.hq, d.hq, d.D);
+      s_act[i] = m > a.delta ? 1 : 0;
+      if (blockIdx.x == 0 && kvh == 0 && blockIdx.z == 0) {
+        if (a.mse) a.mse[(size_t)b * d.B + i] = m;
+        a.active_out[(size_t)b * d.B + i] = s_act[i];
+      }
+    }
+    __syncthreads();
+  }
   // The group rows to estimate: all, or (LoSA) the rows of active tokens (R <= 32).
   if (threadIdx.x == 0) {
     int n = 0;
     for (int r = 0; r < d.R; ++r)
-      if (!a.active || a.active[(size_t)b * d.B + r % d.B]) s_rows[n++] = r;
+      if (own_score ? s_act[r % d.B] != 0 : (!a.active || a.active[(size_t)b * d.B + r % d.B])) s_rows[n++] = r;
     s_nrows = n;
   }
   __syncthreads();
@@ -1367,6 +1403,8 @@ cudaError_t launch_sparse_cfg(const SparseArgs& a, const CUtensorMap& tk, const 
 }
 
 }  // namespace
+
+bool losa_score_in_estimate(const Dims& d) { return d.B * d.hq <= kEstScoreMax && d.B <= kSmallBlockMax; }
 
 int sparse_supported(int D, int row_tile) { return (D == 64 || D == 128) && (row_tile == 16 || row_tile == 32); }
 
