@@ -33,15 +33,16 @@
 //              which is why the key tile is 128 wide.
 //   warps 2-5, 6-9  softmax warpgroups a and b, one query row per thread (TMEM
 //              lane = row): read S_w with tcgen05.ld, online softmax in base 2, and
-//              P_w as bf16 pairs written back over the first half of S_w's columns
-//              (tcgen05.st), where the output MMA reads it; the next score MMA of
-//              the group is issued after that output MMA, and MMAs of one thread
-//              run in issue order.  A quarter of the exponentials run on the FMA
-//              pipe (exp2_fma), the rest on the special-function unit.  O_w is
-//              rescaled in TMEM only when a row's max grows by more than 2^8
-//              (otherwise the stale max is kept; p <= 2^8 is exact enough in bf16
-//              and cannot overflow fp32).  At the end group a merges the two
-//              partial results (the FlashBlock log-space merge).
+//              P_w as bf16 pairs written back (tcgen05.st) over 64 of S_w's columns
+//              whose scores have been read, where the output MMA reads it; the next
+//              score MMA of the group is issued after that output MMA, and MMAs of
+//              one thread run in issue order.  The exponentials run on the
+//              special-function unit (kPolyPair can route pairs to the FMA pipe,
+//              exp2_fma2; measured slower here).  O_w is rescaled in TMEM only when
+//              a row's max grows by more than 2^8 (otherwise the stale max is kept;
+//              p <= 2^8 is exact enough in bf16 and cannot overflow fp32).  At the
+//              end group a merges the two partial results (the FlashBlock log-space
+//              merge).
 //   warp 10    fused step: this split's share of the tile's in-block rows.
 // TMEM: 512 columns (S_a / P_a [0,128), S_b / P_b [128,256), O_a [256,384),
 // O_b [384,512)).  Every mbarrier wait is time bounded; on expiry the roles fall
